@@ -1,0 +1,426 @@
+"""Benchmark of the xKV hot path on B200.
+
+One step = one decode step of Selective-Reconstruction attention over every
+layer of the model for the whole batch (32 layers x batch 4 at 64K context for
+the Llama-3.1-8B shape), captured in one CUDA graph: per layer the library
+scores landmarks, selects the top-k chunks, rebuilds the selected K/V rows from
+the shared basis and attends.  Metric: decode tokens/s (batch / step time) and
+the HBM bandwidth implied by the step's algorithmic bytes.
+
+The compressed caches are produced on the GPU by the library itself before
+timing (synthetic K/V -> xkv_compress_group -> xkv_build_landmarks); that
+prefill work is timed separately and reported under "prefill".
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+    python bench.py --impl reference ...   # the CPU oracle, bounded sample
+
+Multi-GPU (torchrun): every rank runs its own batch (independent sequences, no
+data-path collective: "scaling": "weak"); the step time is the maximum over
+ranks of the device-timed region.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "SR-attn decode tokens/s & HBM GB/s (% of peak), Llama-8B shape, 64K ctx"
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), float(d.get("bf16_tflops_sustained", d["bf16_tflops"])), "measured"
+    return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+def sr_bytes_per_unit(w) -> int:
+    """Algorithmic HBM bytes of one (batch, layer, KV head) SR decode unit."""
+    el = 2 if w.dtype == "bf16" else 4
+    n_mid = w.n_mid
+    return (n_mid * w.head_dim * el                                  # landmarks
+            + w.topk * w.chunk * (w.rank_k + w.rank_v) * el          # selected A slabs
+            + (w.rank_k + w.rank_v) * w.head_dim * el                # Bt slices
+            + (w.sink + w.recent) * w.head_dim * 2 * el              # raw sink/recent K and V
+            + 2 * w.gq * w.head_dim * el)                            # queries in, outputs out
+
+
+def sr_flops_per_unit(w) -> int:
+    rows = w.topk * w.chunk
+    return (2 * rows * w.rank_k * w.head_dim                 # K rebuild
+            + 2 * w.gq * w.n_mid * w.head_dim                # landmark scores
+            + 4 * w.gq * (rows + w.sink + w.recent) * w.head_dim
+            + 2 * w.gq * rows * w.rank_v + 2 * w.gq * w.rank_v * w.head_dim)
+
+
+class Clocks:
+    """nvidia-smi sampling during the timed region."""
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{index}.csv")
+
+    def __enter__(self):
+        os.makedirs(os.path.dirname(self.path), exist_ok=True)
+        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={q}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"], stdout=self.f,
+                                         stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        try:
+            rows = [l.strip().split(",") for l in open(self.path) if l.strip()]
+        except Exception:
+            rows = []
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            try:
+                sm.append(float(r[1]))
+                mx = float(r[2])
+                for nm, v in zip(names, r[5:9]):
+                    if v.strip().lower() == "active":
+                        reasons.add(nm)
+            except (ValueError, IndexError):
+                continue
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ----------------------------------------------------------------- set-up
+def build_model(xkv, w, device, groups=None, log=print):
+    """Compressed caches of every layer: A_K/A_V per group, Bt per layer,
+    landmarks and raw sink/recent rows per layer, q per layer."""
+    import torch
+    bf = torch.bfloat16
+    G, d, T, B = w.group, w.d, w.T, w.batch
+    n_groups = groups or w.n_groups
+    sw_rows = torch.tensor(list(range(w.sink)) + list(range(T - w.recent, T)), device=device)
+    model = {"A_K": [], "A_V": [], "Bt_K": [], "Bt_V": [], "lm": [], "srK": [], "srV": [], "q": []}
+    ws_bytes = xkv.xkv_compress_workspace_size(G, T, d, w.rank_k, synth.oversample(w.rank_k), 8192, bf)
+    ws_bytes = max(ws_bytes, xkv.xkv_compress_workspace_size(G, T, d, w.rank_v, synth.oversample(w.rank_v), 8192, bf))
+    ws = xkv.workspace(ws_bytes, device)
+    prefill = {"compress_ms": [], "landmarks_ms": []}
+    for g in range(n_groups):
+        AK = torch.empty((B, T, w.rank_k), dtype=bf, device=device)
+        AV = torch.empty((B, T, w.rank_v), dtype=bf, device=device)
+        BtK = torch.empty((G * d, w.rank_k), dtype=bf, device=device)
+        BtV = torch.empty((G * d, w.rank_v), dtype=bf, device=device)
+        lms = [torch.empty((B, w.n_kv_heads, w.n_mid, w.head_dim), dtype=bf, device=device) for _ in range(G)]
+        srK = [torch.empty((B, w.sink + w.recent, d), dtype=bf, device=device) for _ in range(G)]
+        srV = [torch.empty((B, w.sink + w.recent, d), dtype=bf, device=device) for _ in range(G)]
+        for b in range(B):
+            for kind, A, Bt, r in (("K", AK, BtK, w.rank_k), ("V", AV, BtV, w.rank_v)):
+                X = synth.kv_group_torch(w, b, g, kind, device)
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record()
+                # the basis of each batch element is its own; Bt of batch 0 is kept
+                # (every batch element shares the layer weights' geometry here)
+                Bt_b = Bt if b == 0 else torch.empty_like(Bt)
+                xkv.xkv_compress_group(X, r, A[b], Bt_b, iters=8, oversample=synth.oversample(r), shard_rows=8192,
+                                       ws=ws)
+                e1.record()
+                e1.synchronize()
+                prefill["compress_ms"].append(e0.elapsed_time(e1))
+                for l in range(G):
+                    if kind == "K":
+                        e0.record()
+                        xkv.xkv_build_landmarks(X[l], w.n_kv_heads, w.head_dim, w.chunk, w.sink, w.recent,
+                                                w.rope_theta, lms[l][b])
+                        e1.record()
+                        e1.synchronize()
+                        prefill["landmarks_ms"].append(e0.elapsed_time(e1))
+                        srK[l][b].copy_(X[l].index_select(0, sw_rows))
+                    else:
+                        srV[l][b].copy_(X[l].index_select(0, sw_rows))
+                del X
+        for l in range(G):
+            model["A_K"].append(AK)
+            model["A_V"].append(AV)
+            model["Bt_K"].append(BtK[l * d:(l + 1) * d])
+            model["Bt_V"].append(BtV[l * d:(l + 1) * d])
+            model["lm"].append(lms[l])
+            model["srK"].append(srK[l])
+            model["srV"].append(srV[l])
+        log(f"group {g + 1}/{n_groups} compressed")
+    for layer in range(n_groups * G):
+        q = synth.normal_torch(synth.stream_key(w.name, "q", layer), B * w.n_q_heads * w.head_dim, device)
+        model["q"].append(q.view(B, w.n_q_heads, w.head_dim).to(bf))
+    return model, prefill
+
+
+def measure_gram(xkv, w, device):
+    """Device time of the Gram of one (batch 0, group 0) K shard set (T rows)."""
+    import torch
+    X = synth.kv_group_torch(w, 0, 0, "K", device)
+    n = w.group * w.d
+    C = torch.zeros((n, n), dtype=torch.float32, device=device)
+    ws = xkv.workspace(xkv.xkv_gram_workspace_size(w.group, 8192, w.d, torch.bfloat16), device)
+    for _ in range(2):
+        for s in range(0, w.T, 8192):
+            xkv.xkv_gram_accumulate([x[s:s + 8192] for x in X], C, ws)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    reps = 3
+    e0.record()
+    for _ in range(reps):
+        for s in range(0, w.T, 8192):
+            xkv.xkv_gram_accumulate([x[s:s + 8192] for x in X], C, ws)
+    e1.record()
+    e1.synchronize()
+    ms = e0.elapsed_time(e1) / reps
+    flops = n * (n + 1) * w.T  # unique entries of the symmetric product, 2 T flops each
+    return ms, flops
+
+
+# ------------------------------------------------------------------- arms
+def run_cuda(args, rank, world, log):
+    import torch
+    import torch.distributed as dist
+    import cross_layer_rank_b200 as xkv
+
+    device = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    torch.cuda.set_device(device)
+    w = synth.WORKLOADS[args.workload]
+    if args.batch:
+        w = w.replace(batch=args.batch)
+    n_groups = args.groups or w.n_groups
+    L = n_groups * w.group
+    bf = torch.bfloat16
+    model, prefill = build_model(xkv, w, device, n_groups, log)
+    gram_ms, gram_flops = measure_gram(xkv, w, device) if args.prefill else (None, None)
+
+    p = xkv.sr_params(w.batch, w.n_q_heads, w.n_kv_heads, w.head_dim, w.T, w.rank_k, w.rank_v, w.chunk, w.topk,
+                      w.sink, w.recent, w.rope_theta, bf)
+    ws = xkv.workspace(xkv.xkv_sr_workspace_size(p), device)
+    outs = [torch.empty((w.batch, w.n_q_heads, w.head_dim), dtype=torch.float32, device=device) for _ in range(L)]
+    stream = torch.cuda.Stream(device)
+
+    def layer_call(l, st):
+        xkv.xkv_sr_attention_decode(p, model["q"][l], model["A_K"][l], model["Bt_K"][l], model["A_V"][l],
+                                    model["Bt_V"][l], model["lm"][l], model["srK"][l], model["srV"][l], outs[l],
+                                    None, ws, st)
+
+    # warm-up (also loads the kernels) then capture one step in a CUDA graph
+    with torch.cuda.stream(stream):
+        for l in range(L):
+            layer_call(l, stream)
+    stream.synchronize()
+    assert xkv.get_device_status(stream) == 0
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        for l in range(L):
+            layer_call(l, stream)
+    # one graph per single layer for the per-call roofline timing
+    g1 = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g1, stream=stream):
+        layer_call(0, stream)
+    for _ in range(args.warmup):
+        graph.replay()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+
+    with Clocks(device.index) as clk:
+        with torch.cuda.stream(stream):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            torch.cuda.synchronize()
+            e0.record(stream)
+            for _ in range(args.steps):
+                graph.replay()
+            e1.record(stream)
+            e1.synchronize()
+        ms_total = e0.elapsed_time(e1)
+        # per-call timing of the dominant call (one layer of SR decode), live
+        with torch.cuda.stream(stream):
+            ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(20)]
+            for a, b_ in ev:
+                a.record(stream)
+                g1.replay()
+                b_.record(stream)
+            torch.cuda.synchronize()
+        call_ms = statistics.median(a.elapsed_time(b_) for a, b_ in ev)
+        # end to end: per step, pinned-host queries in, outputs out, around the same graph
+        q_host = [model["q"][l].cpu().pin_memory() for l in range(L)]
+        o_host = [torch.empty_like(outs[l], device="cpu").pin_memory() for l in range(L)]
+        with torch.cuda.stream(stream):
+            e2, e3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            torch.cuda.synchronize()
+            e2.record(stream)
+            for _ in range(args.steps):
+                for l in range(L):
+                    model["q"][l].copy_(q_host[l], non_blocking=True)
+                graph.replay()
+                for l in range(L):
+                    o_host[l].copy_(outs[l], non_blocking=True)
+            e3.record(stream)
+            e3.synchronize()
+        e2e_ms = e2.elapsed_time(e3)
+    assert xkv.get_device_status(stream) == 0
+    clocks = clk.summary()
+
+    if world > 1:
+        t = torch.tensor([ms_total, e2e_ms], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_total, e2e_ms = float(t[0]), float(t[1])
+    ms_step = ms_total / args.steps
+    tokens = w.batch * world
+    value = tokens / (ms_step / 1e3)
+    units_step = w.batch * L * w.n_kv_heads
+    bytes_step = sr_bytes_per_unit(w) * units_step
+    hbm_gbs_peak, bf16_peak, _, peak_kind = _peaks()
+    achieved_step = bytes_step / (ms_step / 1e3) / 1e9
+    bytes_call = sr_bytes_per_unit(w) * w.batch * w.n_kv_heads
+    achieved_call = bytes_call / (call_ms / 1e3) / 1e9
+    traffic = None
+    tp = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(tp):
+        try:
+            traffic = json.load(open(tp)).get(args.workload)
+        except Exception:
+            traffic = None
+    q_bytes = sum(t.numel() * t.element_size() for t in model["q"])
+    o_bytes = sum(t.numel() * t.element_size() for t in outs)
+    res = {
+        "metric": METRIC, "value": round(value, 2), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": args.workload, "global_batch": tokens, "seq_len": w.T, "layers": L,
+                   "kv_heads": w.n_kv_heads, "q_heads": w.n_q_heads, "head_dim": w.head_dim,
+                   "rank_k": w.rank_k, "rank_v": w.rank_v, "topk": w.topk, "chunk": w.chunk, "sink": w.sink,
+                   "recent": w.recent, "parallelism": f"dp{world}",
+                   "l2": "inputs larger than L2 (%.1f GB touched per step)" % (bytes_step / 1e9)},
+        "hbm_gbs": round(achieved_step, 1),
+        "hbm_frac_of_peak": round(achieved_step / hbm_gbs_peak, 4),
+        "roofline": {"bound": "hbm", "kernel": "xkv_sr_attention_decode (one layer: score, top-k, attend, combine)",
+                     "achieved": round(achieved_call, 1), "peak": hbm_gbs_peak, "unit": "GB/s",
+                     "frac": round(achieved_call / hbm_gbs_peak, 4), "traffic": traffic,
+                     "peak_source": f"{peak_kind} hbm_gbs", "bytes_per_launch": bytes_call,
+                     "launch_ms": round(call_ms, 5)},
+        "e2e": {"value": round(tokens / (e2e_ms / args.steps / 1e3), 2), "unit": "tokens/s",
+                "h2d_bytes_per_step": q_bytes, "d2h_bytes_per_step": o_bytes},
+        "gpu_launches": 4 * L * args.steps,
+        "clocks": clocks,
+        "flops_per_step": sr_flops_per_unit(w) * units_step,
+    }
+    if args.prefill:
+        cm = prefill["compress_ms"]
+        res["prefill"] = {"compress_group_ms_median": round(statistics.median(cm), 3), "groups_compressed": len(cm),
+                          "landmarks_ms_median": round(statistics.median(prefill["landmarks_ms"]), 4),
+                          "gram_ms": round(gram_ms, 4),
+                          "gram_tflops": round(gram_flops / (gram_ms / 1e3) / 1e12, 1),
+                          "gram_frac_of_bf16_peak": round(gram_flops / (gram_ms / 1e3) / 1e12 / bf16_peak, 4)}
+    return res, w
+
+
+def cpu_baseline(w, budget_s: float, log):
+    """The oracle (fp64 C, OpenMP) on a bounded sample of the same decode step."""
+    import oracle
+    wb = w.replace(batch=1)
+    inp = synth.compressed_cache(wb, 0)
+    units_per_layer = wb.n_kv_heads
+    t0 = time.time()
+    done = 0
+    while time.time() - t0 < budget_s and done < 64:
+        oracle.sr_decode(wb, units=list(range(units_per_layer)), **inp)
+        done += units_per_layer
+    dt = time.time() - t0
+    units_step = w.batch * w.n_layers * w.n_kv_heads
+    step_s = dt / done * units_step
+    return {"value": round(w.batch / step_s, 4), "unit": "tokens/s", "cores": oracle.num_threads(),
+            "kind": "oracle",
+            "sample": f"{done} (layer, KV-head) units of one decode step (batch 1, T={w.T}), oracle SR decode in "
+                      f"fp64, scaled to the full {w.n_layers}-layer batch-{w.batch} step ({units_step} units)"}
+
+
+def run_reference(args, log):
+    w = synth.WORKLOADS[args.workload]
+    if args.batch:
+        w = w.replace(batch=args.batch)
+    import oracle
+    oracle.build()
+    budget = max(2.0, min(20.0, 60.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        cpu_baseline(w, budget / 4, log)
+    vals = [cpu_baseline(w, budget, log) for _ in range(args.steps)]
+    v = statistics.median(x["value"] for x in vals)
+    cb = dict(vals[0])
+    cb["value"] = v
+    return {"impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(w.batch / v * 1e3, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": args.workload, "global_batch": w.batch, "seq_len": w.T, "layers": w.n_layers},
+            "cpu_baseline": cb, "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                                        "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
+    ap.add_argument("--workload", default="llama8b_64k_b4", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--batch", type=int, default=0, help="override the batch per GPU")
+    ap.add_argument("--groups", type=int, default=0, help="build only this many layer groups")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-prefill", dest="prefill", action="store_false")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    args = ap.parse_args()
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    log = (lambda *a: print(*a, file=sys.stderr, flush=True)) if rank == 0 else (lambda *a: None)
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args, log)), flush=True)
+        return
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", 0)))
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600))
+    res, w = run_cuda(args, rank, world, log)
+    if rank == 0 and not args.no_cpu_baseline and world == 1:
+        res["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds, log)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,268 @@
+"""B200 (sm_100a) xKV hot path: thin Python binding of libxkv.so.
+
+Every call below marshals torch tensors into the C ABI declared in
+include/xkv.h and returns; all arithmetic runs in the library's CUDA kernels.
+There is no CPU or PyTorch fallback: importing this package fails loudly when
+libxkv.so has not been built (``python cross_layer_rank_b200/build.py``).
+
+Functions keep the C names (xkv_compress_group, xkv_build_landmarks,
+xkv_sr_attention_decode, xkv_full_reconstruct, xkv_ner, ...).  Tensors must be
+CUDA tensors, contiguous, of the dtype named by the call; errors raise
+XKVError carrying the library's status code.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+from typing import Optional, Sequence
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libxkv.so")
+
+XKV_OK = 0
+XKV_ERR_INVALID_ARG = 1
+XKV_ERR_UNSUPPORTED = 2
+XKV_ERR_WORKSPACE = 3
+XKV_ERR_CUDA = 4
+XKV_ERR_NUMERICAL = 5
+XKV_ERR_DEVICE_TIMEOUT = 6
+XKV_F32 = 0
+XKV_BF16 = 1
+
+EXPORTS = (
+    "xkv_status_string", "xkv_version", "xkv_get_device_status",
+    "xkv_gram_workspace_size", "xkv_gram_accumulate",
+    "xkv_compress_workspace_size", "xkv_compress_group",
+    "xkv_build_landmarks",
+    "xkv_sr_workspace_size", "xkv_sr_attention_decode",
+    "xkv_full_reconstruct",
+    "xkv_dense_workspace_size", "xkv_dense_attention_decode",
+    "xkv_ner_workspace_size", "xkv_ner",
+)
+
+
+class XKVError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = int(status)
+        super().__init__(f"{where}: {status_string(status)} (status {status})")
+
+
+class SRParams(C.Structure):
+    """Mirror of xkv_sr_params."""
+    _fields_ = [("batch", C.c_int), ("n_q_heads", C.c_int), ("n_kv_heads", C.c_int), ("head_dim", C.c_int),
+                ("T", C.c_int64), ("rank_k", C.c_int), ("rank_v", C.c_int), ("chunk", C.c_int),
+                ("topk", C.c_int), ("sink", C.c_int), ("recent", C.c_int), ("rope_theta", C.c_float),
+                ("dtype", C.c_int), ("a_k_batch_stride", C.c_int64), ("a_v_batch_stride", C.c_int64),
+                ("bt_k_batch_stride", C.c_int64), ("bt_v_batch_stride", C.c_int64)]
+
+
+class DenseParams(C.Structure):
+    """Mirror of xkv_dense_params."""
+    _fields_ = [("batch", C.c_int), ("n_q_heads", C.c_int), ("n_kv_heads", C.c_int), ("head_dim", C.c_int),
+                ("T", C.c_int64), ("dtype", C.c_int)]
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"libxkv.so not built ({LIB_PATH}); run `python cross_layer_rank_b200/build.py`")
+    lib = C.CDLL(LIB_PATH)
+    vp, i64, sz = C.c_void_p, C.c_int64, C.c_size_t
+    sig = {
+        "xkv_status_string": (C.c_char_p, [C.c_int]),
+        "xkv_version": (C.c_int, []),
+        "xkv_get_device_status": (C.c_int, [vp]),
+        "xkv_gram_workspace_size": (C.c_int, [C.c_int, i64, C.c_int, C.c_int, C.POINTER(sz)]),
+        "xkv_gram_accumulate": (C.c_int, [vp, C.c_int, i64, C.c_int, i64, C.c_int, vp, vp, sz, vp]),
+        "xkv_compress_workspace_size": (C.c_int, [C.c_int, i64, C.c_int, C.c_int, C.c_int, i64, C.c_int,
+                                                  C.POINTER(sz)]),
+        "xkv_compress_group": (C.c_int, [vp, C.c_int, i64, C.c_int, i64, C.c_int, C.c_int, C.c_int, C.c_int, i64,
+                                         C.c_uint64, vp, vp, vp, vp, vp, sz, vp]),
+        "xkv_build_landmarks": (C.c_int, [vp, i64, i64, C.c_int, C.c_int, C.c_int, C.c_int, C.c_int, C.c_int,
+                                          C.c_float, vp, vp]),
+        "xkv_sr_workspace_size": (C.c_int, [C.POINTER(SRParams), C.POINTER(sz)]),
+        "xkv_sr_attention_decode": (C.c_int, [C.POINTER(SRParams), vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz,
+                                              vp]),
+        "xkv_full_reconstruct": (C.c_int, [vp, vp, i64, C.c_int, C.c_int, C.c_int, C.c_int, C.c_int, C.c_float,
+                                           C.c_int, vp, vp]),
+        "xkv_dense_workspace_size": (C.c_int, [C.POINTER(DenseParams), C.POINTER(sz)]),
+        "xkv_dense_attention_decode": (C.c_int, [C.POINTER(DenseParams), vp, vp, vp, vp, vp, sz, vp]),
+        "xkv_ner_workspace_size": (C.c_int, [C.c_int, C.c_int, C.POINTER(sz)]),
+        "xkv_ner": (C.c_int, [vp, C.c_int, C.c_int, C.c_double, vp, vp, vp, vp, sz, vp]),
+    }
+    for name, (res, args) in sig.items():
+        f = getattr(lib, name)
+        f.restype = res
+        f.argtypes = args
+    return lib
+
+
+lib = _load()
+
+
+def status_string(status: int) -> str:
+    return lib.xkv_status_string(int(status)).decode()
+
+
+def _check(status: int, where: str):
+    if status != XKV_OK:
+        raise XKVError(status, where)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("expected a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError("expected a contiguous tensor")
+    return C.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> C.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return C.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def dtype_code(t: torch.dtype) -> int:
+    if t == torch.bfloat16:
+        return XKV_BF16
+    if t == torch.float32:
+        return XKV_F32
+    raise ValueError(f"unsupported dtype {t}")
+
+
+def workspace(nbytes: int, device=None) -> torch.Tensor:
+    """Caller-owned scratch (256-byte aligned, as torch's allocator guarantees)."""
+    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device or "cuda")
+
+
+def _wsize(fn, *args) -> int:
+    n = C.c_size_t(0)
+    _check(fn(*args, C.byref(n)), fn.__name__)
+    return int(n.value)
+
+
+def get_device_status(stream=None) -> int:
+    """Deferred device-side status (synchronises the stream), cleared on read."""
+    return int(lib.xkv_get_device_status(_stream(stream)))
+
+
+# ------------------------------------------------------------------- Gram
+def xkv_gram_workspace_size(G: int, rows: int, d: int, dtype: torch.dtype) -> int:
+    return _wsize(lib.xkv_gram_workspace_size, G, rows, d, dtype_code(dtype))
+
+
+def xkv_gram_accumulate(layers: Sequence[torch.Tensor], C_out: torch.Tensor, ws: Optional[torch.Tensor] = None,
+                        stream=None):
+    """C_out += X^T X over X = [layers...] (each rows x d)."""
+    G = len(layers)
+    rows, d = layers[0].shape
+    ldx = layers[0].stride(0)
+    ptrs = (C.c_void_p * G)(*[t.data_ptr() for t in layers])
+    nbytes = xkv_gram_workspace_size(G, rows, d, layers[0].dtype)
+    ws = ws if ws is not None else workspace(nbytes, layers[0].device)
+    _check(lib.xkv_gram_accumulate(ptrs, G, rows, d, ldx, dtype_code(layers[0].dtype), _ptr(C_out), _ptr(ws),
+                                   ws.numel(), _stream(stream)), "xkv_gram_accumulate")
+
+
+# ------------------------------------------------------------ compression
+def xkv_compress_workspace_size(G, T, d, rank, oversample, shard_rows, dtype: torch.dtype) -> int:
+    return _wsize(lib.xkv_compress_workspace_size, G, T, d, rank, oversample, shard_rows, dtype_code(dtype))
+
+
+def xkv_compress_group(layers: Sequence[torch.Tensor], rank: int, A: torch.Tensor, Bt: torch.Tensor,
+                       iters: int = 8, oversample: int = 64, shard_rows: int = 8192, seed: int = 0x784B56,
+                       eigvals: Optional[torch.Tensor] = None, gram_out: Optional[torch.Tensor] = None,
+                       ws: Optional[torch.Tensor] = None, stream=None):
+    """Cross-layer factorisation of one group into A (T x rank) and Bt (G d x rank)."""
+    G = len(layers)
+    T, d = layers[0].shape
+    ldx = layers[0].stride(0)
+    for t in layers:
+        if t.shape != layers[0].shape or t.stride(0) != ldx or t.stride(1) != 1:
+            raise ValueError("layers must share shape and row stride")
+    dt = dtype_code(layers[0].dtype)
+    nbytes = xkv_compress_workspace_size(G, T, d, rank, oversample, shard_rows, layers[0].dtype)
+    ws = ws if ws is not None else workspace(nbytes, layers[0].device)
+    ptrs = (C.c_void_p * G)(*[t.data_ptr() for t in layers])
+    _check(lib.xkv_compress_group(ptrs, G, T, d, ldx, dt, rank, iters, oversample, shard_rows, seed, _ptr(A),
+                                  _ptr(Bt), _ptr(eigvals), _ptr(gram_out), _ptr(ws), ws.numel(), _stream(stream)),
+           "xkv_compress_group")
+
+
+# -------------------------------------------------------------- landmarks
+def xkv_build_landmarks(K: torch.Tensor, n_kv_heads: int, head_dim: int, chunk: int, sink: int, recent: int,
+                        rope_theta: float, out: torch.Tensor, stream=None):
+    T = K.shape[0]
+    if K.stride(1) != 1:
+        raise ValueError("K rows must be contiguous")
+    _check(lib.xkv_build_landmarks(C.c_void_p(K.data_ptr()), T, K.stride(0), n_kv_heads, head_dim,
+                                   dtype_code(K.dtype), chunk, sink, recent, rope_theta, _ptr(out), _stream(stream)),
+           "xkv_build_landmarks")
+
+
+# -------------------------------------------------------------- SR decode
+def sr_params(batch, n_q_heads, n_kv_heads, head_dim, T, rank_k, rank_v, chunk, topk, sink, recent, rope_theta,
+              dtype: torch.dtype, a_k_batch_stride=None, a_v_batch_stride=None, bt_k_batch_stride=None,
+              bt_v_batch_stride=None) -> SRParams:
+    """Batch strides default to dense [B][T][r] A and per-batch dense [B][d][r] Bt."""
+    d = n_kv_heads * head_dim
+    return SRParams(batch, n_q_heads, n_kv_heads, head_dim, T, rank_k, rank_v, chunk, topk, sink, recent,
+                    float(rope_theta), dtype_code(dtype),
+                    T * rank_k if a_k_batch_stride is None else a_k_batch_stride,
+                    T * rank_v if a_v_batch_stride is None else a_v_batch_stride,
+                    d * rank_k if bt_k_batch_stride is None else bt_k_batch_stride,
+                    d * rank_v if bt_v_batch_stride is None else bt_v_batch_stride)
+
+
+def xkv_sr_workspace_size(p: SRParams) -> int:
+    return _wsize(lib.xkv_sr_workspace_size, C.byref(p))
+
+
+def xkv_sr_attention_decode(p: SRParams, q, A_K, Bt_K, A_V, Bt_V, landmarks, sr_K, sr_V, out,
+                            sel_out=None, ws=None, stream=None):
+    """One SR decode step of one layer; writes out [B][Hq][hd] f32 (and sel_out)."""
+    ws = ws if ws is not None else workspace(xkv_sr_workspace_size(p), q.device)
+    _check(lib.xkv_sr_attention_decode(C.byref(p), _ptr(q), _ptr(A_K), _ptr(Bt_K), _ptr(A_V), _ptr(Bt_V),
+                                       _ptr(landmarks), _ptr(sr_K), _ptr(sr_V), _ptr(out), _ptr(sel_out), _ptr(ws),
+                                       ws.numel(), _stream(stream)), "xkv_sr_attention_decode")
+
+
+# --------------------------------------------------- full reconstruction
+def xkv_full_reconstruct(A, Bt, n_kv_heads: int, head_dim: int, apply_rope: bool, rope_theta: float, out,
+                         stream=None):
+    T, r = A.shape
+    d = Bt.shape[0]
+    _check(lib.xkv_full_reconstruct(_ptr(A), _ptr(Bt), T, r, d, n_kv_heads, head_dim, int(bool(apply_rope)),
+                                    float(rope_theta), dtype_code(A.dtype), _ptr(out), _stream(stream)),
+           "xkv_full_reconstruct")
+
+
+def dense_params(batch, n_q_heads, n_kv_heads, head_dim, T, dtype: torch.dtype) -> DenseParams:
+    return DenseParams(batch, n_q_heads, n_kv_heads, head_dim, T, dtype_code(dtype))
+
+
+def xkv_dense_workspace_size(p: DenseParams) -> int:
+    return _wsize(lib.xkv_dense_workspace_size, C.byref(p))
+
+
+def xkv_dense_attention_decode(p: DenseParams, q, K, V, out, ws=None, stream=None):
+    ws = ws if ws is not None else workspace(xkv_dense_workspace_size(p), q.device)
+    _check(lib.xkv_dense_attention_decode(C.byref(p), _ptr(q), _ptr(K), _ptr(V), _ptr(out), _ptr(ws), ws.numel(),
+                                          _stream(stream)), "xkv_dense_attention_decode")
+
+
+# -------------------------------------------------------------------- NER
+def xkv_ner_workspace_size(n: int, block: int) -> int:
+    return _wsize(lib.xkv_ner_workspace_size, n, block)
+
+
+def xkv_ner(gram: torch.Tensor, block: int, ner_out, erank_out=None, rank_out=None, rank_rel_tol: float = 1e-9,
+            ws=None, stream=None):
+    n = gram.shape[0]
+    ws = ws if ws is not None else workspace(xkv_ner_workspace_size(n, block), gram.device)
+    _check(lib.xkv_ner(_ptr(gram), n, block, rank_rel_tol, _ptr(ner_out), _ptr(erank_out), _ptr(rank_out), _ptr(ws),
+                       ws.numel(), _stream(stream)), "xkv_ner")

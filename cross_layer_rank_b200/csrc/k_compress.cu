@@ -1,0 +1,419 @@
+// Prefill-time cross-layer factorisation of one group of G layers (xKV
+// explainer, "xKV 到底做了什么"; xKV abstract) with the incremental covariance
+// of KV-CoRE (2.A):
+//   1. C = sum over token shards of X_s^T X_s, X = [X_1 | ... | X_G] read through
+//      the G layer pointers (never concatenated).  bf16: each shard is
+//      transposed to a K-major copy and multiplied on tcgen05 tensor cores,
+//      upper-triangular 128 x 128 tiles with a mirrored fp32 epilogue.
+//   2. top-r subspace: block subspace iteration Y = C Q, Q = qr(Y) (shifted
+//      Cholesky QR, two passes, fp64 small factors), started from a Gaussian
+//      block (Philox4x32-10 + Box-Muller on the device);
+//      Rayleigh-Ritz: H = Q^T C Q, eigenpairs of H by one-sided block Jacobi,
+//      V_r = Q U[:, top r].
+//   3. A = X V_r: tcgen05 GEMM over the layer tensor maps with V_r split into a
+//      bf16 hi/lo pair (two MMAs per step keep ~16 significant bits of V_r);
+//      Bt = V_r stored in the cache dtype (layer l owns rows l d .. l d + d - 1).
+#include <algorithm>
+
+#include "k_gemm_tc.cuh"
+#include "xkv_common.cuh"
+#include "xkv_internal.h"
+#include "xkv_linalg.cuh"
+
+namespace xkv {
+namespace {
+
+// X_s (rows x d per layer, row stride ldx) -> Xt (n x ldt), Xt[l d + c][t] = X_l[t][c].
+struct LayerPtrs {
+  const void* p[8];
+};
+
+__global__ void __launch_bounds__(256) transpose_layers_kernel(const LayerPtrs X, int d, int64_t ldx, int64_t rows,
+                                                               __nv_bfloat16* __restrict__ Xt, int64_t ldt) {
+  __shared__ __nv_bfloat16 tile[64][66];
+  const int l = blockIdx.z;
+  const int64_t t0 = static_cast<int64_t>(blockIdx.x) * 64;
+  const int c0 = blockIdx.y * 64;
+  const __nv_bfloat16* src = static_cast<const __nv_bfloat16*>(X.p[l]);
+  for (int i = threadIdx.x; i < 64 * 64; i += 256) {
+    const int r = i / 64, c = i % 64;
+    const int64_t t = t0 + r;
+    tile[r][c] = t < rows ? src[t * ldx + c0 + c] : __float2bfloat16_rn(0.f);
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < 64 * 64; i += 256) {
+    const int c = i / 64, r = i % 64;
+    const int64_t t = t0 + r;
+    if (t < ldt) Xt[static_cast<int64_t>(l * d + c0 + c) * ldt + t] = tile[r][c];
+  }
+}
+
+// Philox4x32-10 (Salmon et al., SC'11) keyed by the seed; Box-Muller pairs.
+__device__ __forceinline__ void philox10(uint32_t c[4], uint32_t k0, uint32_t k1) {
+#pragma unroll
+  for (int r = 0; r < 10; ++r) {
+    const uint64_t p0 = static_cast<uint64_t>(0xD2511F53u) * c[0];
+    const uint64_t p1 = static_cast<uint64_t>(0xCD9E8D57u) * c[2];
+    const uint32_t n0 = static_cast<uint32_t>(p1 >> 32) ^ c[1] ^ k0;
+    const uint32_t n2 = static_cast<uint32_t>(p0 >> 32) ^ c[3] ^ k1;
+    c[1] = static_cast<uint32_t>(p1);
+    c[3] = static_cast<uint32_t>(p0);
+    c[0] = n0;
+    c[2] = n2;
+    k0 += 0x9E3779B9u;
+    k1 += 0xBB67AE85u;
+  }
+}
+
+__global__ void gaussian_kernel(float* __restrict__ out, int64_t count, uint64_t seed) {
+  for (int64_t blk = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; blk * 4 < count;
+       blk += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    uint32_t c[4] = {static_cast<uint32_t>(blk), static_cast<uint32_t>(blk >> 32), 0u, 0u};
+    philox10(c, static_cast<uint32_t>(seed), static_cast<uint32_t>(seed >> 32));
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const float u1 = (static_cast<float>(c[2 * h] >> 8) + 0.5f) * (1.0f / 16777216.0f);
+      const float u2 = (static_cast<float>(c[2 * h + 1] >> 8) + 0.5f) * (1.0f / 16777216.0f);
+      const float rad = sqrtf(-2.0f * logf(u1));
+      float s, co;
+      sincospif(2.0f * u2, &s, &co);
+      const int64_t e = blk * 4 + 2 * h;
+      if (e < count) out[e] = rad * co;
+      if (e + 1 < count) out[e + 1] = rad * s;
+    }
+  }
+}
+
+// Ur[k][i] = U[order[i]][k]  (U column-major b x b: column c at U + c b)
+__global__ void gather_ritz_kernel(const double* __restrict__ U, const int* __restrict__ order, int b, int r,
+                                   float* __restrict__ Ur, const double* __restrict__ lam, float* __restrict__ eig) {
+  const int64_t total = static_cast<int64_t>(b) * r;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int k = static_cast<int>(i / r), c = static_cast<int>(i % r);
+    Ur[i] = static_cast<float>(U[static_cast<int64_t>(order[c]) * b + k]);
+  }
+  if (eig && blockIdx.x == 0)
+    for (int c = threadIdx.x; c < r; c += blockDim.x) eig[c] = static_cast<float>(lam[order[c]]);
+}
+
+// Bt (n x r, dtype) = Vr; Vt hi/lo (r x n bf16) = transposed split of Vr.
+template <typename T>
+__global__ void emit_factors_kernel(const float* __restrict__ Vr, int n, int r, T* __restrict__ Bt,
+                                    __nv_bfloat16* __restrict__ vhi, __nv_bfloat16* __restrict__ vlo) {
+  const int64_t total = static_cast<int64_t>(n) * r;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const float v = Vr[i];
+    store_f(Bt + i, v);
+    if (vhi) {
+      const int k = static_cast<int>(i / r), c = static_cast<int>(i % r);
+      const __nv_bfloat16 h = __float2bfloat16_rn(v);
+      vhi[static_cast<int64_t>(c) * n + k] = h;
+      vlo[static_cast<int64_t>(c) * n + k] = __float2bfloat16_rn(v - __bfloat162float(h));
+    }
+  }
+}
+
+// Gram tile C[tm-block][tn-block] += X_s^T X_s (upper-triangular tile list),
+// operands from the K-major transposed shard Xt.  The tensor cores accumulate
+// only kGramChunk rows into a TMEM buffer (two buffers, double-buffered); the
+// epilogue warps add each chunk's tile into fp32 registers with IEEE adds.
+// Keeping the in-MMA accumulation chain short (8 MMAs of 16 rows) removes the
+// drift a long chain of tensor-core accumulations shows over thousands of
+// rows; the outer sum is an ordinary round-to-nearest fp32 chain.
+constexpr int kGramChunkStages = 2;  // 2 x 64 rows per TMEM chunk
+constexpr int kGramStages = 4;
+constexpr int kGramThreads = 192;
+
+inline size_t gram_tc_smem() { return 1024 + kGramStages * 2 * 16384 + (2 * kGramStages + 4) * 8 + 16; }
+
+__global__ void __launch_bounds__(kGramThreads, 1)
+    gram_tc_kernel(const __grid_constant__ CUtensorMap xmap, int nk, int tiles_n, float* __restrict__ C, int64_t ldc,
+                   int* status) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kGramStages * 2 * 16384);
+  uint64_t* empty = full + kGramStages;
+  uint64_t* accfull = empty + kGramStages;
+  uint64_t* accempty = accfull + 2;
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(accempty + 2);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  int idx = blockIdx.x, tm = 0, len = tiles_n;
+  while (idx >= len) { idx -= len; ++tm; --len; }
+  const int tn = tm + idx;
+  const int m0 = tm * 128, n0 = tn * 128;
+  const int nchunks = (nk + kGramChunkStages - 1) / kGramChunkStages;
+  if (tid == 0) {
+    for (int i = 0; i < kGramStages; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
+    for (int i = 0; i < 2; ++i) { mbar_init(&accfull[i], 1); mbar_init(&accempty[i], 128); }
+    fence_mbar_init();
+  }
+  if (warp == 1) tmem_alloc(tslot, 256);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tslot;
+  if (warp == 0) {
+    if (lane == 0) {
+      for (int a = 0; a < nk; ++a) {
+        const int slot = a % kGramStages;
+        if (!mbar_wait(&empty[slot], ((a / kGramStages) & 1) ^ 1, status)) break;
+        uint8_t* st = smem + slot * 2 * 16384;
+        mbar_arrive_expect_tx(&full[slot], 2 * 16384);
+        tma_load_2d(st, &xmap, &full[slot], a * 64, m0);
+        tma_load_2d(st + 16384, &xmap, &full[slot], a * 64, n0);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idesc = umma_idesc_bf16(128, 128);
+      int a = 0;
+      bool ok = true;
+      for (int c = 0; c < nchunks && ok; ++c) {
+        const int buf = c & 1;
+        if (!mbar_wait(&accempty[buf], ((c >> 1) & 1) ^ 1, status)) break;
+        tc_fence_after();
+        for (int s = 0; s < kGramChunkStages && a < nk; ++s, ++a) {
+          const int slot = a % kGramStages;
+          if (!mbar_wait(&full[slot], (a / kGramStages) & 1, status)) { ok = false; break; }
+          tc_fence_after();
+          uint8_t* st = smem + slot * 2 * 16384;
+          const uint64_t ad = umma_desc_sw128(smem_u32(st));
+          const uint64_t bd = umma_desc_sw128(smem_u32(st + 16384));
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            umma_bf16(tmem + buf * 128, ad + 2 * kk, bd + 2 * kk, idesc, (s | kk) ? 1u : 0u);
+          umma_commit(&empty[slot]);
+        }
+        umma_commit(&accfull[buf]);
+      }
+    }
+  } else {
+    const int lq = warp & 3;
+    const int row = lq * 32 + lane;
+    const uint32_t tbase = tmem + (static_cast<uint32_t>(lq * 32) << 16);
+    float acc[128];
+#pragma unroll
+    for (int i = 0; i < 128; ++i) acc[i] = 0.f;
+    bool ok = true;
+    for (int c = 0; c < nchunks; ++c) {
+      const int buf = c & 1;
+      if (!mbar_wait(&accfull[buf], (c >> 1) & 1, status)) { ok = false; break; }
+      tc_fence_after();
+#pragma unroll
+      for (int jb = 0; jb < 8; ++jb) {
+        float v[16];
+        tmem_ld16(tbase + buf * 128 + jb * 16, v);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) acc[jb * 16 + i] += v[i];
+      }
+      tc_fence_before();
+      mbar_arrive(&accempty[buf]);
+    }
+    if (ok) {
+      const int m = m0 + row;
+      float* crow = C + static_cast<int64_t>(m) * ldc + n0;
+#pragma unroll
+      for (int i = 0; i < 128; i += 4) {
+        float4 cv = *reinterpret_cast<float4*>(crow + i);
+        cv.x += acc[i]; cv.y += acc[i + 1]; cv.z += acc[i + 2]; cv.w += acc[i + 3];
+        *reinterpret_cast<float4*>(crow + i) = cv;
+      }
+      if (tm != tn) {
+#pragma unroll
+        for (int i = 0; i < 128; ++i) C[static_cast<int64_t>(n0 + i) * ldc + m] += acc[i];
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 256);
+  }
+}
+
+bool gram_tc_ok(int G, int d, xkv_dtype dt) { return dt == XKV_BF16 && (G * d) % 128 == 0 && !force_simt(); }
+
+}  // namespace
+
+size_t gram_workspace(int G, int64_t rows, int d, xkv_dtype dt) {
+  if (!gram_tc_ok(G, d, dt)) return kAlign;
+  const int64_t ldt = (rows + 7) / 8 * 8;
+  return align_up(static_cast<size_t>(G) * d * ldt * 2);
+}
+
+xkv_status gram_launch(const void* const* X, int G, int64_t rows, int d, int64_t ldx, xkv_dtype dt, float* C,
+                       void* ws, cudaStream_t st) {
+  const int n = G * d;
+  if (rows <= 0) return XKV_OK;
+  if (gram_tc_ok(G, d, dt)) {
+    const int64_t ldt = (rows + 7) / 8 * 8;
+    __nv_bfloat16* Xt = static_cast<__nv_bfloat16*>(ws);
+    LayerPtrs lp;
+    for (int l = 0; l < 8; ++l) lp.p[l] = l < G ? X[l] : nullptr;
+    dim3 tg(static_cast<unsigned>((ldt + 63) / 64), d / 64, G);
+    transpose_layers_kernel<<<tg, 256, 0, st>>>(lp, d, ldx, rows, Xt, ldt);
+    CUtensorMap xm;
+    const uint64_t dims[2] = {static_cast<uint64_t>(rows), static_cast<uint64_t>(n)};
+    const uint64_t str[1] = {static_cast<uint64_t>(ldt) * 2};
+    const uint32_t box[2] = {64, 128};
+    if (!make_tmap(&xm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, Xt, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B))
+      return XKV_ERR_CUDA;
+    const int tiles_n = n / 128;
+    const int nk = static_cast<int>((rows + 63) / 64);
+    const size_t smem = gram_tc_smem();
+    cudaFuncSetAttribute(gram_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    gram_tc_kernel<<<tiles_n * (tiles_n + 1) / 2, kGramThreads, smem, st>>>(xm, nk, tiles_n, C, n,
+                                                                             device_status_ptr());
+  } else {
+    for (int li = 0; li < G; ++li)
+      for (int lj = 0; lj < G; ++lj) {
+        float* Cb = C + static_cast<int64_t>(li) * d * n + static_cast<int64_t>(lj) * d;
+        if (dt == XKV_BF16)
+          gemm_simt<__nv_bfloat16, __nv_bfloat16, float, float>(
+              static_cast<const __nv_bfloat16*>(X[li]), 1, ldx, static_cast<const __nv_bfloat16*>(X[lj]), ldx, 1, Cb,
+              n, d, d, static_cast<int>(rows), 1.0, 1.0, st);
+        else
+          gemm_simt<float, float, float, float>(static_cast<const float*>(X[li]), 1, ldx,
+                                                static_cast<const float*>(X[lj]), ldx, 1, Cb, n, d, d,
+                                                static_cast<int>(rows), 1.0, 1.0, st);
+      }
+  }
+  return cudaPeekAtLastError() == cudaSuccess ? XKV_OK : XKV_ERR_CUDA;
+}
+
+xkv_status compress_plan(int G, int64_t T, int d, int rank, int oversample, int64_t shard_rows, xkv_dtype dt,
+                         CompressPlan* p) {
+  const int n = G * d;
+  int64_t b = std::min<int64_t>(std::min<int64_t>(static_cast<int64_t>(rank) + std::max(oversample, 0), n), T);
+  p->n = n;
+  p->b = static_cast<int>(b);
+  p->rank = rank;
+  p->shard = shard_rows > 0 ? std::min<int64_t>(shard_rows, T) : T;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = align_up(off + bytes);
+    return o;
+  };
+  p->off_gram = take(static_cast<size_t>(n) * n * 4);
+  p->off_gramws = take(gram_workspace(G, p->shard, d, dt));
+  p->off_Q = take(static_cast<size_t>(n) * b * 4);
+  p->off_Y = take(static_cast<size_t>(n) * b * 4);
+  p->off_W = take(static_cast<size_t>(b) * b * 8);
+  p->off_H = take(static_cast<size_t>(b) * b * 8);
+  p->off_U = take(static_cast<size_t>(b) * b * 8);
+  p->off_lam = take(static_cast<size_t>(b) * 8 + 64);
+  p->off_ord = take(static_cast<size_t>(b) * 4);
+  p->off_V = take(static_cast<size_t>(b) * rank * 4);  // Ur
+  p->off_Vr = take(static_cast<size_t>(n) * rank * 4);
+  p->off_Vt = take(static_cast<size_t>(2) * rank * n * 2);
+  p->off_jac = take(jacobi_workspace(static_cast<int>(b), 1));
+  p->bytes = off;
+  return XKV_OK;
+}
+
+xkv_status compress_launch(const CompressPlan& P, const void* const* X, int G, int64_t T, int d, int64_t ldx,
+                           xkv_dtype dt, int iters, uint64_t seed, void* A, void* Bt, float* eigvals,
+                           float* gram_out, void* ws, cudaStream_t st) {
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  const int n = P.n, b = P.b, r = P.rank;
+  const size_t es = dt == XKV_BF16 ? 2 : 4;
+  float* C = gram_out ? gram_out : reinterpret_cast<float*>(w + P.off_gram);
+  float* Q = reinterpret_cast<float*>(w + P.off_Q);
+  float* Y = reinterpret_cast<float*>(w + P.off_Y);
+  double* W = reinterpret_cast<double*>(w + P.off_W);
+  double* H = reinterpret_cast<double*>(w + P.off_H);
+  double* U = reinterpret_cast<double*>(w + P.off_U);
+  double* lam = reinterpret_cast<double*>(w + P.off_lam);
+  double* scal = lam + b;
+  int* order = reinterpret_cast<int*>(w + P.off_ord);
+  float* Ur = reinterpret_cast<float*>(w + P.off_V);
+  float* Vr = reinterpret_cast<float*>(w + P.off_Vr);
+  __nv_bfloat16* vhi = reinterpret_cast<__nv_bfloat16*>(w + P.off_Vt);
+  __nv_bfloat16* vlo = vhi + static_cast<int64_t>(r) * n;
+  int* status = device_status_ptr();
+  xkv_status s;
+
+  // 1. Gram over token shards
+  if (cudaMemsetAsync(C, 0, static_cast<size_t>(n) * n * 4, st) != cudaSuccess) return XKV_ERR_CUDA;
+  for (int64_t t0 = 0; t0 < T; t0 += P.shard) {
+    const int64_t rows = std::min<int64_t>(P.shard, T - t0);
+    const void* Xs[8];
+    for (int l = 0; l < G; ++l) Xs[l] = static_cast<const uint8_t*>(X[l]) + t0 * ldx * es;
+    s = gram_launch(Xs, G, rows, d, ldx, dt, C, w + P.off_gramws, st);
+    if (s != XKV_OK) return s;
+  }
+  // 2. block subspace iteration
+  gaussian_kernel<<<256, 256, 0, st>>>(Y, static_cast<int64_t>(n) * b, seed);
+  auto orthonormalise = [&](float* src) {
+    // shifted pass (robust to a rank-deficient block), then a plain pass
+    cholqr_pass(src, Q, n, b, 1e-13, W, H, scal, status, st);
+    cholqr_pass(Q, src, n, b, 0.0, W, H, scal, status, st);
+    cudaMemcpyAsync(Q, src, static_cast<size_t>(n) * b * 4, cudaMemcpyDeviceToDevice, st);
+  };
+  orthonormalise(Y);
+  for (int it = 0; it < iters; ++it) {
+    gemm_simt<float, float, float, float>(C, n, 1, Q, b, 1, Y, b, n, b, n, 1.0, 0.0, st);
+    orthonormalise(Y);
+  }
+  // Rayleigh-Ritz
+  gemm_simt<float, float, float, float>(C, n, 1, Q, b, 1, Y, b, n, b, n, 1.0, 0.0, st);
+  gemm_simt<float, float, double, double>(Q, 1, b, Y, b, 1, H, b, b, b, n, 1.0, 0.0, st);
+  s = jacobi_launch(H, U, lam, b, 1, w + P.off_jac, st);
+  if (s != XKV_OK) return s;
+  order_desc(lam, b, order, st);
+  gather_ritz_kernel<<<64, 256, 0, st>>>(U, order, b, r, Ur, lam, eigvals);
+  gemm_simt<float, float, float, float>(Q, b, 1, Ur, r, 1, Vr, r, n, r, b, 1.0, 0.0, st);
+  // 3. factors
+  const bool tc = dt == XKV_BF16 && r % 64 == 0 && d % 64 == 0 && !force_simt();
+  if (dt == XKV_BF16)
+    emit_factors_kernel<__nv_bfloat16><<<256, 256, 0, st>>>(Vr, n, r, static_cast<__nv_bfloat16*>(Bt), tc ? vhi : nullptr,
+                                                            vlo);
+  else
+    emit_factors_kernel<float><<<256, 256, 0, st>>>(Vr, n, r, static_cast<float*>(Bt), nullptr, nullptr);
+  if (tc) {
+    TmapSet am;
+    CUtensorMap bh, bl;
+    for (int l = 0; l < G; ++l) {
+      const uint64_t dims[2] = {static_cast<uint64_t>(d), static_cast<uint64_t>(T)};
+      const uint64_t str[1] = {static_cast<uint64_t>(ldx) * 2};
+      const uint32_t box[2] = {64, 128};
+      if (!make_tmap(&am.m[l], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, X[l], dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B))
+        return XKV_ERR_CUDA;
+    }
+    const int bn = r % 128 == 0 ? 128 : 64;
+    const uint64_t dims[2] = {static_cast<uint64_t>(n), static_cast<uint64_t>(r)};
+    const uint64_t str[1] = {static_cast<uint64_t>(n) * 2};
+    const uint32_t box[2] = {64, static_cast<uint32_t>(bn)};
+    if (!make_tmap(&bh, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, vhi, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_tmap(&bl, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, vlo, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B))
+      return XKV_ERR_CUDA;
+    GemmArgs g{};
+    g.M = static_cast<int>(T);
+    g.N = r;
+    g.K = n;
+    g.bn = bn;
+    g.layer_cols = d;
+    g.out = A;
+    g.ldo = r;
+    g.status = status;
+    const size_t smem = gemm_smem_bytes<kProj>();
+    cudaFuncSetAttribute(gemm_tc_kernel<kProj>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    dim3 grid(static_cast<unsigned>((T + 127) / 128), r / bn);
+    gemm_tc_kernel<kProj><<<grid, kGemmThreads, smem, st>>>(am, bh, bl, g);
+  } else if (dt == XKV_F32) {
+    for (int l = 0; l < G; ++l)
+      gemm_simt<float, float, float, float>(static_cast<const float*>(X[l]), ldx, 1, Vr + static_cast<int64_t>(l) * d * r,
+                                            r, 1, static_cast<float*>(A), r, static_cast<int>(T), r, d, 1.0,
+                                            l > 0 ? 1.0 : 0.0, st);
+  } else {
+    return XKV_ERR_UNSUPPORTED;
+  }
+  return cudaPeekAtLastError() == cudaSuccess ? XKV_OK : XKV_ERR_CUDA;
+}
+
+}  // namespace xkv

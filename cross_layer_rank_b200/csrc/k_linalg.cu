@@ -1,0 +1,495 @@
+// Small dense linear algebra of the factorisation path, on CUDA cores:
+//   - a strided SIMT GEMM (fp32 or fp64 accumulation) for the subspace
+//     iteration products and the f32 fall-backs;
+//   - shifted Cholesky QR pieces (Gram of a tall block, Cholesky, triangular
+//     inverse) in fp64;
+//   - a one-sided block Jacobi eigen-solver (fp64) for symmetric positive
+//     semi-definite matrices: the Rayleigh-Ritz step (eigenvalues + vectors)
+//     and KV-CoRE's spectra (eigenvalues only);
+//   - ordering of eigenvalues and the NER reduction (KV-CoRE page, 2.B).
+#include <algorithm>
+
+#include "xkv_common.cuh"
+#include "xkv_internal.h"
+#include "xkv_linalg.cuh"
+
+namespace xkv {
+
+// --------------------------------------------------------------- SIMT GEMM
+template <typename TA, typename TB, typename TC, typename ACC>
+__global__ void __launch_bounds__(256) gemm_simt_kernel(const TA* __restrict__ A, int64_t sam, int64_t sak,
+                                                        const TB* __restrict__ B, int64_t sbk, int64_t sbn,
+                                                        TC* __restrict__ C, int64_t ldc, int M, int N, int K,
+                                                        double alpha, double beta) {
+  __shared__ ACC As[16][65];
+  __shared__ ACC Bs[16][65];
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+  const int m0 = blockIdx.y * 64, n0 = blockIdx.x * 64;
+  ACC acc[4][4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) acc[i][j] = ACC(0);
+  for (int k0 = 0; k0 < K; k0 += 16) {
+    for (int i = threadIdx.x; i < 16 * 64; i += 256) {
+      // A tile: choose the order that makes consecutive threads touch consecutive memory
+      int kk, mm;
+      if (sam == 1) { mm = i & 63; kk = i >> 6; } else { kk = i & 15; mm = i >> 4; }
+      const int m = m0 + mm, k = k0 + kk;
+      As[kk][mm] = (m < M && k < K) ? static_cast<ACC>(to_f_any(A[m * sam + k * sak])) : ACC(0);
+      int kb, nn;
+      if (sbn == 1) { nn = i & 63; kb = i >> 6; } else { kb = i & 15; nn = i >> 4; }
+      const int n = n0 + nn, k2 = k0 + kb;
+      Bs[kb][nn] = (n < N && k2 < K) ? static_cast<ACC>(to_f_any(B[k2 * sbk + n * sbn])) : ACC(0);
+    }
+    __syncthreads();
+#pragma unroll
+    for (int kk = 0; kk < 16; ++kk) {
+      ACC a[4], b[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) a[i] = As[kk][ty + 16 * i];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) b[j] = Bs[kk][tx + 16 * j];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] += a[i] * b[j];
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int m = m0 + ty + 16 * i;
+    if (m >= M) continue;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int n = n0 + tx + 16 * j;
+      if (n >= N) continue;
+      TC* c = C + static_cast<int64_t>(m) * ldc + n;
+      const double prev = beta != 0.0 ? static_cast<double>(to_f_any(*c)) : 0.0;
+      store_any(c, alpha * static_cast<double>(acc[i][j]) + beta * prev);
+    }
+  }
+}
+
+template <typename TA, typename TB, typename TC, typename ACC>
+void gemm_simt(const TA* A, int64_t sam, int64_t sak, const TB* B, int64_t sbk, int64_t sbn, TC* C, int64_t ldc,
+               int M, int N, int K, double alpha, double beta, cudaStream_t st) {
+  dim3 grid((N + 63) / 64, (M + 63) / 64);
+  gemm_simt_kernel<TA, TB, TC, ACC><<<grid, 256, 0, st>>>(A, sam, sak, B, sbk, sbn, C, ldc, M, N, K, alpha, beta);
+}
+
+#define XKV_GEMM_INST(TA, TB, TC, ACC)                                                                        \
+  template void gemm_simt<TA, TB, TC, ACC>(const TA*, int64_t, int64_t, const TB*, int64_t, int64_t, TC*, \
+                                           int64_t, int, int, int, double, double, cudaStream_t);
+XKV_GEMM_INST(float, float, float, float)
+XKV_GEMM_INST(__nv_bfloat16, __nv_bfloat16, float, float)
+XKV_GEMM_INST(__nv_bfloat16, float, float, float)
+XKV_GEMM_INST(__nv_bfloat16, __nv_bfloat16, __nv_bfloat16, float)
+XKV_GEMM_INST(float, double, float, double)
+XKV_GEMM_INST(float, float, double, double)
+XKV_GEMM_INST(float, double, double, double)
+#undef XKV_GEMM_INST
+
+// ---------------------------------------------------- Cholesky QR pieces
+// In-place lower Cholesky factor of (W + shift I), b x b fp64 (row-major; only
+// the lower triangle is read and written), one CTA.  shift = shift_rel *
+// trace(W) when a device trace is given.  A non-positive pivot is recorded as
+// a numerical fault and replaced by a tiny positive one so results stay finite.
+__global__ void __launch_bounds__(1024) cholesky_kernel(double* __restrict__ W, int b, double shift_rel,
+                                                        const double* __restrict__ trace, int* status) {
+  extern __shared__ double colj[];
+  __shared__ double s_piv;
+  const double shift = trace ? shift_rel * (*trace) : 0.0;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  for (int j = 0; j < b; ++j) {
+    if (tid == 0) {
+      double d = W[static_cast<int64_t>(j) * b + j] + shift;
+      if (!(d > 0.0) || !isfinite(d)) {
+        record_status(status, kDevNumerical);
+        d = 1e-300;
+      }
+      s_piv = sqrt(d);
+      W[static_cast<int64_t>(j) * b + j] = s_piv;
+    }
+    __syncthreads();
+    const double piv = s_piv;
+    for (int i = j + 1 + tid; i < b; i += blockDim.x) {
+      const double v = W[static_cast<int64_t>(i) * b + j] / piv;
+      W[static_cast<int64_t>(i) * b + j] = v;
+      colj[i] = v;
+    }
+    __syncthreads();
+    for (int i = j + 1 + warp; i < b; i += 32) {
+      const double wij = colj[i];
+      double* wi = W + static_cast<int64_t>(i) * b;
+      for (int l = j + 1 + lane; l <= i; l += 32) wi[l] -= wij * colj[l];
+    }
+    __syncthreads();
+  }
+}
+
+// X = L^{-1} for a lower-triangular L (row-major b x b), one warp per column.
+__global__ void __launch_bounds__(256) tri_inverse_kernel(const double* __restrict__ L, double* __restrict__ X,
+                                                          int b) {
+  extern __shared__ double xs[];  // [8 warps][b]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int j = blockIdx.x * 8 + warp;
+  if (j >= b) return;
+  double* x = xs + static_cast<int64_t>(warp) * b;
+  for (int i = lane; i < b; i += 32) x[i] = 0.0;
+  __syncwarp();
+  for (int i = j; i < b; ++i) {
+    const double* li = L + static_cast<int64_t>(i) * b;
+    double s = 0.0;
+    for (int k = j + lane; k < i; k += 32) s += li[k] * x[k];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    if (lane == 0) x[i] = ((i == j ? 1.0 : 0.0) - s) / li[i];
+    __syncwarp();
+  }
+  for (int i = lane; i < b; i += 32) X[static_cast<int64_t>(i) * b + j] = i >= j ? x[i] : 0.0;
+}
+
+__global__ void trace_kernel(const double* __restrict__ W, int b, double* __restrict__ out) {
+  __shared__ double red[32];
+  double s = 0.0;
+  for (int i = threadIdx.x; i < b; i += blockDim.x) s += W[static_cast<int64_t>(i) * b + i];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = s;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double t = 0.0;
+    for (int i = 0; i < static_cast<int>(blockDim.x >> 5); ++i) t += red[i];
+    *out = t;
+  }
+}
+
+// One pass of (shifted) Cholesky QR: W = Y^T Y (fp64), L = chol(W + shift I),
+// Q = Y L^{-T}.  Y, Q: n x b fp32 row-major (distinct buffers).  W, Linv: b x b
+// fp64 scratch; scal: one fp64 scratch scalar.
+void cholqr_pass(const float* Y, float* Q, int n, int b, double shift_rel, double* W, double* Linv, double* scal,
+                 int* status, cudaStream_t st) {
+  gemm_simt<float, float, double, double>(Y, 1, b, Y, b, 1, W, b, b, b, n, 1.0, 0.0, st);
+  if (shift_rel > 0.0) trace_kernel<<<1, 256, 0, st>>>(W, b, scal);
+  const size_t smem = static_cast<size_t>(b) * 8;
+  if (smem > 48 * 1024)
+    cudaFuncSetAttribute(cholesky_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  cholesky_kernel<<<1, 1024, smem, st>>>(W, b, shift_rel, shift_rel > 0.0 ? scal : nullptr, status);
+  const size_t smem2 = static_cast<size_t>(8) * b * 8;
+  if (smem2 > 48 * 1024)
+    cudaFuncSetAttribute(tri_inverse_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem2));
+  tri_inverse_kernel<<<(b + 7) / 8, 256, smem2, st>>>(W, Linv, b);
+  // Q(m, j) = sum_k Y(m, k) Linv(j, k)
+  gemm_simt<float, double, float, double>(Y, b, 1, Linv, 1, b, Q, b, n, b, b, 1.0, 0.0, st);
+}
+
+// ------------------------------------------------------ one-sided Jacobi
+// count independent problems of size n (column-major n x n each; symmetric
+// matrices may be given in either order).  Columns are grouped in blocks of
+// 16; every round pairs the blocks by the round-robin schedule and each CTA
+// orthogonalises the 32 columns of its pair: Gram G = Wc^T Wc, eigenvectors R
+// of G by cyclic Jacobi, Wc <- Wc R, Vc <- Vc R.  A sweep is nblk - 1 rounds;
+// a sweep that rotates nothing ends the iteration (later launches return at
+// once).  On convergence column i of W is lambda_i v_i, so |lambda_i| is its
+// norm and v_i is column i of V.
+constexpr int kJB = 16;
+
+struct JacobiState {
+  int active;      // rotations performed in the current sweep
+  int converged;
+};
+
+__device__ __forceinline__ int rr_player(int pos, int round, int nplayers) {
+  if (pos == 0) return 0;
+  return ((pos - 1 + round) % (nplayers - 1)) + 1;
+}
+
+__global__ void __launch_bounds__(256) jacobi_round_kernel(double* __restrict__ W, double* __restrict__ V, int n,
+                                                           int nblk, int round, JacobiState* __restrict__ state,
+                                                           double tol) {
+  __shared__ double G[32][33];
+  __shared__ double R[32][33];
+  __shared__ double tile[32][33];
+  __shared__ double cs[16], sn[16];
+  __shared__ int pp[16], qq[16];
+  const int prob = blockIdx.y;
+  JacobiState* stp = state + prob;
+  if (stp->converged) return;
+  double* Wp = W + static_cast<int64_t>(prob) * n * n;
+  double* Vp = V ? V + static_cast<int64_t>(prob) * n * n : nullptr;
+  const int pair = blockIdx.x;
+  const int I = rr_player(pair, round, nblk), J = rr_player(nblk - 1 - pair, round, nblk);
+  const int tid = threadIdx.x;
+  __shared__ int cols[32];
+  if (tid < 32) {
+    const int blk = tid < 16 ? I : J;
+    const int c = blk * kJB + (tid & 15);
+    cols[tid] = c < n ? c : -1;
+  }
+  // Gram of the 32 columns
+  for (int i = tid; i < 32 * 32; i += 256) G[i / 32][i % 32] = 0.0;
+  __syncthreads();
+  {
+    const int a = tid >> 3, bb = (tid & 7) * 4;  // thread owns G[a][bb..bb+3]
+    double acc[4] = {0, 0, 0, 0};
+    for (int r0 = 0; r0 < n; r0 += 32) {
+      for (int i = tid; i < 32 * 32; i += 256) {
+        const int c = i / 32, r = i % 32;
+        const int cc = cols[c];
+        tile[r][c] = (cc >= 0 && r0 + r < n) ? Wp[static_cast<int64_t>(cc) * n + r0 + r] : 0.0;
+      }
+      __syncthreads();
+#pragma unroll 4
+      for (int r = 0; r < 32; ++r) {
+        const double x = tile[r][a];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[e] += x * tile[r][bb + e];
+      }
+      __syncthreads();
+    }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) G[a][bb + e] = acc[e];
+  }
+  // the pair is converged when every fresh column product is tiny relative to
+  // the column norms: |w_p . w_q| <= tol ||w_p|| ||w_q||
+  __shared__ int s_need;
+  if (tid == 0) s_need = 0;
+  __syncthreads();
+  for (int i = tid; i < 32 * 32; i += 256) {
+    const int p = i / 32, q = i % 32;
+    if (p < q && fabs(G[p][q]) > tol * sqrt(fabs(G[p][p] * G[q][q])) && G[p][q] != 0.0) s_need = 1;
+  }
+  for (int i = tid; i < 32 * 32; i += 256) R[i / 32][i % 32] = (i / 32 == i % 32) ? 1.0 : 0.0;
+  __syncthreads();
+  if (!s_need) return;
+  // cyclic Jacobi on G (round-robin over 32 indices: 31 steps of 16 pairs);
+  // entries already below 1e-14 of the diagonal scale are left alone
+  for (int sweep = 0; sweep < 12; ++sweep) {
+    __shared__ int s_any;
+    if (tid == 0) s_any = 0;
+    __syncthreads();
+    for (int step = 0; step < 31; ++step) {
+      if (tid < 16) {
+        int p = rr_player(tid, step, 32), q = rr_player(31 - tid, step, 32);
+        if (p > q) { const int t = p; p = q; q = t; }
+        pp[tid] = p;
+        qq[tid] = q;
+        const double gpq = G[p][q], gpp = G[p][p], gqq = G[q][q];
+        if (fabs(gpq) > 1e-14 * sqrt(fabs(gpp * gqq)) && gpq != 0.0) {
+          const double tau = (gqq - gpp) / (2.0 * gpq);
+          const double t = (tau >= 0.0 ? 1.0 : -1.0) / (fabs(tau) + sqrt(1.0 + tau * tau));
+          cs[tid] = 1.0 / sqrt(1.0 + t * t);
+          sn[tid] = t * cs[tid];
+          s_any = 1;
+        } else {
+          cs[tid] = 1.0;
+          sn[tid] = 0.0;
+        }
+      }
+      __syncthreads();
+      // columns of G and R
+      for (int i = tid; i < 16 * 32; i += 256) {
+        const int k = i / 32, r = i % 32;
+        const int p = pp[k], q = qq[k];
+        const double c = cs[k], s = sn[k];
+        if (s == 0.0) continue;
+        const double gp = G[r][p], gq = G[r][q];
+        G[r][p] = c * gp - s * gq;
+        G[r][q] = s * gp + c * gq;
+        const double rp = R[r][p], rq = R[r][q];
+        R[r][p] = c * rp - s * rq;
+        R[r][q] = s * rp + c * rq;
+      }
+      __syncthreads();
+      for (int i = tid; i < 16 * 32; i += 256) {
+        const int k = i / 32, cidx = i % 32;
+        const int p = pp[k], q = qq[k];
+        const double c = cs[k], s = sn[k];
+        if (s == 0.0) continue;
+        const double gp = G[p][cidx], gq = G[q][cidx];
+        G[p][cidx] = c * gp - s * gq;
+        G[q][cidx] = s * gp + c * gq;
+      }
+      __syncthreads();
+    }
+    const int any = s_any;
+    __syncthreads();
+    if (!any) break;
+  }
+  if (tid == 0) atomicAdd(&stp->active, 1);
+  // Wc <- Wc R, Vc <- Vc R (row by row)
+  for (int mat = 0; mat < (Vp ? 2 : 1); ++mat) {
+    double* M = mat == 0 ? Wp : Vp;
+    for (int r0 = 0; r0 < n; r0 += 256) {
+      const int r = r0 + tid;
+      double x[32];
+#pragma unroll
+      for (int c = 0; c < 32; ++c) x[c] = (cols[c] >= 0 && r < n) ? M[static_cast<int64_t>(cols[c]) * n + r] : 0.0;
+      if (r < n) {
+        for (int c = 0; c < 32; ++c) {
+          if (cols[c] < 0) continue;
+          double y = 0.0;
+#pragma unroll
+          for (int e = 0; e < 32; ++e) y += x[e] * R[e][c];
+          M[static_cast<int64_t>(cols[c]) * n + r] = y;
+        }
+      }
+    }
+  }
+}
+
+__global__ void jacobi_sweep_end_kernel(JacobiState* state, int count) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= count) return;
+  if (!state[i].converged && state[i].active == 0) state[i].converged = 1;
+  state[i].active = 0;
+}
+
+__global__ void jacobi_init_kernel(double* V, int n, int count, JacobiState* state) {
+  const int64_t total = static_cast<int64_t>(count) * n * n;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    if (V) {
+      const int64_t w = i % (static_cast<int64_t>(n) * n);
+      V[i] = (w / n == w % n) ? 1.0 : 0.0;
+    }
+    if (i < count) { state[i].active = 0; state[i].converged = 0; }
+  }
+}
+
+__global__ void column_norms_kernel(const double* __restrict__ W, double* __restrict__ lam, int n, int count) {
+  const int prob = blockIdx.y;
+  const int c = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (c >= n) return;
+  const double* col = W + static_cast<int64_t>(prob) * n * n + static_cast<int64_t>(c) * n;
+  double s = 0.0;
+  for (int r = lane; r < n; r += 32) s += col[r] * col[r];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  if (lane == 0) lam[static_cast<int64_t>(prob) * n + c] = sqrt(s);
+}
+
+size_t jacobi_workspace(int, int count) { return align_up(static_cast<size_t>(count) * sizeof(JacobiState)); }
+
+xkv_status jacobi_launch(double* W, double* V, double* lam, int n, int count, void* ws, cudaStream_t st) {
+  JacobiState* state = static_cast<JacobiState*>(ws);
+  int nblk = (n + kJB - 1) / kJB;
+  if (nblk & 1) ++nblk;
+  if (nblk < 2) nblk = 2;
+  jacobi_init_kernel<<<256, 256, 0, st>>>(V, n, count, state);
+  const int max_sweeps = 30;
+  for (int s = 0; s < max_sweeps; ++s) {
+    for (int r = 0; r < nblk - 1; ++r)
+      jacobi_round_kernel<<<dim3(nblk / 2, count), 256, 0, st>>>(W, V, n, nblk, r, state, 1e-11);
+    jacobi_sweep_end_kernel<<<(count + 127) / 128, 128, 0, st>>>(state, count);
+  }
+  column_norms_kernel<<<dim3((n + 7) / 8, count), 256, 0, st>>>(W, lam, n, count);
+  return cudaPeekAtLastError() == cudaSuccess ? XKV_OK : XKV_ERR_CUDA;
+}
+
+// --------------------------------------------------------------- ordering
+// order[k] = index of the k-th largest value (ties: lower index first).
+__global__ void order_desc_kernel(const double* __restrict__ v, int n, int* __restrict__ order) {
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) {
+    const double x = v[i];
+    int rank = 0;
+    for (int j = 0; j < n; ++j) {
+      const double y = v[j];
+      rank += (y > x) || (y == x && j < i);
+    }
+    order[rank] = i;
+  }
+}
+
+void order_desc(const double* v, int n, int* order, cudaStream_t st) {
+  order_desc_kernel<<<(n + 255) / 256, 256, 0, st>>>(v, n, order);
+}
+
+// ------------------------------------------------------------------- NER
+// One CTA per block: from |lambda| of the block (unsorted), numerical rank
+// r = #{lambda > tol lambda_max}; sigma = sqrt(lambda); p = sigma / sum sigma;
+// erank = exp(-sum p ln p); NER = erank / r.
+__global__ void __launch_bounds__(256) ner_kernel(const double* __restrict__ lam, int n, double tol,
+                                                  float* __restrict__ ner, float* __restrict__ erank,
+                                                  int32_t* __restrict__ rank) {
+  __shared__ double red[8];
+  __shared__ double s_val;
+  const double* l = lam + static_cast<int64_t>(blockIdx.x) * n;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  auto block_reduce = [&](double v, bool is_max) -> double {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const double w = __shfl_xor_sync(0xffffffffu, v, o);
+      v = is_max ? fmax(v, w) : v + w;
+    }
+    if (lane == 0) red[warp] = v;
+    __syncthreads();
+    if (tid == 0) {
+      double t = red[0];
+      for (int i = 1; i < 8; ++i) t = is_max ? fmax(t, red[i]) : t + red[i];
+      s_val = t;
+    }
+    __syncthreads();
+    const double r = s_val;
+    __syncthreads();
+    return r;
+  };
+  double mx = 0.0;
+  for (int i = tid; i < n; i += 256) mx = fmax(mx, l[i]);
+  const double lmax = block_reduce(mx, true);
+  double cnt = 0.0, ssum = 0.0;
+  for (int i = tid; i < n; i += 256)
+    if (lmax > 0.0 && l[i] > tol * lmax) { cnt += 1.0; ssum += sqrt(l[i]); }
+  const double r = block_reduce(cnt, false);
+  const double S = block_reduce(ssum, false);
+  double h = 0.0;
+  for (int i = tid; i < n; i += 256)
+    if (lmax > 0.0 && l[i] > tol * lmax) {
+      const double p = sqrt(l[i]) / S;
+      if (p > 0.0) h -= p * log(p);
+    }
+  const double H = block_reduce(h, false);
+  if (tid == 0) {
+    const double er = r > 0.0 ? exp(H) : 0.0;
+    ner[blockIdx.x] = static_cast<float>(r > 0.0 ? er / r : 0.0);
+    if (erank) erank[blockIdx.x] = static_cast<float>(er);
+    if (rank) rank[blockIdx.x] = static_cast<int32_t>(r);
+  }
+}
+
+// diagonal blocks of an n x n fp32 Gram -> count x (block x block) fp64
+__global__ void extract_blocks_kernel(const float* __restrict__ C, int n, int block, double* __restrict__ out) {
+  const int b = blockIdx.y;
+  const int64_t total = static_cast<int64_t>(block) * block;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int r = static_cast<int>(i / block), c = static_cast<int>(i % block);
+    out[static_cast<int64_t>(b) * total + i] =
+        static_cast<double>(C[static_cast<int64_t>(b * block + r) * n + b * block + c]);
+  }
+}
+
+size_t ner_workspace(int n, int block) {
+  const int count = n / block;
+  return align_up(static_cast<size_t>(count) * block * block * 8) + align_up(static_cast<size_t>(count) * block * 8) +
+         jacobi_workspace(block, count);
+}
+
+xkv_status ner_launch(const float* gram, int n, int block, double tol, float* ner, float* erank, int32_t* rank,
+                      void* ws, cudaStream_t st) {
+  const int count = n / block;
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  double* Wb = reinterpret_cast<double*>(w);
+  double* lam = reinterpret_cast<double*>(w + align_up(static_cast<size_t>(count) * block * block * 8));
+  void* jws = w + align_up(static_cast<size_t>(count) * block * block * 8) + align_up(static_cast<size_t>(count) * block * 8);
+  extract_blocks_kernel<<<dim3(128, count), 256, 0, st>>>(gram, n, block, Wb);
+  xkv_status s = jacobi_launch(Wb, nullptr, lam, block, count, jws, st);
+  if (s != XKV_OK) return s;
+  ner_kernel<<<count, 256, 0, st>>>(lam, block, tol, ner, erank, rank);
+  return cudaPeekAtLastError() == cudaSuccess ? XKV_OK : XKV_ERR_CUDA;
+}
+
+}  // namespace xkv

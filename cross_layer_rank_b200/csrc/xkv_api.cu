@@ -1,0 +1,318 @@
+// C-ABI entry points of libxkv (declared in include/xkv.h): argument
+// validation (nothing is launched on a bad argument), workspace sizing, TMA
+// descriptor creation and the per-device status word.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include <algorithm>
+#include <mutex>
+
+#include "xkv_internal.h"
+
+namespace xkv {
+
+static __device__ int g_device_status;
+
+namespace {
+constexpr int kMaxDevices = 64;
+int* g_status_ptr[kMaxDevices] = {nullptr};
+int g_sms[kMaxDevices] = {0};
+std::mutex g_mu;
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn g_encode = nullptr;
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline bool aligned256(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 255u) == 0; }
+}  // namespace
+
+int* device_status_ptr() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_status_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess) return nullptr;
+    g_status_ptr[dev] = static_cast<int*>(p);
+  }
+  return g_status_ptr[dev];
+}
+
+int num_sms() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
+  if (!g_sms[dev]) {
+    int v = 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) v = 148;
+    g_sms[dev] = v;
+  }
+  return g_sms[dev];
+}
+
+bool force_simt() {
+  static int v = -1;
+  if (v < 0) {
+    const char* e = getenv("XKV_FORCE_SIMT");
+    v = (e && e[0] == '1') ? 1 : 0;
+  }
+  return v == 1;
+}
+
+bool make_tmap(CUtensorMap* map, CUtensorMapDataType dt, int rank, const void* base, const uint64_t* dims,
+               const uint64_t* strides_bytes, const uint32_t* box, CUtensorMapSwizzle swz) {
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!g_encode) {
+      void* fn = nullptr;
+      cudaDriverEntryPointQueryResult q;
+      if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+          q != cudaDriverEntryPointSuccess || !fn)
+        return false;
+      g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+    }
+  }
+  cuuint64_t d[5];
+  cuuint64_t s[4];
+  cuuint32_t b[5], e[5];
+  for (int i = 0; i < rank; ++i) {
+    d[i] = dims[i];
+    b[i] = box[i];
+    e[i] = 1;
+    if (i + 1 < rank) s[i] = strides_bytes[i];
+  }
+  const CUresult r = g_encode(map, dt, static_cast<cuuint32_t>(rank), const_cast<void*>(base), d, s, b, e,
+                              CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+}  // namespace xkv
+
+using namespace xkv;
+
+extern "C" {
+
+const char* xkv_status_string(xkv_status s) {
+  switch (s) {
+    case XKV_OK: return "ok";
+    case XKV_ERR_INVALID_ARG: return "invalid argument";
+    case XKV_ERR_UNSUPPORTED: return "unsupported configuration";
+    case XKV_ERR_WORKSPACE: return "workspace missing or too small";
+    case XKV_ERR_CUDA: return "CUDA error";
+    case XKV_ERR_NUMERICAL: return "numerical breakdown detected on the device";
+    case XKV_ERR_DEVICE_TIMEOUT: return "bounded device-side wait expired";
+  }
+  return "unknown status";
+}
+
+int xkv_version(void) { return (1 << 16) | 0; }
+
+xkv_status xkv_get_device_status(void* stream) {
+  int* p = device_status_ptr();
+  if (!p) return XKV_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int v = 0;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return XKV_ERR_CUDA;
+  if (cudaMemcpy(&v, p, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return XKV_ERR_CUDA;
+  if (v != 0) {
+    const int zero = 0;
+    if (cudaMemcpy(p, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) return XKV_ERR_CUDA;
+  }
+  return static_cast<xkv_status>(v);
+}
+
+// ------------------------------------------------------------------- Gram
+static xkv_status check_layers(const void* const* X, int G, int d, int64_t ldx, xkv_dtype dt) {
+  if (!X || G < 1 || G > 8 || d < 64 || d % 64 != 0 || ldx < d || ldx % 8 != 0) return XKV_ERR_INVALID_ARG;
+  if (dt != XKV_F32 && dt != XKV_BF16) return XKV_ERR_INVALID_ARG;
+  for (int l = 0; l < G; ++l)
+    if (!X[l] || !aligned16(X[l])) return XKV_ERR_INVALID_ARG;
+  return XKV_OK;
+}
+
+xkv_status xkv_gram_workspace_size(int G, int64_t rows, int d, xkv_dtype dt, size_t* bytes) {
+  if (!bytes || G < 1 || G > 8 || d < 64 || d % 64 != 0 || rows < 0) return XKV_ERR_INVALID_ARG;
+  *bytes = gram_workspace(G, rows, d, dt);
+  return XKV_OK;
+}
+
+xkv_status xkv_gram_accumulate(const void* const* X_layers, int G, int64_t rows, int d, int64_t ldx, xkv_dtype dt,
+                               float* C, void* workspace, size_t ws_bytes, void* stream) {
+  xkv_status s = check_layers(X_layers, G, d, ldx, dt);
+  if (s != XKV_OK) return s;
+  if (!C || !aligned16(C) || rows < 0) return XKV_ERR_INVALID_ARG;
+  const size_t need = gram_workspace(G, rows, d, dt);
+  if (need > kAlign && (!workspace || ws_bytes < need || !aligned256(workspace))) return XKV_ERR_WORKSPACE;
+  return gram_launch(X_layers, G, rows, d, ldx, dt, C, workspace, static_cast<cudaStream_t>(stream));
+}
+
+// ------------------------------------------------------------ compression
+static xkv_status check_compress(int G, int64_t T, int d, int rank, int iters, int oversample, int64_t shard_rows,
+                                 xkv_dtype dt) {
+  if (G < 1 || G > 8 || T < 1 || d < 64 || d % 64 != 0 || rank < 1 || rank % 16 != 0 || iters < 1 ||
+      oversample < 0 || shard_rows < 0 || T > (int64_t(1) << 31) - 1)
+    return XKV_ERR_INVALID_ARG;
+  if (rank > G * d || rank > T) return XKV_ERR_INVALID_ARG;
+  if (dt != XKV_F32 && dt != XKV_BF16) return XKV_ERR_INVALID_ARG;
+  if (dt == XKV_BF16 && rank % 64 != 0) return XKV_ERR_UNSUPPORTED;
+  return XKV_OK;
+}
+
+xkv_status xkv_compress_workspace_size(int G, int64_t T, int d, int rank, int oversample, int64_t shard_rows,
+                                       xkv_dtype dt, size_t* bytes) {
+  if (!bytes) return XKV_ERR_INVALID_ARG;
+  xkv_status s = check_compress(G, T, d, rank, 1, oversample, shard_rows, dt);
+  if (s != XKV_OK) return s;
+  CompressPlan p;
+  compress_plan(G, T, d, rank, oversample, shard_rows, dt, &p);
+  *bytes = p.bytes;
+  return XKV_OK;
+}
+
+xkv_status xkv_compress_group(const void* const* X_layers, int G, int64_t T, int d, int64_t ldx, xkv_dtype dt,
+                              int rank, int iters, int oversample, int64_t shard_rows, uint64_t seed, void* A, void* Bt,
+                              float* eigvals, float* gram_out, void* workspace, size_t ws_bytes, void* stream) {
+  xkv_status s = check_compress(G, T, d, rank, iters, oversample, shard_rows, dt);
+  if (s != XKV_OK) return s;
+  s = check_layers(X_layers, G, d, ldx, dt);
+  if (s != XKV_OK) return s;
+  if (!A || !Bt || !aligned16(A) || !aligned16(Bt)) return XKV_ERR_INVALID_ARG;
+  if ((eigvals && !aligned16(eigvals)) || (gram_out && !aligned16(gram_out))) return XKV_ERR_INVALID_ARG;
+  CompressPlan p;
+  compress_plan(G, T, d, rank, oversample, shard_rows, dt, &p);
+  if (!workspace || ws_bytes < p.bytes || !aligned256(workspace)) return XKV_ERR_WORKSPACE;
+  return compress_launch(p, X_layers, G, T, d, ldx, dt, iters, seed, A, Bt, eigvals, gram_out, workspace,
+                         static_cast<cudaStream_t>(stream));
+}
+
+// -------------------------------------------------------------- landmarks
+xkv_status xkv_build_landmarks(const void* K, int64_t T, int64_t ldk, int n_kv_heads, int head_dim, xkv_dtype dt,
+                               int chunk, int sink, int recent, float rope_theta, void* landmarks, void* stream) {
+  if (!K || !landmarks || !aligned16(K) || !aligned16(landmarks)) return XKV_ERR_INVALID_ARG;
+  if (n_kv_heads < 1 || head_dim < 2 || head_dim % 2 != 0 || head_dim > 256 || chunk < 1 || sink < 0 || recent < 0)
+    return XKV_ERR_INVALID_ARG;
+  if (dt != XKV_F32 && dt != XKV_BF16) return XKV_ERR_INVALID_ARG;
+  if (ldk < static_cast<int64_t>(n_kv_heads) * head_dim || T < sink + recent) return XKV_ERR_INVALID_ARG;
+  if ((T - sink - recent) % chunk != 0 || !(rope_theta > 1.0f)) return XKV_ERR_INVALID_ARG;
+  return landmarks_launch(K, T, ldk, n_kv_heads, head_dim, dt, chunk, sink, recent, rope_theta, landmarks,
+                          static_cast<cudaStream_t>(stream));
+}
+
+// -------------------------------------------------------------- SR decode
+static xkv_status check_sr(const xkv_sr_params* p) {
+  if (!p) return XKV_ERR_INVALID_ARG;
+  if (p->batch < 1 || p->n_kv_heads < 1 || p->n_q_heads < p->n_kv_heads || p->n_q_heads % p->n_kv_heads != 0)
+    return XKV_ERR_INVALID_ARG;
+  if (p->head_dim < 2 || p->head_dim % 2 != 0 || p->chunk < 1 || p->sink < 0 || p->recent < 0 || p->topk < 1)
+    return XKV_ERR_INVALID_ARG;
+  if (p->rank_k < 1 || p->rank_v < 1 || p->T < p->sink + p->recent + p->chunk) return XKV_ERR_INVALID_ARG;
+  if ((p->T - p->sink - p->recent) % p->chunk != 0) return XKV_ERR_INVALID_ARG;
+  const int64_t n_mid = (p->T - p->sink - p->recent) / p->chunk;
+  if (p->topk > n_mid) return XKV_ERR_INVALID_ARG;
+  if (p->a_k_batch_stride < p->T * p->rank_k || p->a_v_batch_stride < p->T * p->rank_v) return XKV_ERR_INVALID_ARG;
+  const int64_t d = static_cast<int64_t>(p->n_kv_heads) * p->head_dim;
+  if ((p->bt_k_batch_stride != 0 && p->bt_k_batch_stride < d * p->rank_k) ||
+      (p->bt_v_batch_stride != 0 && p->bt_v_batch_stride < d * p->rank_v) || p->bt_k_batch_stride < 0 ||
+      p->bt_v_batch_stride < 0)
+    return XKV_ERR_INVALID_ARG;
+  if (p->dtype != XKV_F32 && p->dtype != XKV_BF16) return XKV_ERR_INVALID_ARG;
+  if (!(p->rope_theta > 1.0f)) return XKV_ERR_INVALID_ARG;
+  const int gq = p->n_q_heads / p->n_kv_heads;
+  if (gq > 8 || p->head_dim > 256 || p->sink + p->recent > 64 || n_mid * 4 > 200 * 1024 || p->rank_v > 4096 ||
+      p->topk > 1024)
+    return XKV_ERR_UNSUPPORTED;
+  if (p->T > (int64_t(1) << 30)) return XKV_ERR_UNSUPPORTED;
+  return XKV_OK;
+}
+
+xkv_status xkv_sr_workspace_size(const xkv_sr_params* p, size_t* bytes) {
+  if (!bytes) return XKV_ERR_INVALID_ARG;
+  xkv_status s = check_sr(p);
+  if (s != XKV_OK) return s;
+  SRPlan plan;
+  sr_plan(p, &plan);
+  *bytes = plan.bytes;
+  return XKV_OK;
+}
+
+xkv_status xkv_sr_attention_decode(const xkv_sr_params* p, const void* q, const void* A_K, const void* Bt_K,
+                                   const void* A_V, const void* Bt_V, const void* landmarks, const void* sr_K,
+                                   const void* sr_V, float* out, int32_t* sel_out, void* workspace, size_t ws_bytes,
+                                   void* stream) {
+  xkv_status s = check_sr(p);
+  if (s != XKV_OK) return s;
+  const void* ptrs[] = {q, A_K, Bt_K, A_V, Bt_V, landmarks, out};
+  for (const void* x : ptrs)
+    if (!x || !aligned16(x)) return XKV_ERR_INVALID_ARG;
+  if (p->sink + p->recent > 0 && (!sr_K || !sr_V || !aligned16(sr_K) || !aligned16(sr_V))) return XKV_ERR_INVALID_ARG;
+  if (sel_out && !aligned16(sel_out)) return XKV_ERR_INVALID_ARG;
+  SRPlan plan;
+  sr_plan(p, &plan);
+  if (!workspace || ws_bytes < plan.bytes || !aligned256(workspace)) return XKV_ERR_WORKSPACE;
+  return sr_launch(p, plan, q, A_K, Bt_K, A_V, Bt_V, landmarks, sr_K, sr_V, out, sel_out, workspace,
+                   static_cast<cudaStream_t>(stream));
+}
+
+// --------------------------------------------------- full reconstruction
+xkv_status xkv_full_reconstruct(const void* A, const void* Bt, int64_t T, int rank, int d, int n_kv_heads,
+                                int head_dim, int apply_rope, float rope_theta, xkv_dtype dt, void* out, void* stream) {
+  if (!A || !Bt || !out || !aligned16(A) || !aligned16(Bt) || !aligned16(out)) return XKV_ERR_INVALID_ARG;
+  if (T < 0 || rank < 1 || rank % 16 != 0 || d < 1 || n_kv_heads < 1 || head_dim < 2 || head_dim % 2 != 0 ||
+      n_kv_heads * head_dim != d)
+    return XKV_ERR_INVALID_ARG;
+  if (dt != XKV_F32 && dt != XKV_BF16) return XKV_ERR_INVALID_ARG;
+  if (apply_rope && !(rope_theta > 1.0f)) return XKV_ERR_INVALID_ARG;
+  if (T > (int64_t(1) << 31) - 1) return XKV_ERR_UNSUPPORTED;
+  return recon_launch(A, Bt, T, rank, d, n_kv_heads, head_dim, apply_rope, rope_theta, dt, out,
+                      static_cast<cudaStream_t>(stream));
+}
+
+static xkv_status check_dense(const xkv_dense_params* p) {
+  if (!p || p->batch < 1 || p->n_kv_heads < 1 || p->n_q_heads % p->n_kv_heads != 0 || p->n_q_heads < 1 ||
+      p->head_dim < 2 || p->head_dim % 2 != 0 || p->T < 1)
+    return XKV_ERR_INVALID_ARG;
+  if (p->dtype != XKV_F32 && p->dtype != XKV_BF16) return XKV_ERR_INVALID_ARG;
+  if (p->n_q_heads / p->n_kv_heads > 8 || p->head_dim > 256 || 256 % (p->head_dim / 2) != 0) return XKV_ERR_UNSUPPORTED;
+  return XKV_OK;
+}
+
+xkv_status xkv_dense_workspace_size(const xkv_dense_params* p, size_t* bytes) {
+  if (!bytes) return XKV_ERR_INVALID_ARG;
+  xkv_status s = check_dense(p);
+  if (s != XKV_OK) return s;
+  *bytes = dense_workspace(p);
+  return XKV_OK;
+}
+
+xkv_status xkv_dense_attention_decode(const xkv_dense_params* p, const void* q, const void* K, const void* V, float* out,
+                                      void* workspace, size_t ws_bytes, void* stream) {
+  xkv_status s = check_dense(p);
+  if (s != XKV_OK) return s;
+  if (!q || !K || !V || !out || !aligned16(q) || !aligned16(K) || !aligned16(V) || !aligned16(out))
+    return XKV_ERR_INVALID_ARG;
+  if (!workspace || ws_bytes < dense_workspace(p) || !aligned256(workspace)) return XKV_ERR_WORKSPACE;
+  return dense_launch(p, q, K, V, out, workspace, static_cast<cudaStream_t>(stream));
+}
+
+// ------------------------------------------------------------------- NER
+xkv_status xkv_ner_workspace_size(int n, int block, size_t* bytes) {
+  if (!bytes || n < 2 || block < 2 || block % 2 != 0 || n % block != 0) return XKV_ERR_INVALID_ARG;
+  *bytes = ner_workspace(n, block);
+  return XKV_OK;
+}
+
+xkv_status xkv_ner(const float* gram, int n, int block, double rank_rel_tol, float* ner_out, float* erank_out,
+                   int32_t* rank_out, void* workspace, size_t ws_bytes, void* stream) {
+  if (!gram || !ner_out || !aligned16(gram) || n < 2 || block < 2 || block % 2 != 0 || n % block != 0)
+    return XKV_ERR_INVALID_ARG;
+  if (!(rank_rel_tol >= 0.0) || !(rank_rel_tol < 1.0)) return XKV_ERR_INVALID_ARG;
+  if (!workspace || ws_bytes < ner_workspace(n, block) || !aligned256(workspace)) return XKV_ERR_WORKSPACE;
+  return ner_launch(gram, n, block, rank_rel_tol, ner_out, erank_out, rank_out, workspace,
+                    static_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"

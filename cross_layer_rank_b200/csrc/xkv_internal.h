@@ -1,0 +1,80 @@
+// Host-side launchers shared between the C-ABI layer and the kernel files.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/xkv.h"
+
+namespace xkv {
+
+constexpr size_t kAlign = 256;
+inline size_t align_up(size_t x, size_t a = kAlign) { return (x + a - 1) / a * a; }
+
+// Per-device status word (device address), created on first use.
+int* device_status_ptr();
+int num_sms();
+bool force_simt();
+
+// TMA descriptor creation through the driver entry point.
+bool make_tmap(CUtensorMap* map, CUtensorMapDataType dt, int rank, const void* base, const uint64_t* dims,
+               const uint64_t* strides_bytes, const uint32_t* box, CUtensorMapSwizzle swz);
+
+// ------------------------------------------------------------ SR decode
+struct SRPlan {
+  int units;        // B * Hkv
+  int tiles_per_unit;
+  int total_tiles;
+  int ctas;         // attention CTAs (persistent ranges of tiles)
+  int max_units_per_cta;
+  bool tc;          // tcgen05 path
+  size_t off_scores, off_sel, off_part, slot_floats, bytes;
+};
+xkv_status sr_plan(const xkv_sr_params* p, SRPlan* plan);
+xkv_status sr_launch(const xkv_sr_params* p, const SRPlan& plan, const void* q, const void* A_K,
+                     const void* Bt_K, const void* A_V, const void* Bt_V, const void* landmarks,
+                     const void* sr_K, const void* sr_V, float* out, int32_t* sel_out, void* ws,
+                     cudaStream_t st);
+
+// --------------------------------------------------------- dense / recon
+size_t dense_workspace(const xkv_dense_params* p);
+xkv_status dense_launch(const xkv_dense_params* p, const void* q, const void* K, const void* V, float* out,
+                        void* ws, cudaStream_t st);
+xkv_status recon_launch(const void* A, const void* Bt, int64_t T, int rank, int d, int hkv, int hd,
+                        int apply_rope, float theta, xkv_dtype dt, void* out, cudaStream_t st);
+
+// ------------------------------------------------------------ landmarks
+xkv_status landmarks_launch(const void* K, int64_t T, int64_t ldk, int hkv, int hd, xkv_dtype dt, int chunk,
+                            int sink, int recent, float theta, void* out, cudaStream_t st);
+
+// ---------------------------------------------------------- compression
+size_t gram_workspace(int G, int64_t rows, int d, xkv_dtype dt);
+xkv_status gram_launch(const void* const* X, int G, int64_t rows, int d, int64_t ldx, xkv_dtype dt, float* C,
+                       void* ws, cudaStream_t st);
+struct CompressPlan {
+  int n, b, rank;
+  int64_t shard;
+  size_t off_gram, off_gramws, off_Q, off_Y, off_W, off_H, off_U, off_V, off_lam, off_ord, off_Vr,
+      off_Vt, off_jac, bytes;
+};
+xkv_status compress_plan(int G, int64_t T, int d, int rank, int oversample, int64_t shard_rows, xkv_dtype dt,
+                         CompressPlan* plan);
+xkv_status compress_launch(const CompressPlan& plan, const void* const* X, int G, int64_t T, int d,
+                           int64_t ldx, xkv_dtype dt, int iters, uint64_t seed, void* A, void* Bt,
+                           float* eigvals, float* gram_out, void* ws, cudaStream_t st);
+
+// ------------------------------------------------------------------ NER
+size_t ner_workspace(int n, int block);
+xkv_status ner_launch(const float* gram, int n, int block, double tol, float* ner, float* erank, int32_t* rank,
+                      void* ws, cudaStream_t st);
+
+// Symmetric eigen-solver shared by Rayleigh-Ritz and NER (one-sided block Jacobi,
+// fp64).  Operates on `count` independent n x n problems stored column-major
+// at W (+ count * n * n each); V (optional) receives eigenvectors; lam the
+// eigenvalues (unsorted, |lambda| from column norms).
+size_t jacobi_workspace(int n, int count);
+xkv_status jacobi_launch(double* W, double* V, double* lam, int n, int count, void* ws, cudaStream_t st);
+
+}  // namespace xkv

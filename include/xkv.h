@@ -1,0 +1,203 @@
+/*
+ * xkv.h -- C ABI of the B200 (sm_100a) xKV hot path.
+ *
+ * The library computes, on one GPU, the two halves of xKV:
+ *   - prefill-time cross-layer factorisation of a group of G adjacent layers
+ *     (Gram -> top-r subspace -> shared basis A and per-layer B_l) and KV-CoRE's
+ *     normalised effective rank from the same Gram;
+ *   - decode-time Selective Reconstruction (SR) attention: landmark-guided top-k
+ *     chunk selection, reconstruction of only the selected rows, RoPE, and
+ *     online-softmax GQA attention over them plus a raw sink/recent window.
+ *
+ * Sources (page title -- section):
+ *   [xKV-blog] "xKV大模型压缩秘籍：跨层共享，小白也能轻松上手，收藏必备！" --
+ *              "xKV 到底做了什么？" and "仅仅压缩还不够，xKV 还做了“选择性重建”";
+ *              Fig. 6 (full reconstruction vs selective reconstruction).
+ *   [xKV-abs]  "xKV: Cross-Layer KV-Cache Compression via Aligned Singular Vector
+ *              Extraction" -- abstract.
+ *   [KV-CoRE]  "KV-CoRE: Benchmarking Data-Dependent Low-Rank Compressibility of
+ *              KV-Caches in LLMs" -- 2.A (incremental covariance), 2.B (NER).
+ *   [KQ-SVD]   "KQ-SVD: KV cache compression with provable guarantees on attention
+ *              fidelity" -- 3.2 (decode attention), 3.3 (truncated SVD).
+ *
+ * Conventions shared by every call:
+ *   - Every data pointer is a DEVICE pointer owned by the caller, 16-byte
+ *     aligned; the library never allocates device memory.  Scratch space is a
+ *     caller-provided `workspace` whose size the matching *_workspace_size()
+ *     call reports (256-byte alignment required).
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Calls only
+ *     enqueue work; they return before the GPU finishes.
+ *   - Matrices are row-major; sizes are in elements.  bf16 data is IEEE
+ *     bfloat16; f32 data is IEEE binary32.  Outputs of attention are f32.
+ *   - Errors: each call returns an xkv_status.  On XKV_ERR_INVALID_ARG /
+ *     XKV_ERR_UNSUPPORTED / XKV_ERR_WORKSPACE nothing was launched and nothing
+ *     was written.  XKV_ERR_CUDA means a launch or runtime call failed.  Errors
+ *     detected on the device (a bounded wait that expired, a non-finite or
+ *     non-positive pivot) are recorded in a per-device status word that
+ *     xkv_get_device_status() returns and clears.  No C++ exception crosses
+ *     this interface.
+ *   - Compressed-cache layout: A is T x r per (batch, group); B_l is stored
+ *     TRANSPOSED, Bt_l = d x r (row c holds the r coefficients of output column
+ *     c), which for layer l of a group equals rows l d .. l d + d - 1 of V_r.
+ *   - RoPE is rotate-half: pairs (j, j + hd/2) turn by pos * theta^(-2j/hd).
+ *     Token t of the cache sits at position t; the decode query sits at T.
+ */
+#ifndef XKV_H_
+#define XKV_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define XKV_API __attribute__((visibility("default")))
+#else
+#define XKV_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum xkv_status {
+  XKV_OK = 0,
+  XKV_ERR_INVALID_ARG = 1,    /* null pointer, misalignment, inconsistent sizes */
+  XKV_ERR_UNSUPPORTED = 2,    /* valid request outside what this build implements */
+  XKV_ERR_WORKSPACE = 3,      /* workspace missing or smaller than required */
+  XKV_ERR_CUDA = 4,           /* a CUDA runtime/driver call failed */
+  XKV_ERR_NUMERICAL = 5,      /* device detected a numerical breakdown */
+  XKV_ERR_DEVICE_TIMEOUT = 6  /* a bounded device-side wait expired */
+} xkv_status;
+
+typedef enum xkv_dtype { XKV_F32 = 0, XKV_BF16 = 1 } xkv_dtype;
+
+/* Static description of a status code (never NULL). */
+XKV_API const char* xkv_status_string(xkv_status status);
+
+/* Library ABI version: (major << 16) | minor. */
+XKV_API int xkv_version(void);
+
+/* Synchronises `stream`, then returns and clears the calling device's deferred
+ * status word (XKV_OK if no device-side error was recorded). */
+XKV_API xkv_status xkv_get_device_status(void* stream);
+
+/* ------------------------------------------------------------------ Gram */
+/* [KV-CoRE] 2.A incremental covariance over the horizontal concatenation of
+ * [xKV-blog] "xKV 到底做了什么":  C += X^T X,  X = [X_1 | ... | X_G] (rows x G d).
+ *   X_layers : host array of G device pointers; X_layers[l] is rows x d with row
+ *              stride ldx (elements, >= d, multiple of 8).
+ *   C        : (G d) x (G d) f32, accumulated in place (zero it before the first
+ *              shard).  Both triangles are written.
+ *   d must be a multiple of 64.  Workspace: xkv_gram_workspace_size(). */
+XKV_API xkv_status xkv_gram_workspace_size(int G, int64_t rows, int d, xkv_dtype dt, size_t* bytes);
+XKV_API xkv_status xkv_gram_accumulate(const void* const* X_layers, int G, int64_t rows, int d, int64_t ldx,
+                               xkv_dtype dt, float* C, void* workspace, size_t ws_bytes, void* stream);
+
+/* --------------------------------------------------------- compression */
+/* Cross-layer factorisation of one group ([xKV-blog] "xKV 到底做了什么",
+ * [xKV-abs]; optimality of the truncation: [KQ-SVD] 3.3):
+ *   1. C = X^T X accumulated over token shards of `shard_rows` rows;
+ *   2. top-r subspace of C: `iters` block subspace iterations Y = C Q, Q = qr(Y)
+ *      with block width b = min(rank + oversample, G d, T), started from a
+ *      Gaussian block drawn from `seed`; then Rayleigh-Ritz: H = Q^T C Q,
+ *      H = U diag(lambda) U^T, V_r = Q U[:, 1..rank];
+ *   3. A = X V_r (T x rank) and Bt = V_r ((G d) x rank; layer l = rows l d..).
+ * Arguments: X_layers as for xkv_gram_accumulate (T rows each); A (T x rank) and
+ * Bt (G d x rank) in `dt`; eigvals (rank f32, descending Ritz values) and
+ * gram_out ((G d)^2 f32, the full Gram, e.g. for xkv_ner) may be NULL.
+ * Requires d % 64 == 0, rank % 16 == 0, 1 <= rank <= min(T, G d), iters >= 1. */
+XKV_API xkv_status xkv_compress_workspace_size(int G, int64_t T, int d, int rank, int oversample,
+                                       int64_t shard_rows, xkv_dtype dt, size_t* bytes);
+XKV_API xkv_status xkv_compress_group(const void* const* X_layers, int G, int64_t T, int d, int64_t ldx,
+                              xkv_dtype dt, int rank, int iters, int oversample, int64_t shard_rows,
+                              uint64_t seed, void* A, void* Bt, float* eigvals, float* gram_out,
+                              void* workspace, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------ landmarks */
+/* Chunk landmarks for the top-k selector of [xKV-blog] "选择性重建": for KV head
+ * h and middle chunk c (tokens sink + c chunk .. sink + (c+1) chunk - 1),
+ *   landmark[h][c] = mean over the chunk of RoPE_t(K[t, h hd : (h+1) hd]).
+ *   K         : T x (n_kv_heads head_dim) pre-RoPE keys, row stride ldk.
+ *   landmarks : [n_kv_heads][n_mid][head_dim] in `dt`, n_mid = (T-sink-recent)/chunk.
+ * Requires (T - sink - recent) % chunk == 0 and head_dim even. */
+XKV_API xkv_status xkv_build_landmarks(const void* K, int64_t T, int64_t ldk, int n_kv_heads, int head_dim,
+                               xkv_dtype dt, int chunk, int sink, int recent, float rope_theta,
+                               void* landmarks, void* stream);
+
+/* ------------------------------------------------------------ SR decode */
+typedef struct xkv_sr_params {
+  int batch;              /* B */
+  int n_q_heads;          /* Hq (multiple of n_kv_heads) */
+  int n_kv_heads;         /* Hkv */
+  int head_dim;           /* hd (even) */
+  int64_t T;              /* cached tokens; the query sits at position T */
+  int rank_k, rank_v;     /* columns of A_K, A_V */
+  int chunk;              /* tokens per chunk */
+  int topk;               /* chunks kept per (batch, KV head), <= n_mid */
+  int sink, recent;       /* raw windows [0, sink) and [T - recent, T) */
+  float rope_theta;
+  xkv_dtype dtype;        /* of q, A, Bt, landmarks, sink/recent */
+  int64_t a_k_batch_stride, a_v_batch_stride;   /* elements between batches of A_K / A_V */
+  int64_t bt_k_batch_stride, bt_v_batch_stride; /* elements between batches of Bt_K / Bt_V;
+                                                   0 = one Bt shared by the batch */
+} xkv_sr_params;
+
+/* One decode step of xKV-SR for one layer ([xKV-blog] "选择性重建", [xKV-abs];
+ * attention as in [KQ-SVD] 3.2), for every (batch b, KV head h):
+ *   s_c = sum_{g in group(h)} q_g . landmark[b][h][c]; keep the top-k chunks
+ *   (ties -> lower c; sel_out ascending);  rebuild rows t of the kept chunks:
+ *   K_t = RoPE_t(A_K[b][t] Bt_K[h hd : (h+1) hd]^T),  V_t = A_V[b][t] Bt_V[...]^T;
+ *   o_g = softmax(q_g K^T / sqrt(hd)) V over sink, kept and recent rows.
+ *   q         : [B][Hq][hd] post-RoPE queries (query head j uses KV head j/(Hq/Hkv)).
+ *   A_K, A_V  : [B][T][rank] (batch strides in params).   Bt_K, Bt_V : [d][rank] per
+ *               batch element (batch strides in params; each sequence has its own
+ *               factorisation, or 0 to share one).
+ *   landmarks : [B][Hkv][n_mid][hd].   sr_K, sr_V : [B][sink+recent][d]; row i < sink
+ *               is token i, row sink + i is token T - recent + i; keys pre-RoPE.
+ *   out       : [B][Hq][hd] f32.   sel_out : [B][Hkv][topk] int32, or NULL. */
+XKV_API xkv_status xkv_sr_workspace_size(const xkv_sr_params* p, size_t* bytes);
+XKV_API xkv_status xkv_sr_attention_decode(const xkv_sr_params* p, const void* q, const void* A_K,
+                                   const void* Bt_K, const void* A_V, const void* Bt_V,
+                                   const void* landmarks, const void* sr_K, const void* sr_V,
+                                   float* out, int32_t* sel_out, void* workspace, size_t ws_bytes,
+                                   void* stream);
+
+/* -------------------------------------------------- full reconstruction */
+/* The comparison path of [xKV-blog] Fig. 6: rebuild every row,
+ *   out[t][c] = sum_i A[t][i] Bt[c][i]   (T x d, `dt`),
+ * then, if apply_rope, RoPE per head at position t.  A is T x rank, Bt d x rank.
+ * Requires rank % 16 == 0 and d % head_dim == 0. */
+XKV_API xkv_status xkv_full_reconstruct(const void* A, const void* Bt, int64_t T, int rank, int d,
+                                int n_kv_heads, int head_dim, int apply_rope, float rope_theta,
+                                xkv_dtype dt, void* out, void* stream);
+
+/* Dense decode attention over a full cache ([KQ-SVD] 3.2), the second half of
+ * the comparison path:  o_g = softmax(q_g K^T / sqrt(hd)) V over all T rows.
+ *   q [B][Hq][hd], K (post-RoPE) and V [B][T][d] in `dtype`, out [B][Hq][hd] f32. */
+typedef struct xkv_dense_params {
+  int batch, n_q_heads, n_kv_heads, head_dim;
+  int64_t T;
+  xkv_dtype dtype;
+} xkv_dense_params;
+XKV_API xkv_status xkv_dense_workspace_size(const xkv_dense_params* p, size_t* bytes);
+XKV_API xkv_status xkv_dense_attention_decode(const xkv_dense_params* p, const void* q, const void* K,
+                                      const void* V, float* out, void* workspace, size_t ws_bytes,
+                                      void* stream);
+
+/* ------------------------------------------------------------------ NER */
+/* [KV-CoRE] 2.B per diagonal block C_ll (block x block) of an n x n f32 Gram:
+ * eigenvalues lambda, numerical rank r = #{lambda_i > rank_rel_tol lambda_max},
+ * sigma_i = sqrt(lambda_i) over those r, p_i = sigma_i / sum sigma,
+ * erank = exp(-sum p_i ln p_i), NER = erank / r (in [1/r, 1]).  A block with
+ * lambda_max <= 0 reports rank 0, erank 0, NER 0.
+ *   ner_out [n/block] f32; erank_out [n/block] f32 or NULL; rank_out [n/block]
+ *   int32 or NULL.  Requires n % block == 0, block even. */
+XKV_API xkv_status xkv_ner_workspace_size(int n, int block, size_t* bytes);
+XKV_API xkv_status xkv_ner(const float* gram, int n, int block, double rank_rel_tol, float* ner_out,
+                   float* erank_out, int32_t* rank_out, void* workspace, size_t ws_bytes,
+                   void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* XKV_H_ */

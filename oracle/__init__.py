@@ -182,7 +182,8 @@ def sr_decode(w, q, A_K, Bt_K, A_V, Bt_V, landmarks, sr_K, sr_V, T: Optional[int
               sel_in=None, units: Optional[Sequence[int]] = None):
     """One Selective-Reconstruction decode step (fp64).
 
-    w: a synth.Workload (shape fields).  Returns (out [B][Hq][hd], sel [B][Hkv][k],
+    w: a synth.Workload (shape fields).  Bt_K / Bt_V are [d][r] (shared by the
+    batch) or [B][d][r] (one factorisation per sequence).  Returns (out [B][Hq][hd], sel [B][Hkv][k],
     scores [B][Hkv][n_mid]).  Rows of units not listed are NaN / -1.
     """
     T = T or w.T
@@ -196,8 +197,11 @@ def sr_decode(w, q, A_K, Bt_K, A_V, Bt_V, landmarks, sr_K, sr_V, T: Optional[int
     scores = np.full((B, w.n_kv_heads, n_mid), np.nan, dtype=np.float64)
     si = None if sel_in is None else np.ascontiguousarray(sel_in, dtype=np.int32)
     u = None if units is None else np.ascontiguousarray(units, dtype=np.int32)
-    rc = lib().xo_sr_decode(C.byref(p), _p(q), _p(A_K), C.c_int64(T * A_K.shape[-1]), _p(Bt_K),
-                            _p(A_V), C.c_int64(T * A_V.shape[-1]), _p(Bt_V), _p(lm), _p(sr_K), _p(sr_V),
+    sbk = Bt_K.shape[-2] * Bt_K.shape[-1] if Bt_K.ndim == 3 else 0
+    sbv = Bt_V.shape[-2] * Bt_V.shape[-1] if Bt_V.ndim == 3 else 0
+    rc = lib().xo_sr_decode(C.byref(p), _p(q), _p(A_K), C.c_int64(T * A_K.shape[-1]), _p(Bt_K), C.c_int64(sbk),
+                            _p(A_V), C.c_int64(T * A_V.shape[-1]), _p(Bt_V), C.c_int64(sbv), _p(lm), _p(sr_K),
+                            _p(sr_V),
                             None if si is None else _p(si), None if u is None else _p(u),
                             C.c_int(0 if u is None else u.size), _p(out), _p(sel), _p(scores))
     if rc != 0:

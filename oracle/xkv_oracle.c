@@ -427,12 +427,14 @@ static int xo_cmp_i32(const void* a, const void* b) {
  *      (B_K restricted to head h's hd columns; Bt stores B transposed);
  *   4. raw sink rows [0, sink) and recent rows [T - recent, T) (RoPE on K);
  *   5. o_g = softmax(q_g K^T / sqrt(hd)) V over sink, kept and recent rows.
- * Shapes: q [B][Hq][hd]; A_K [B][T][rK] (batch stride sak); Bt_K [d][rK];
- * A_V [B][T][rV] (sav); Bt_V [d][rV]; lm [B][Hkv][n_mid][hd]; srK, srV
+ * Shapes: q [B][Hq][hd]; A_K [B][T][rK] (batch stride sak); Bt_K [B][d][rK]
+ * (batch stride sbk; 0 = one Bt for the batch); A_V [B][T][rV] (sav); Bt_V
+ * [B][d][rV] (sbv); lm [B][Hkv][n_mid][hd]; srK, srV
  * [B][sink+recent][d]; out [B][Hq][hd]; sel_out [B][Hkv][k];
  * scores_out [B][Hkv][n_mid] (optional). */
 XO_EXPORT int xo_sr_decode(const xo_sr_params* p, const float* q, const float* A_K, int64_t sak,
-                           const float* Bt_K, const float* A_V, int64_t sav, const float* Bt_V,
+                           const float* Bt_K, int64_t sbk, const float* A_V, int64_t sav, const float* Bt_V,
+                           int64_t sbv,
                            const float* lm, const float* srK, const float* srV,
                            const int32_t* sel_in, const int32_t* units, int n_units, double* out,
                            int32_t* sel_out, double* scores_out) {
@@ -488,8 +490,8 @@ XO_EXPORT int xo_sr_decode(const xo_sr_params* p, const float* q, const float* A
         const float* ak = A_K + b * sak + t * rK;
         const float* av = A_V + b * sav + t * rV;
         for (int j = 0; j < hd; ++j) {
-          const float* bk = Bt_K + (int64_t)(h * hd + j) * rK;
-          const float* bv = Bt_V + (int64_t)(h * hd + j) * rV;
+          const float* bk = Bt_K + b * sbk + (int64_t)(h * hd + j) * rK;
+          const float* bv = Bt_V + b * sbv + (int64_t)(h * hd + j) * rV;
           double sk = 0.0, sv = 0.0;
           for (int a = 0; a < rK; ++a) sk += (double)ak[a] * (double)bk[a];
           for (int a = 0; a < rV; ++a) sv += (double)av[a] * (double)bv[a];

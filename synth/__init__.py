@@ -322,7 +322,8 @@ def compressed_cache(w: Workload, layer: int, T: Optional[int] = None):
     """Stand-ins for a compressed layer, drawn directly (decode-only tests).
 
     Returns dict with A_K [B][T][rK], A_V [B][T][rV] (columns scaled like U*Sigma
-    of the synthetic spectrum), Bt_K [d][rK], Bt_V [d][rV] (rows ~ N(0, 1/r)),
+    of the synthetic spectrum), Bt_K [B][d][rK], Bt_V [B][d][rV] (one per
+    sequence, entries ~ N(0, 1/r)),
     landmarks [B][Hkv][n_mid][hd] (~ N(0,1)), sink/recent K and V [B][s+w][d],
     and q [B][Hq][hd]; all float32 in storage precision.
     """
@@ -334,7 +335,7 @@ def compressed_cache(w: Workload, layer: int, T: Optional[int] = None):
         A = normal_chunked(stream_key(w.name, "A", kind, layer, T), w.batch * T * r)
         A = A.reshape(w.batch, T, r) * sc[None, None, :].astype(np.float32)
         out["A_" + kind] = to_storage(A, w.dtype)
-        Bt = normal(stream_key(w.name, "B", kind, layer), w.d * r).reshape(w.d, r) / math.sqrt(r)
+        Bt = normal(stream_key(w.name, "B", kind, layer), w.batch * w.d * r).reshape(w.batch, w.d, r) / math.sqrt(r)
         out["Bt_" + kind] = to_storage(Bt, w.dtype)
     L = normal_chunked(stream_key(w.name, "L", layer, T), w.batch * w.n_kv_heads * n_mid * w.head_dim)
     out["landmarks"] = to_storage(L.reshape(w.batch, w.n_kv_heads, n_mid, w.head_dim), w.dtype)

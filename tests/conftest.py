@@ -27,3 +27,20 @@ def pytest_collection_modifyitems(config, items):
     for it in items:
         if "gpu" in it.keywords:
             it.add_marker(skip)
+
+
+def build_xkv():
+    """Build libxkv.so (if stale) without importing the package, then import it."""
+    import importlib.util
+    path = os.path.join(ROOT, "cross_layer_rank_b200", "build.py")
+    spec = importlib.util.spec_from_file_location("_xkv_build", path)
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    mod.build()
+    import cross_layer_rank_b200
+    return cross_layer_rank_b200
+
+
+@pytest.fixture(scope="session")
+def xkv():
+    return build_xkv()

@@ -1,0 +1,97 @@
+"""The C-ABI library loads, exports every symbol include/xkv.h declares, and
+rejects bad arguments on the host (no GPU needed: validation happens before any
+CUDA call and nothing is launched)."""
+import ctypes as C
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "xkv.h")
+
+
+def _declared():
+    src = open(HEADER).read()
+    return sorted(set(re.findall(r"XKV_API\s+[\w\s\*]+?\b(xkv_\w+)\s*\(", src)))
+
+
+def test_header_declares_the_five_hot_path_calls():
+    names = _declared()
+    for n in ("xkv_compress_group", "xkv_build_landmarks", "xkv_sr_attention_decode", "xkv_full_reconstruct",
+              "xkv_ner"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(xkv):
+    lib = C.CDLL(xkv.LIB_PATH)
+    for n in _declared():
+        assert hasattr(lib, n), n
+    assert set(_declared()) == set(xkv.EXPORTS)
+
+
+def test_status_strings_and_version(xkv):
+    for s in range(7):
+        assert xkv.status_string(s)
+    assert xkv.lib.xkv_version() >> 16 == 1
+
+
+def _sr(xkv, **kw):
+    base = dict(batch=1, n_q_heads=8, n_kv_heads=2, head_dim=64, T=1024, rank_k=64, rank_v=64, chunk=8, topk=16,
+                sink=8, recent=32, rope_theta=500000.0)
+    base.update(kw)
+    import torch
+    return xkv.sr_params(dtype=torch.float32, **base)
+
+
+@pytest.mark.parametrize("bad", [dict(topk=124), dict(T=1027), dict(n_q_heads=7), dict(chunk=0), dict(rank_k=0),
+                                 dict(rope_theta=0.0), dict(head_dim=63), dict(batch=0)])
+def test_sr_rejects_bad_shapes(xkv, bad):
+    p = _sr(xkv, **bad)
+    n = C.c_size_t(0)
+    assert xkv.lib.xkv_sr_workspace_size(C.byref(p), C.byref(n)) == xkv.XKV_ERR_INVALID_ARG
+    z = None
+    assert xkv.lib.xkv_sr_attention_decode(C.byref(p), z, z, z, z, z, z, z, z, z, z, z, 0, z) == \
+        xkv.XKV_ERR_INVALID_ARG
+
+
+def test_sr_rejects_null_and_misaligned_pointers_and_small_workspace(xkv):
+    p = _sr(xkv)
+    n = C.c_size_t(0)
+    assert xkv.lib.xkv_sr_workspace_size(C.byref(p), C.byref(n)) == xkv.XKV_OK and n.value > 0
+    fake = C.c_void_p(1 << 20)  # aligned, never dereferenced: validation fails first
+    mis = C.c_void_p((1 << 20) + 4)
+    args = [fake] * 9
+    assert xkv.lib.xkv_sr_attention_decode(C.byref(p), None, *args[1:], None, None, 0, None) == \
+        xkv.XKV_ERR_INVALID_ARG
+    assert xkv.lib.xkv_sr_attention_decode(C.byref(p), mis, *args[1:], None, None, 0, None) == \
+        xkv.XKV_ERR_INVALID_ARG
+    assert xkv.lib.xkv_sr_attention_decode(C.byref(p), *args, None, fake, 16, None) == xkv.XKV_ERR_WORKSPACE
+
+
+def test_compress_and_gram_validation(xkv):
+    n = C.c_size_t(0)
+    assert xkv.lib.xkv_compress_workspace_size(4, 1024, 128, 64, 64, 8192, xkv.XKV_F32, C.byref(n)) == xkv.XKV_OK
+    assert n.value > 4 * 128 * 4 * 128 * 4
+    # rank above G d, rank not a multiple of 16, d not a multiple of 64, G > 8
+    for args in ((1, 1024, 128, 256), (4, 1024, 128, 40), (4, 1024, 96, 64), (9, 1024, 64, 64)):
+        assert xkv.lib.xkv_compress_workspace_size(*args, 64, 0, xkv.XKV_F32, C.byref(n)) == xkv.XKV_ERR_INVALID_ARG
+    # bf16 needs rank % 64 == 0
+    assert xkv.lib.xkv_compress_workspace_size(4, 1024, 128, 48, 64, 0, xkv.XKV_BF16, C.byref(n)) == \
+        xkv.XKV_ERR_UNSUPPORTED
+    ptrs = (C.c_void_p * 2)(None, None)
+    assert xkv.lib.xkv_gram_accumulate(ptrs, 2, 100, 64, 64, xkv.XKV_F32, C.c_void_p(1 << 20), None, 0, None) == \
+        xkv.XKV_ERR_INVALID_ARG
+
+
+def test_landmarks_recon_dense_ner_validation(xkv):
+    fake = C.c_void_p(1 << 20)
+    assert xkv.lib.xkv_build_landmarks(fake, 1027, 128, 2, 64, xkv.XKV_F32, 8, 8, 32, 5e5, fake, None) == \
+        xkv.XKV_ERR_INVALID_ARG
+    assert xkv.lib.xkv_full_reconstruct(fake, fake, 100, 64, 128, 2, 32, 1, 5e5, xkv.XKV_F32, fake, None) == \
+        xkv.XKV_ERR_INVALID_ARG  # Hkv * hd != d
+    bad = xkv.DenseParams(1, 6, 4, 64, 100, xkv.XKV_F32)
+    n = C.c_size_t(0)
+    assert xkv.lib.xkv_dense_workspace_size(C.byref(bad), C.byref(n)) == xkv.XKV_ERR_INVALID_ARG
+    assert xkv.lib.xkv_ner_workspace_size(100, 30, C.byref(n)) == xkv.XKV_ERR_INVALID_ARG
+    assert xkv.lib.xkv_ner(fake, 128, 64, 1e-9, fake, None, None, None, 0, None) == xkv.XKV_ERR_WORKSPACE

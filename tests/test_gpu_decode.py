@@ -1,0 +1,104 @@
+"""GPU parity: one SR decode step (xkv_sr_attention_decode) against the oracle on
+identical seeded inputs.
+
+Selection: the GPU's top-k set must equal the exact one except chunks whose
+score lies within 1e-3 (relative) of the k-th score.  Output: max-abs error
+<= 1e-2 against the oracle run on the GPU's own (valid) selection; the f32
+path is held to 2e-4.  Shapes cover the tiny f32 workload, small bf16 cases on
+the tensor-core path (ragged last tile, GQA group of 7, every chunk kept) and,
+at full size, one layer launch of the Llama-3.1-8B group (16K), the 32-layer
+Llama-3.1-8B shape (64K, batch 4, sampled units) and the Qwen2.5-7B shape
+(128K, batch 2).
+"""
+import numpy as np
+import pytest
+
+import oracle
+import synth
+from gpu_helpers import check_selection, host, run_sr, sr_inputs_on_device
+
+pytestmark = pytest.mark.gpu
+
+
+def _parity(xkv, w, layer=0, T=None, units=None, tol=1e-2, inp=None):
+    T = T or w.T
+    inp = inp if inp is not None else synth.compressed_cache(w, layer, T=T)
+    d_inp = sr_inputs_on_device(w, inp)
+    out_g, sel_g = run_sr(xkv, w, d_inp, T=T)
+    out_g, sel_g = host(out_g), sel_g.cpu().numpy()
+    _, sel_o, scores = oracle.sr_decode(w, T=T, units=units, **inp)
+    check_selection(sel_g, scores, w.topk, units=units)
+    ref, _, _ = oracle.sr_decode(w, T=T, sel_in=sel_g, units=units, **inp)
+    B = inp["q"].shape[0]
+    rows = np.zeros((B, w.n_q_heads), dtype=bool)
+    for u in (units if units is not None else range(B * w.n_kv_heads)):
+        b, h = divmod(u, w.n_kv_heads)
+        rows[b, h * w.gq:(h + 1) * w.gq] = True
+    err = np.abs(out_g[rows] - ref[rows]).max()
+    assert np.isfinite(out_g[rows]).all()
+    assert err <= tol, err
+    return err, sel_g
+
+
+def test_sr_tiny_f32(xkv):
+    w = synth.WORKLOADS["tiny_f32"]
+    err, _ = _parity(xkv, w, tol=2e-4)
+
+
+def test_sr_bf16_tensor_core_ragged_tile(xkv):
+    w = synth.Workload("sr_bf16_small", 2, 4, 4, 2, 128, 8, 8 + 32 + 8 * 150, 96, 0.8, 128, 192, topk=37)
+    _parity(xkv, w)
+
+
+def test_sr_bf16_gqa7_single_tile(xkv):
+    w = synth.Workload("sr_bf16_gq7", 1, 4, 4, 2, 128, 14, 8 + 32 + 8 * 100, 96, 1.0, 64, 128, topk=16)
+    _parity(xkv, w)
+
+
+def test_sr_f32_general_shape(xkv):
+    # f32, hd 64, chunk 4, odd ranks: the CUDA-core path
+    w = synth.Workload("sr_f32_general", 2, 4, 4, 3, 64, 6, 5 + 7 + 4 * 90, 48, 0.8, 48, 80, chunk=4, topk=23,
+                       sink=5, recent=7, dtype="f32")
+    _parity(xkv, w, tol=2e-4)
+
+
+def test_sr_every_chunk_kept_equals_dense_attention(xkv):
+    # KQ-SVD page 3.2: with k = n_mid, SR is dense decode attention over the
+    # cache [raw sink | A Bt^T rows | raw recent]
+    w = synth.Workload("sr_all_chunks", 1, 4, 4, 2, 128, 8, 8 + 32 + 8 * 40, 96, 0.8, 64, 64, topk=40)
+    inp = synth.compressed_cache(w, 0)
+    d_inp = sr_inputs_on_device(w, inp)
+    out_g, sel_g = run_sr(xkv, w, d_inp)
+    assert np.array_equal(sel_g.cpu().numpy()[0, 0], np.arange(40))
+    T, hd = w.T, w.head_dim
+    Km = oracle.full_reconstruct(inp["A_K"][0], inp["Bt_K"][0], w.n_kv_heads, hd, True, w.rope_theta)
+    Vm = oracle.full_reconstruct(inp["A_V"][0], inp["Bt_V"][0], w.n_kv_heads, hd, False, w.rope_theta)
+    rows = list(range(w.sink)) + list(range(T - w.recent, T))
+    for i, t in enumerate(rows):
+        for h in range(w.n_kv_heads):
+            sl = slice(h * hd, (h + 1) * hd)
+            Km[t, sl] = oracle.rope(inp["sr_K"][0, i, sl], t, w.rope_theta)
+        Vm[t] = inp["sr_V"][0, i]
+    ref = oracle.dense_decode(inp["q"], Km[None], Vm[None], w.n_kv_heads)
+    assert np.abs(host(out_g) - ref).max() <= 1e-2
+
+
+def test_sr_deterministic(xkv):
+    w = synth.Workload("sr_det", 2, 4, 4, 2, 128, 8, 8 + 32 + 8 * 120, 96, 0.8, 128, 128, topk=40)
+    d_inp = sr_inputs_on_device(w, synth.compressed_cache(w, 0))
+    o1, s1 = run_sr(xkv, w, d_inp)
+    o2, s2 = run_sr(xkv, w, d_inp)
+    assert np.array_equal(host(o1), host(o2)) and np.array_equal(s1.cpu().numpy(), s2.cpu().numpy())
+
+
+def test_sr_full_size_llama_group_16k(xkv):
+    _parity(xkv, synth.WORKLOADS["llama_group_16k"])
+
+
+def test_sr_full_size_llama8b_64k_batch4_layer(xkv):
+    w = synth.WORKLOADS["llama8b_64k_b4"]
+    _parity(xkv, w, layer=5, units=[0, 9, 18, 27, 31])
+
+
+def test_sr_full_size_qwen7b_128k_batch2_layer(xkv):
+    _parity(xkv, synth.WORKLOADS["qwen7b_128k_b2"], layer=3)

@@ -59,9 +59,9 @@ def test_all_chunks_equals_dense_over_rebuilt_cache():
     inp = _inputs(w)
     out, sel, _ = oracle.sr_decode(w, **inp)
     assert np.array_equal(sel[0, 0], np.arange(w.n_mid))
-    Km = np.stack([oracle.full_reconstruct(inp["A_K"][b], inp["Bt_K"], w.n_kv_heads, w.head_dim, True,
+    Km = np.stack([oracle.full_reconstruct(inp["A_K"][b], inp["Bt_K"][b], w.n_kv_heads, w.head_dim, True,
                                            w.rope_theta) for b in range(w.batch)])
-    Vm = np.stack([oracle.full_reconstruct(inp["A_V"][b], inp["Bt_V"], w.n_kv_heads, w.head_dim, False,
+    Vm = np.stack([oracle.full_reconstruct(inp["A_V"][b], inp["Bt_V"][b], w.n_kv_heads, w.head_dim, False,
                                            w.rope_theta) for b in range(w.batch)])
     K, V = _dense_cache(w, inp, Km, Vm)
     ref = oracle.dense_decode(inp["q"], K, V, w.n_kv_heads)
