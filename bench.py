@@ -82,7 +82,7 @@ class Clocks:
         try:
             self.f = open(self.path, "w")
             self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={q}",
-                                          "--format=csv,noheader,nounits", "-lms", "100"], stdout=self.f,
+                                          "--format=csv,noheader,nounits", "-lms", "50"], stdout=self.f,
                                          stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
@@ -134,20 +134,18 @@ def build_model(xkv, w, device, groups=None, log=print):
     for g in range(n_groups):
         AK = torch.empty((B, T, w.rank_k), dtype=bf, device=device)
         AV = torch.empty((B, T, w.rank_v), dtype=bf, device=device)
-        BtK = torch.empty((G * d, w.rank_k), dtype=bf, device=device)
-        BtV = torch.empty((G * d, w.rank_v), dtype=bf, device=device)
+        BtK = torch.empty((B, G * d, w.rank_k), dtype=bf, device=device)
+        BtV = torch.empty((B, G * d, w.rank_v), dtype=bf, device=device)
         lms = [torch.empty((B, w.n_kv_heads, w.n_mid, w.head_dim), dtype=bf, device=device) for _ in range(G)]
         srK = [torch.empty((B, w.sink + w.recent, d), dtype=bf, device=device) for _ in range(G)]
         srV = [torch.empty((B, w.sink + w.recent, d), dtype=bf, device=device) for _ in range(G)]
         for b in range(B):
+            # each sequence of the batch is factorised on its own
             for kind, A, Bt, r in (("K", AK, BtK, w.rank_k), ("V", AV, BtV, w.rank_v)):
                 X = synth.kv_group_torch(w, b, g, kind, device)
                 e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
                 e0.record()
-                # the basis of each batch element is its own; Bt of batch 0 is kept
-                # (every batch element shares the layer weights' geometry here)
-                Bt_b = Bt if b == 0 else torch.empty_like(Bt)
-                xkv.xkv_compress_group(X, r, A[b], Bt_b, iters=8, oversample=synth.oversample(r), shard_rows=8192,
+                xkv.xkv_compress_group(X, r, A[b], Bt[b], iters=8, oversample=synth.oversample(r), shard_rows=8192,
                                        ws=ws)
                 e1.record()
                 e1.synchronize()
@@ -167,11 +165,13 @@ def build_model(xkv, w, device, groups=None, log=print):
         for l in range(G):
             model["A_K"].append(AK)
             model["A_V"].append(AV)
-            model["Bt_K"].append(BtK[l * d:(l + 1) * d])
-            model["Bt_V"].append(BtV[l * d:(l + 1) * d])
+            # per-layer factors [B][d][r] (batch stride d r)
+            model["Bt_K"].append(BtK[:, l * d:(l + 1) * d].contiguous())
+            model["Bt_V"].append(BtV[:, l * d:(l + 1) * d].contiguous())
             model["lm"].append(lms[l])
             model["srK"].append(srK[l])
             model["srV"].append(srV[l])
+        del BtK, BtV
         log(f"group {g + 1}/{n_groups} compressed")
     for layer in range(n_groups * G):
         q = synth.normal_torch(synth.stream_key(w.name, "q", layer), B * w.n_q_heads * w.head_dim, device)
@@ -387,8 +387,8 @@ def run_reference(args, log):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
     ap.add_argument("--workload", default="llama8b_64k_b4", choices=sorted(synth.WORKLOADS))
     ap.add_argument("--batch", type=int, default=0, help="override the batch per GPU")

@@ -30,10 +30,12 @@ namespace {
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kTileChunks = 16;   // chunks of 8 rows per 128-row tile (tcgen05 path)
 constexpr int kMaxGQ = 8;
-constexpr int kKStages = 4;
-constexpr int kVStages = 4;
+constexpr int kKStages = 3;   // key stages: 16 chunks x kKAtoms 64-column atoms
+constexpr int kKAtoms = 2;
+constexpr int kBStages = 2;   // Bt_K atoms (128 rows x 64 columns)
+constexpr int kVStages = 4;   // value stages: 2 chunks x full rank
 constexpr int kAtomBytes = 16384;  // 128 rows x 64 bf16
-constexpr int kAttendThreads = 448;  // 14 warps: TMA, MMA, 4 epilogue, 8 value
+constexpr int kAttendThreads = 480;  // 15 warps: 8 key epilogue, 4 value epilogue, 2 TMA, 1 MMA
 
 // ----------------------------------------------------------------- helpers
 __host__ __device__ inline int tile_begin(int c, int n_tiles, int ctas) {
@@ -107,24 +109,35 @@ __global__ void __launch_bounds__(256) sr_score_kernel(const T* __restrict__ q, 
   const T* base = lm + static_cast<int64_t>(unit) * n_mid * hd;
   float* out = scores + static_cast<int64_t>(unit) * n_mid;
   if (sizeof(T) == 2 && hd == 128) {
-    // 16 lanes x 16 B cover one 256-B landmark row; a warp scores 2 rows per load.
+    // 16 lanes x 16 B cover one 256-B landmark row; a warp scores 2 rows per
+    // load and keeps 8 rows (4 loads per lane) in flight.
     const int half = lane >> 4, hl = lane & 15;
     float qv[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) qv[i] = qbar[hl * 8 + i];
-    for (int64_t c = c0 + warp * 2 + half; c < c1; c += 16) {
-      const uint4 w = *reinterpret_cast<const uint4*>(base + c * 128 + hl * 8);
-      const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
-      float s = 0.f;
+    constexpr int U = 8;
+    for (int64_t cb = c0 + warp * 2 * U; cb < c1; cb += 16 * U) {
+      uint4 w[U];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float2 f = bf2_to_f2(ww[i]);
-        s = fmaf(qv[2 * i], f.x, s);
-        s = fmaf(qv[2 * i + 1], f.y, s);
+      for (int k = 0; k < U; ++k) {
+        const int64_t c = cb + 2 * k + half;
+        w[k] = c < c1 ? *reinterpret_cast<const uint4*>(base + c * 128 + hl * 8) : make_uint4(0, 0, 0, 0);
       }
 #pragma unroll
-      for (int o = 8; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-      if (hl == 0) out[c] = s;
+      for (int k = 0; k < U; ++k) {
+        const uint32_t ww[4] = {w[k].x, w[k].y, w[k].z, w[k].w};
+        float s = 0.f;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float2 f = bf2_to_f2(ww[i]);
+          s = fmaf(qv[2 * i], f.x, s);
+          s = fmaf(qv[2 * i + 1], f.y, s);
+        }
+#pragma unroll
+        for (int o = 8; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+        const int64_t c = cb + 2 * k + half;
+        if (hl == 0 && c < c1) out[c] = s;
+      }
     }
   } else {
     for (int64_t c = c0 + warp; c < c1; c += 8) {
@@ -137,76 +150,162 @@ __global__ void __launch_bounds__(256) sr_score_kernel(const T* __restrict__ q, 
 }
 
 // ------------------------------------------------------------- sr_topk
-// Exact top-k of one unit's chunk scores (1024 threads): radix select of the
-// k-th largest key over 4 passes of 8 bits, then an ordered compaction that
-// keeps every key above it and the lowest-index ties.
-__global__ void __launch_bounds__(1024) sr_topk_kernel(const float* __restrict__ scores, int32_t* __restrict__ sel,
-                                                        int32_t* __restrict__ sel_out, int64_t n_mid, int k) {
-  extern __shared__ uint32_t keys[];
-  __shared__ uint32_t hist[256];
+// Exact top-k of one unit's chunk scores (1024 threads, one CTA per unit).
+//   1. scores -> order-preserving 32-bit keys; their range [lo, hi];
+//   2. a 1024-bucket histogram of floor((key - lo) * 1024 / (hi - lo + 1))
+//      (fp32 arithmetic: a monotone map, so every key of a higher bucket is
+//      larger than every key of a lower one);
+//   3. a suffix scan finds the boundary bucket B holding the k-th largest key;
+//      keys above B are kept, `need` more come from B;
+//   4. the keys of B are compacted in ascending index order and the `need`
+//      largest of them found bit by bit (ties -> lower index);
+//   5. an ordered compaction writes the selection ascending by chunk.
+// Thread t owns the contiguous index segment [t per, (t+1) per), stored
+// transposed (element j of every thread's segment is contiguous) so that the
+// segment loops are free of shared-memory bank conflicts.
+constexpr int kTopkThreads = 1024;
+constexpr int kBuckets = 1024;
+
+__device__ __forceinline__ uint32_t topk_bucket(uint32_t key, uint32_t lo, float scale) {
+  const float x = static_cast<float>(key - lo) * scale;
+  return min(static_cast<uint32_t>(x), static_cast<uint32_t>(kBuckets - 1));
+}
+
+__global__ void __launch_bounds__(kTopkThreads) sr_topk_kernel(const float* __restrict__ scores, int32_t* __restrict__ sel,
+                                                               int32_t* __restrict__ sel_out, int64_t n_mid, int k) {
+  extern __shared__ uint32_t ksm[];  // [per][1024] keys (transposed), then [n] candidate indices
+  __shared__ uint32_t hist[kBuckets];
   __shared__ uint32_t warp_tot[32];
-  __shared__ uint32_t s_digit, s_kk, s_total;
+  __shared__ uint32_t s_wcnt[3 * 64];
+  __shared__ uint32_t s_lo, s_hi, s_total, s_bucket, s_need;
   const int unit = blockIdx.x;
   const int n = static_cast<int>(n_mid);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int nt = static_cast<int>(blockDim.x), nwarps = nt >> 5;
+  const int per = (n + nt - 1) / nt;
+  uint32_t* ckey = ksm + per * nt;
   const float* sc = scores + static_cast<int64_t>(unit) * n_mid;
-  for (int i = threadIdx.x; i < n; i += blockDim.x) keys[i] = order_key(sc[i]);
-  uint32_t prefix = 0, pmask = 0;
-  if (threadIdx.x == 0) s_kk = static_cast<uint32_t>(k);
-  for (int shift = 24; shift >= 0; shift -= 8) {
-    for (int i = threadIdx.x; i < 256; i += blockDim.x) hist[i] = 0;
-    __syncthreads();
-    for (int i = threadIdx.x; i < n; i += blockDim.x) {
-      const uint32_t key = keys[i];
-      if ((key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
-    }
-    __syncthreads();
-    if (threadIdx.x < 32) {
-      // lane l owns digits 255-8l .. 248-8l (descending)
-      const int lane = threadIdx.x;
-      uint32_t loc = 0;
-      for (int i = 0; i < 8; ++i) loc += hist[255 - 8 * lane - i];
-      uint32_t incl = loc;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += y;
-      }
-      const uint32_t kk = s_kk;
-      const uint32_t excl = incl - loc;
-      const bool mine = excl < kk && incl >= kk;
-      const uint32_t ballot = __ballot_sync(0xffffffffu, mine);
-      if (mine) {
-        uint32_t cum = excl;
-        int dsel = 255 - 8 * lane;
-        for (int i = 0; i < 8; ++i) {
-          const int dgt = 255 - 8 * lane - i;
-          if (cum + hist[dgt] >= kk) { dsel = dgt; break; }
-          cum += hist[dgt];
-        }
-        s_digit = static_cast<uint32_t>(dsel);
-        s_kk = kk - cum;
-      }
-      (void)ballot;
-    }
-    __syncthreads();
-    prefix |= s_digit << shift;
-    pmask |= 255u << shift;
+  // 1. keys and their range
+  uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
+  for (int j = 0; j < per; ++j) {
+    const int i = tid * per + j;
+    const uint32_t key = i < n ? order_key(sc[i]) : 0u;
+    ksm[j * nt + tid] = key;
+    if (i < n) { kmin = min(kmin, key); kmax = max(kmax, key); }
   }
-  const uint32_t tau = prefix;     // key of the k-th largest score
-  const uint32_t need_eq = s_kk;   // how many keys equal to tau are kept
-  // ordered compaction over contiguous per-thread segments
-  const int per = (n + blockDim.x - 1) / blockDim.x;
-  const int i0 = min(n, static_cast<int>(threadIdx.x) * per), i1 = min(n, i0 + per);
+  hist[tid] = 0u;
+  if (tid == 0) { s_lo = 0xFFFFFFFFu; s_hi = 0u; }
+  __syncthreads();
+  kmin = __reduce_min_sync(0xffffffffu, kmin);
+  kmax = __reduce_max_sync(0xffffffffu, kmax);
+  if (lane == 0) { atomicMin(&s_lo, kmin); atomicMax(&s_hi, kmax); }
+  __syncthreads();
+  const uint32_t lo = s_lo;
+  const float scale = static_cast<float>(kBuckets) / (static_cast<float>(s_hi - lo) + 1.0f);
+  const int i0 = tid * per, cnt = max(0, min(per, n - i0));
+  // 2. histogram
+  for (int j = 0; j < cnt; ++j) atomicAdd(&hist[topk_bucket(ksm[j * nt + tid], lo, scale)], 1u);
+  __syncthreads();
+  // 3. suffix scan: thread t owns bucket kBuckets - 1 - t
+  {
+    const uint32_t hv = hist[kBuckets - 1 - tid];
+    const uint32_t excl = block_exclusive_scan(hv, warp_tot, &s_total);  // keys in higher buckets
+    if (excl < static_cast<uint32_t>(k) && excl + hv >= static_cast<uint32_t>(k)) {
+      s_bucket = kBuckets - 1 - tid;
+      s_need = static_cast<uint32_t>(k) - excl;
+    }
+  }
+  __syncthreads();
+  const uint32_t B = s_bucket, need = s_need;
+  // 4. candidates of the boundary bucket (their keys, ascending index)
+  uint32_t nc = 0;
+  for (int j = 0; j < cnt; ++j) nc += topk_bucket(ksm[j * nt + tid], lo, scale) == B;
+  uint32_t cpos = block_exclusive_scan(nc, warp_tot, &s_total);
+  const uint32_t m = s_total;
+  for (int j = 0; j < cnt; ++j) {
+    const uint32_t key = ksm[j * nt + tid];
+    if (topk_bucket(key, lo, scale) == B) ckey[cpos++] = key;
+  }
+  __syncthreads();
+  // bit-serial selection of the `need` largest candidate keys: warp 0 runs the
+  // passes when the list is short, the whole block otherwise
+  __shared__ uint32_t s_prefix, s_himask, s_kk, s_all;
+  const bool block_wide = m > 2048;
+  if (m == need) {
+    if (tid == 0) { s_prefix = 0u; s_himask = 0u; s_kk = need; s_all = 1u; }
+  } else if (!block_wide) {
+    if (warp == 0) {
+      uint32_t prefix = 0u, himask = 0u, kk = need, all = 0u;
+      for (int bit = 31; bit >= 0; --bit) {
+        uint32_t c = 0, cm = 0;
+        for (uint32_t i = lane; i < m; i += 32) {
+          const uint32_t key = ckey[i];
+          const uint32_t match = (key & himask) == prefix;
+          cm += match;
+          c += match & (key >> bit);
+        }
+        const uint32_t c1 = __reduce_add_sync(0xffffffffu, c);
+        const uint32_t cand = __reduce_add_sync(0xffffffffu, cm);
+        if (cand == kk) { all = 1u; break; }
+        if (c1 >= kk) prefix |= 1u << bit;
+        else kk -= c1;
+        himask |= 1u << bit;
+      }
+      if (lane == 0) { s_prefix = prefix; s_himask = himask; s_kk = kk; s_all = all; }
+    }
+  } else {
+    uint32_t prefix = 0u, himask = 0u, kk = need, all = 0u;
+    int pass = 0;
+    for (int bit = 31; bit >= 0; --bit, ++pass) {
+      uint32_t c = 0, cm = 0;
+      for (uint32_t i = tid; i < m; i += nt) {
+        const uint32_t key = ckey[i];
+        const uint32_t match = (key & himask) == prefix;
+        cm += match;
+        c += match & (key >> bit);
+      }
+      c = __reduce_add_sync(0xffffffffu, c);
+      cm = __reduce_add_sync(0xffffffffu, cm);
+      uint32_t* slot = s_wcnt + (pass % 3) * 64;
+      if (lane == 0) { slot[warp] = c; slot[32 + warp] = cm; }
+      __syncthreads();
+      const uint32_t c1 = __reduce_add_sync(0xffffffffu, lane < nwarps ? slot[lane] : 0u);
+      const uint32_t cand = __reduce_add_sync(0xffffffffu, lane < nwarps ? slot[32 + lane] : 0u);
+      if (cand == kk) { all = 1u; break; }
+      if (c1 >= kk) prefix |= 1u << bit;
+      else kk -= c1;
+      himask |= 1u << bit;
+    }
+    if (tid == 0) { s_prefix = prefix; s_himask = himask; s_kk = kk; s_all = all; }
+  }
+  __syncthreads();
+  const uint32_t prefix = s_prefix, himask = s_himask, kk = s_kk;
+  const bool all_taken = s_all != 0u;
+  // inside B: keep keys above tau and the first need_eq keys equal to it, or
+  // every candidate whose top bits reach the prefix (all_taken)
+  const uint32_t tau = prefix;
+  const uint32_t need_eq = all_taken ? 0xFFFFFFFFu : kk;
+  auto in_b_keep = [&](uint32_t key, uint32_t& e) -> bool {
+    if (all_taken) return (key & himask) >= prefix;
+    if (key > tau) return true;
+    if (key == tau) { const bool t = e < need_eq; ++e; return t; }
+    return false;
+  };
+  // 5. ordered compaction of the selection
   uint32_t n_eq = 0;
-  for (int i = i0; i < i1; ++i) n_eq += (keys[i] == tau);
-  uint32_t eq_before = block_exclusive_scan(n_eq, warp_tot, &s_total);
+  if (!all_taken)
+    for (int j = 0; j < cnt; ++j) {
+      const uint32_t key = ksm[j * nt + tid];
+      n_eq += (key == tau && topk_bucket(key, lo, scale) == B);
+    }
+  const uint32_t eq_before = block_exclusive_scan(n_eq, warp_tot, &s_total);
   uint32_t n_sel = 0;
   {
     uint32_t e = eq_before;
-    for (int i = i0; i < i1; ++i) {
-      const uint32_t key = keys[i];
-      if (key > tau) ++n_sel;
-      else if (key == tau) { if (e < need_eq) ++n_sel; ++e; }
+    for (int j = 0; j < cnt; ++j) {
+      const uint32_t key = ksm[j * nt + tid];
+      const uint32_t bk = topk_bucket(key, lo, scale);
+      n_sel += bk > B || (bk == B && in_b_keep(key, e));
     }
   }
   uint32_t pos = block_exclusive_scan(n_sel, warp_tot, &s_total);
@@ -214,14 +313,12 @@ __global__ void __launch_bounds__(1024) sr_topk_kernel(const float* __restrict__
     uint32_t e = eq_before;
     int32_t* o = sel + static_cast<int64_t>(unit) * k;
     int32_t* o2 = sel_out ? sel_out + static_cast<int64_t>(unit) * k : nullptr;
-    for (int i = i0; i < i1; ++i) {
-      const uint32_t key = keys[i];
-      bool take = false;
-      if (key > tau) take = true;
-      else if (key == tau) { take = e < need_eq; ++e; }
-      if (take) {
-        o[pos] = i;
-        if (o2) o2[pos] = i;
+    for (int j = 0; j < cnt; ++j) {
+      const uint32_t key = ksm[j * nt + tid];
+      const uint32_t bk = topk_bucket(key, lo, scale);
+      if (bk > B || (bk == B && in_b_keep(key, e))) {
+        o[pos] = i0 + j;
+        if (o2) o2[pos] = i0 + j;
         ++pos;
       }
     }
@@ -240,7 +337,17 @@ struct AttendArgs {
   int tiles_per_unit, n_tiles, ctas, max_units;
   int slot_floats;
   float theta;
+  double ft[128];  // RoPE turns per position of each frequency pair (host-computed, fp64)
 };
+
+__device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y,
+                                            int z, int w) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5, %6}], "
+      "[%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z), "r"(w)
+      : "memory");
+}
 
 __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y,
                                             int z) {
@@ -251,32 +358,70 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, u
       : "memory");
 }
 
+// Shared-memory plan of the tensor-core attend kernel (offsets from a 1 KiB
+// aligned base): K ring (A atoms, Bt atoms), V ring (value slabs, 128-byte
+// swizzled so they serve directly as the MN-major operand of the value MMA),
+// P double buffer (bf16 softmax weights, K-major swizzled B operand), alpha,
+// scaled queries ([j][g] interleaved), RoPE tables (per-chunk base angle and
+// per-offset rotation, rows padded to 130 floats so lanes of different chunks
+// hit different banks), reductions, barriers.
+constexpr int kRopeStride = 130;
+constexpr int kPBytes = 4096;  // [2 K-atoms][16 rows][128 B]
+constexpr int kKStageBytes = kTileChunks * kKAtoms * 1024;
+constexpr int kSmemKa = 0;
+constexpr int kSmemKb = kSmemKa + kKStages * kKStageBytes;
+constexpr int kSmemV = kSmemKb + kBStages * kAtomBytes;
+constexpr int kSmemP = kSmemV + kVStages * 16384;
+constexpr int kSmemAlpha = kSmemP + 2 * kPBytes;
+constexpr int kSmemQ = kSmemAlpha + 2 * kMaxGQ * 4;
+constexpr int kSmemBase = kSmemQ + 128 * kMaxGQ * 4;
+constexpr int kSmemRot = kSmemBase + kTileChunks * kRopeStride * 4;
+constexpr int kSmemFt = kSmemRot + 8 * kRopeStride * 4;
+constexpr int kSmemRed = kSmemFt + 64 * 8;
+constexpr int kSmemSpart = kSmemRed + 64 * 4;                         // [128][8] partial scores of half 1
+constexpr int kSmemBars = kSmemSpart + 128 * kMaxGQ * 4;
+constexpr int kNumBars = 2 * kKStages + 2 * kBStages + 2 * kVStages + 12;
+constexpr int kSmemEnd = kSmemBars + kNumBars * 8 + 16;
+constexpr int kVAccCol = 256;  // TMEM columns of the value accumulators (2 x 64)
+
+// Warp roles: 0-7 key epilogue (warp w reads TMEM lane quarter w % 4 and the
+// frequency pairs of half w / 4), 8-11 value epilogue, 12 key TMA producer,
+// 13 value TMA producer, 14 MMA issuer (TMEM owner).
 template <int GQ>
 __global__ void __launch_bounds__(kAttendThreads, 1)
     sr_attend_tc_kernel(const __grid_constant__ CUtensorMap mapAK, const __grid_constant__ CUtensorMap mapBK,
                         const __grid_constant__ CUtensorMap mapAV, const AttendArgs args) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const int NKA = args.rK / 64, NAV = args.rV / 64;
-  const int vstage_bytes = 2 * NAV * 1024;
-  uint8_t* Ka = smem;
-  uint8_t* Kb = Ka + kKStages * kAtomBytes;
-  uint8_t* Vs = Kb + kKStages * kAtomBytes;
-  float* p_s = reinterpret_cast<float*>(Vs + kVStages * 16384);  // [2][128][8]
-  float* alpha_s = p_s + 2 * 128 * kMaxGQ;                          // [2][8]
-  float* q_s = alpha_s + 2 * kMaxGQ;                                // [GQ][128]
-  double* ft = reinterpret_cast<double*>(q_s + kMaxGQ * 128);       // [64]
-  float* red = reinterpret_cast<float*>(ft + 64);                   // [2][4][8]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(red + 64);
+  const int NKA = args.rK / 64;
+  const int NMB = (args.rV + 127) / 128;  // value M-blocks of 128 rank columns
+  const int NAVp = 2 * NMB;               // 64-column atoms per value slab (zero-padded)
+  const int NAV = args.rV / 64;           // atoms actually loaded
+  uint8_t* Ka = smem + kSmemKa;
+  uint8_t* Kb = smem + kSmemKb;
+  uint8_t* Vs = smem + kSmemV;
+  uint8_t* Ps = smem + kSmemP;
+  float* alpha_s = reinterpret_cast<float*>(smem + kSmemAlpha);
+  float* q_s = reinterpret_cast<float*>(smem + kSmemQ);
+  float* base_s = reinterpret_cast<float*>(smem + kSmemBase);
+  float* rot_s = reinterpret_cast<float*>(smem + kSmemRot);
+  double* ft = reinterpret_cast<double*>(smem + kSmemFt);
+  float* red = reinterpret_cast<float*>(smem + kSmemRed);
+  float* spart = reinterpret_cast<float*>(smem + kSmemSpart);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kSmemBars);
   uint64_t* kfull = bars;
   uint64_t* kempty = kfull + kKStages;
-  uint64_t* vfull = kempty + kKStages;
+  uint64_t* bfull = kempty + kKStages;
+  uint64_t* bempty = bfull + kBStages;
+  uint64_t* vfull = bempty + kBStages;
   uint64_t* vempty = vfull + kVStages;
   uint64_t* accfull = vempty + kVStages;
   uint64_t* accempty = accfull + 2;
   uint64_t* pfull = accempty + 2;
   uint64_t* pempty = pfull + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(pempty + 2);
+  uint64_t* vaccfull = pempty + 2;
+  uint64_t* vaccempty = vaccfull + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(vaccempty + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -286,32 +431,48 @@ __global__ void __launch_bounds__(kAttendThreads, 1)
 
   if (tid == 0) {
     for (int i = 0; i < kKStages; ++i) { mbar_init(&kfull[i], 1); mbar_init(&kempty[i], 1); }
-    for (int i = 0; i < kVStages; ++i) { mbar_init(&vfull[i], 1); mbar_init(&vempty[i], 256); }
+    for (int i = 0; i < kBStages; ++i) { mbar_init(&bfull[i], 1); mbar_init(&bempty[i], 1); }
+    for (int i = 0; i < kVStages; ++i) { mbar_init(&vfull[i], 1); mbar_init(&vempty[i], 1); }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&accfull[i], 1);
-      mbar_init(&accempty[i], 128);
+      mbar_init(&accempty[i], 256);
       mbar_init(&pfull[i], 128);
-      mbar_init(&pempty[i], 256);
+      mbar_init(&pempty[i], 129);
+      mbar_init(&vaccfull[i], 1);
+      mbar_init(&vaccempty[i], 128);
     }
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (tid < 64) ft[tid] = rope_turns(static_cast<double>(args.theta), tid, 128);
-  if (warp == 1) tmem_alloc(tmem_slot, 256);
-  if (warp == 0 && lane == 0) {
+  if (tid < 64) ft[tid] = args.ft[tid];
+  // rows of P beyond the query group, and value atoms past the rank (when it
+  // is not a multiple of 128), are never loaded and stay zero
+  for (int i = tid; i < 2 * kPBytes / 16; i += blockDim.x) reinterpret_cast<uint4*>(Ps)[i] = make_uint4(0, 0, 0, 0);
+  for (int i = tid; i < kVStages * 16384 / 16; i += blockDim.x) reinterpret_cast<uint4*>(Vs)[i] = make_uint4(0, 0, 0, 0);
+  __syncthreads();
+  for (int i = tid; i < 8 * 64; i += blockDim.x) {
+    const int e = i >> 6, j = i & 63;
+    float c, sn;
+    rope_cs(ft[j], static_cast<double>(e), &c, &sn);
+    rot_s[e * kRopeStride + 2 * j] = c;
+    rot_s[e * kRopeStride + 2 * j + 1] = sn;
+  }
+  if (warp == 14) tmem_alloc(tmem_slot, 512);
+  if (warp == 12 && lane == 0) {
     prefetch_tmap(&mapAK);
     prefetch_tmap(&mapBK);
     prefetch_tmap(&mapAV);
   }
+  fence_proxy_async();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer
+  if (warp == 12) {
+    // ------------------------------------------------------ TMA producer (keys)
     if (lane == 0) {
-      uint32_t ks = 0, vsn = 0;
+      uint32_t ks = 0, bs = 0;
       for (int x = tb; x < te && !*abort_flag; ++x) {
         const int u = x / tpu, ti = x % tpu;
         const int b = u / args.Hkv, h = u % args.Hkv;
@@ -320,89 +481,159 @@ __global__ void __launch_bounds__(kAttendThreads, 1)
         int rows[kTileChunks];
 #pragma unroll
         for (int ch = 0; ch < kTileChunks; ++ch) rows[ch] = ch < nch ? args.sink + su[ch] * 8 : 0;
-        for (int a = 0; a < NKA; ++a, ++ks) {
+        // one 4-D box per chunk covers kKAtoms atoms (8 rows x 128 columns);
+        // the Bt_K atoms of the stage follow on their own ring (L2 hits)
+        bool ok = true;
+        for (int sk = 0; sk < NKA / kKAtoms && ok; ++sk, ++ks) {
           const int slot = ks % kKStages;
-          if (!mbar_wait(&kempty[slot], ((ks / kKStages) & 1) ^ 1, args.status)) { *abort_flag = 1; break; }
-          mbar_arrive_expect_tx(&kfull[slot], nch * 1024 + kAtomBytes);
+          if (!mbar_wait(&kempty[slot], ((ks / kKStages) & 1) ^ 1, args.status)) { *abort_flag = 1; ok = false; break; }
+          mbar_arrive_expect_tx(&kfull[slot], nch * kKAtoms * 1024);
           for (int ch = 0; ch < nch; ++ch)
-            tma_load_3d(Ka + slot * kAtomBytes + ch * 1024, &mapAK, &kfull[slot], a * 64, rows[ch], b);
-          tma_load_3d(Kb + slot * kAtomBytes, &mapBK, &kfull[slot], a * 64, h * 128, args.sbk ? b : 0);
+            tma_load_4d(Ka + slot * kKStageBytes + ch * kKAtoms * 1024, &mapAK, &kfull[slot], 0, rows[ch],
+                        sk * kKAtoms, b);
+          for (int a = 0; a < kKAtoms; ++a, ++bs) {
+            const int bslot = bs % kBStages;
+            if (!mbar_wait(&bempty[bslot], ((bs / kBStages) & 1) ^ 1, args.status)) { *abort_flag = 1; ok = false; break; }
+            mbar_arrive_expect_tx(&bfull[bslot], kAtomBytes);
+            tma_load_3d(Kb + bslot * kAtomBytes, &mapBK, &bfull[bslot], (sk * kKAtoms + a) * 64, h * 128,
+                        args.sbk ? b : 0);
+          }
         }
+      }
+    }
+  } else if (warp == 13) {
+    // ---------------------------------------------------- TMA producer (values)
+    // a stage holds two chunks (16 rows); a missing second chunk is replaced by
+    // the first (finite data; its softmax weights are zero)
+    if (lane == 0) {
+      uint32_t vsn = 0;
+      for (int x = tb; x < te && !*abort_flag; ++x) {
+        const int u = x / tpu, ti = x % tpu;
+        const int b = u / args.Hkv;
+        const int nch = min(kTileChunks, k - ti * kTileChunks);
+        const int32_t* su = args.sel + static_cast<int64_t>(u) * k + ti * kTileChunks;
+        int rows[kTileChunks];
+#pragma unroll
+        for (int ch = 0; ch < kTileChunks; ++ch) rows[ch] = ch < nch ? args.sink + su[ch] * 8 : 0;
         for (int v = 0; v < (nch + 1) / 2 && !*abort_flag; ++v, ++vsn) {
           const int slot = vsn % kVStages;
           if (!mbar_wait(&vempty[slot], ((vsn / kVStages) & 1) ^ 1, args.status)) { *abort_flag = 1; break; }
-          const int nv = min(2, nch - 2 * v);
-          mbar_arrive_expect_tx(&vfull[slot], nv * NAV * 1024);
-          for (int c2 = 0; c2 < nv; ++c2)
-            for (int a = 0; a < NAV; ++a)
-              tma_load_3d(Vs + slot * 16384 + (c2 * NAV + a) * 1024, &mapAV, &vfull[slot], a * 64,
-                          rows[2 * v + c2], b);
+          mbar_arrive_expect_tx(&vfull[slot], 2 * NAV * 1024);
+          for (int c2 = 0; c2 < 2; ++c2) {
+            const int ch = (2 * v + c2 < nch) ? 2 * v + c2 : 2 * v;
+            tma_load_4d(Vs + slot * 16384 + c2 * NAVp * 1024, &mapAV, &vfull[slot], 0, rows[ch], 0, b);
+          }
         }
       }
     }
-  } else if (warp == 1) {
+  } else if (warp == 14) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      const uint32_t idesc = umma_idesc_bf16(128, 128);
-      uint32_t ks = 0;
-      int j = 0;
-      for (int x = tb; x < te && !*abort_flag; ++x, ++j) {
+      const uint32_t idk = umma_idesc_bf16(128, 128);
+      const uint32_t idv = umma_idesc_bf16(128, 16, true, false);
+      uint32_t ks = 0, bs = 0, vsn = 0;
+      auto issue_keys = [&](int j) -> bool {
         const int buf = j & 1;
-        if (!mbar_wait(&accempty[buf], ((j >> 1) & 1) ^ 1, args.status)) { *abort_flag = 1; break; }
+        if (!mbar_wait(&accempty[buf], ((j >> 1) & 1) ^ 1, args.status)) return false;
         tc_fence_after();
         const uint32_t dtm = tmem + buf * 128;
-        for (int a = 0; a < NKA; ++a, ++ks) {
+        for (int sk = 0; sk < NKA / kKAtoms; ++sk, ++ks) {
           const int slot = ks % kKStages;
-          if (!mbar_wait(&kfull[slot], (ks / kKStages) & 1, args.status)) { *abort_flag = 1; break; }
-          tc_fence_after();
-          const uint64_t ad = umma_desc_sw128(smem_u32(Ka + slot * kAtomBytes));
-          const uint64_t bd = umma_desc_sw128(smem_u32(Kb + slot * kAtomBytes));
+          if (!mbar_wait(&kfull[slot], (ks / kKStages) & 1, args.status)) return false;
+          for (int a = 0; a < kKAtoms; ++a, ++bs) {
+            const int bslot = bs % kBStages;
+            if (!mbar_wait(&bfull[bslot], (bs / kBStages) & 1, args.status)) return false;
+            tc_fence_after();
+            const uint64_t ad = umma_desc_sw128(smem_u32(Ka + slot * kKStageBytes + a * 1024), kKAtoms * 1024);
+            const uint64_t bd = umma_desc_sw128(smem_u32(Kb + bslot * kAtomBytes));
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) umma_bf16(dtm, ad + 2 * kk, bd + 2 * kk, idesc, (a | kk) ? 1u : 0u);
+            for (int kk = 0; kk < 4; ++kk)
+              umma_bf16(dtm, ad + 2 * kk, bd + 2 * kk, idk, (sk | a | kk) ? 1u : 0u);
+            umma_commit(&bempty[bslot]);
+          }
           umma_commit(&kempty[slot]);
         }
         umma_commit(&accfull[buf]);
+        return true;
+      };
+      auto issue_values = [&](int j, int x) -> bool {
+        const int pb = j & 1;
+        const int ti = x % tpu;
+        const int nch = min(kTileChunks, k - ti * kTileChunks);
+        if (!mbar_wait(&pfull[pb], (j >> 1) & 1, args.status)) return false;
+        if (!mbar_wait(&vaccempty[pb], ((j >> 1) & 1) ^ 1, args.status)) return false;
+        tc_fence_after();
+        const uint32_t dtm = tmem + kVAccCol + pb * 64;
+        for (int v = 0; v < (nch + 1) / 2; ++v, ++vsn) {
+          const int slot = vsn % kVStages;
+          if (!mbar_wait(&vfull[slot], (vsn / kVStages) & 1, args.status)) return false;
+          tc_fence_after();
+          const uint64_t pd = umma_desc_sw128(smem_u32(Ps + pb * kPBytes + (v >> 2) * 2048 + (v & 3) * 32));
+          for (int mb = 0; mb < NMB; ++mb) {
+            const uint64_t ad = umma_desc_sw128_mn(smem_u32(Vs + slot * 16384 + 2 * mb * 1024), 1024, NAVp * 1024);
+            umma_bf16(dtm + mb * 16, ad, pd, idv, v > 0 ? 1u : 0u);
+          }
+          umma_commit(&vempty[slot]);
+        }
+        umma_commit(&vaccfull[pb]);
+        umma_commit(&pempty[pb]);
+        return true;
+      };
+      bool ok = tb < te ? issue_keys(0) : true;
+      int j = 0;
+      for (int x = tb; x < te && ok && !*abort_flag; ++x, ++j) {
+        if (x + 1 < te) ok = issue_keys(j + 1);
+        if (ok) ok = issue_values(j, x);
       }
+      if (!ok) *abort_flag = 1;
     }
-  } else if (warp < 6) {
+  } else if (warp < 8) {
     // --------------------------------------- key epilogue: RoPE, q.k, softmax
-    const int lq = warp & 3;
+    const int lq = warp & 3, hf = warp >> 2;  // lane quarter, frequency half
     const int row = lq * 32 + lane;
-    const int et = tid - 64;
+    const int et = tid;                       // 0..255
     const float qscale = rsqrtf(128.0f) * kLog2e;
-    // queries of the unit are (re)loaded when the unit changes
     float m[GQ], l[GQ];
     int cur_u = -1, j = 0;
     for (int x = tb; x < te && !*abort_flag; ++x, ++j) {
       const int u = x / tpu, ti = x % tpu;
+      const int nch = min(kTileChunks, k - ti * kTileChunks);
+      const int32_t* su = args.sel + static_cast<int64_t>(u) * k + ti * kTileChunks;
+      named_bar_sync(1, 256);  // the previous tile's readers of q_s / base_s / spart are done
       if (u != cur_u) {
-        named_bar_sync(1, 128);
         const int b = u / args.Hkv, h = u % args.Hkv;
-        for (int i = et; i < GQ * 128; i += 128) {
-          const int g = i / 128, jj = i % 128;
-          q_s[g * 128 + jj] =
-              to_f(reinterpret_cast<const __nv_bfloat16*>(args.q)[(static_cast<int64_t>(b) * args.Hq + h * GQ + g) * 128 + jj]) *
-              qscale;
+        for (int i = et; i < 128 * kMaxGQ; i += 256) {
+          const int jj = i / kMaxGQ, g = i % kMaxGQ;
+          q_s[i] = g < GQ ? to_f(reinterpret_cast<const __nv_bfloat16*>(args.q)[(static_cast<int64_t>(b) * args.Hq +
+                                                                                 h * GQ + g) * 128 + jj]) * qscale
+                          : 0.f;
         }
-        named_bar_sync(1, 128);
         cur_u = u;
 #pragma unroll
         for (int g = 0; g < GQ; ++g) { m[g] = -INFINITY; l[g] = 0.f; }
       }
+      // base angle of every chunk of the tile: (cos, sin)(t0 f_j), t0 = first token
+      for (int i = et; i < kTileChunks * 64; i += 256) {
+        const int ch = i >> 6, jj = i & 63;
+        float c = 1.f, sn = 0.f;
+        if (ch < nch) rope_cs(ft[jj], static_cast<double>(args.sink + static_cast<int64_t>(su[ch]) * 8), &c, &sn);
+        base_s[ch * kRopeStride + 2 * jj] = c;
+        base_s[ch * kRopeStride + 2 * jj + 1] = sn;
+      }
+      named_bar_sync(1, 256);
       const int ch = row >> 3, e = row & 7;
-      const bool valid = ti * kTileChunks + ch < k;
-      const double pos =
-          valid ? static_cast<double>(args.sink + static_cast<int64_t>(args.sel[static_cast<int64_t>(u) * k + ti * kTileChunks + ch]) * 8 + e)
-                : 0.0;
+      const bool valid = ch < nch;
+      const float2* bse = reinterpret_cast<const float2*>(base_s + ch * kRopeStride);
+      const float2* rte = reinterpret_cast<const float2*>(rot_s + e * kRopeStride);
       const int buf = j & 1;
       if (!mbar_wait(&accfull[buf], (j >> 1) & 1, args.status)) { *abort_flag = 1; break; }
       tc_fence_after();
       const uint32_t taddr = tmem + (static_cast<uint32_t>(lq * 32) << 16) + buf * 128;
-      float s[GQ];
+      float s0[GQ], s1[GQ];
 #pragma unroll
-      for (int g = 0; g < GQ; ++g) s[g] = 0.f;
+      for (int g = 0; g < GQ; ++g) { s0[g] = 0.f; s1[g] = 0.f; }
 #pragma unroll 1
-      for (int jb = 0; jb < 4; ++jb) {
+      for (int jb = 2 * hf; jb < 2 * hf + 2; ++jb) {
         float lo[16], hi[16];
         tmem_ld16(taddr + jb * 16, lo);
         tmem_ld16(taddr + 64 + jb * 16, hi);
@@ -410,49 +641,82 @@ __global__ void __launch_bounds__(kAttendThreads, 1)
 #pragma unroll
         for (int jj = 0; jj < 16; ++jj) {
           const int jx = jb * 16 + jj;
-          float c, sn;
-          rope_cs(ft[jx], pos, &c, &sn);
+          const float2 b0 = bse[jx], r0 = rte[jx];
+          const float c = b0.x * r0.x - b0.y * r0.y;
+          const float sn = b0.y * r0.x + b0.x * r0.y;
           const float y0 = lo[jj] * c - hi[jj] * sn;
           const float y1 = hi[jj] * c + lo[jj] * sn;
+          const float4* q0 = reinterpret_cast<const float4*>(q_s + jx * kMaxGQ);
+          const float4* q1 = reinterpret_cast<const float4*>(q_s + (64 + jx) * kMaxGQ);
+          float qa[8], qb[8];
+          *reinterpret_cast<float4*>(qa) = q0[0];
+          *reinterpret_cast<float4*>(qb) = q1[0];
+          if (GQ > 4) {
+            *reinterpret_cast<float4*>(qa + 4) = q0[1];
+            *reinterpret_cast<float4*>(qb + 4) = q1[1];
+          }
 #pragma unroll
-          for (int g = 0; g < GQ; ++g) s[g] = fmaf(q_s[g * 128 + jx], y0, fmaf(q_s[g * 128 + 64 + jx], y1, s[g]));
+          for (int g = 0; g < GQ; ++g) {
+            if (jj & 1) s1[g] = fmaf(qa[g], y0, fmaf(qb[g], y1, s1[g]));
+            else s0[g] = fmaf(qa[g], y0, fmaf(qb[g], y1, s0[g]));
+          }
         }
       }
       tc_fence_before();
       mbar_arrive(&accempty[buf]);
-      // tile maximum per query head
+      if (hf == 1) {
+#pragma unroll
+        for (int g = 0; g < GQ; ++g) spart[row * kMaxGQ + g] = s0[g] + s1[g];
+      }
+      named_bar_sync(1, 256);
+      if (hf == 1) continue;
+      float s[GQ];
+#pragma unroll
+      for (int g = 0; g < GQ; ++g) s[g] = s0[g] + s1[g] + spart[row * kMaxGQ + g];
+      // tile maximum per query head (the 128 threads of half 0)
       float tmax[GQ];
 #pragma unroll
       for (int g = 0; g < GQ; ++g) {
         if (!valid) s[g] = -INFINITY;
         const float w = warp_max(s[g]);
-        if (lane == 0) red[(lq)*8 + g] = w;
+        if (lane == 0) red[lq * 8 + g] = w;
       }
-      named_bar_sync(1, 128);
+      named_bar_sync(2, 128);
 #pragma unroll
       for (int g = 0; g < GQ; ++g)
         tmax[g] = fmaxf(fmaxf(red[0 * 8 + g], red[1 * 8 + g]), fmaxf(red[2 * 8 + g], red[3 * 8 + g]));
-      float alpha[GQ], p[GQ];
+      float alpha[GQ];
+      __nv_bfloat16 pbf[GQ];
 #pragma unroll
       for (int g = 0; g < GQ; ++g) {
         const float mn = fmaxf(m[g], tmax[g]);
         alpha[g] = exp2f(m[g] - mn);
-        p[g] = valid ? exp2f(s[g] - mn) : 0.f;
+        // the weights enter the value MMA as bf16: the sum uses the same values
+        pbf[g] = __float2bfloat16_rn(valid ? exp2f(s[g] - mn) : 0.f);
         m[g] = mn;
-        const float w = warp_sum(p[g]);
+        const float w = warp_sum(__bfloat162float(pbf[g]));
         if (lane == 0) red[32 + lq * 8 + g] = w;
       }
-      named_bar_sync(1, 128);
+      named_bar_sync(2, 128);
 #pragma unroll
       for (int g = 0; g < GQ; ++g)
         l[g] = l[g] * alpha[g] + (red[32 + g] + red[40 + g] + red[48 + g] + red[56 + g]);
       const int pb = j & 1;
       if (!mbar_wait(&pempty[pb], ((j >> 1) & 1) ^ 1, args.status)) { *abort_flag = 1; break; }
+      // P[g][t] (K-major, 128-byte swizzle): row g of the K-atom t / 64
+      {
+        const int katom = row >> 6, kin = row & 63;
+        uint8_t* pbase = Ps + pb * kPBytes + katom * 2048;
 #pragma unroll
-      for (int g = 0; g < GQ; ++g) p_s[(pb * 128 + row) * kMaxGQ + g] = p[g];
+        for (int g = 0; g < GQ; ++g) {
+          const int off = (g >> 3) * 1024 + (g & 7) * 128 + ((((kin * 2) >> 4) ^ (g & 7)) << 4) + ((kin * 2) & 15);
+          *reinterpret_cast<__nv_bfloat16*>(pbase + off) = pbf[g];
+        }
+      }
       if (et == 0)
 #pragma unroll
         for (int g = 0; g < GQ; ++g) alpha_s[pb * kMaxGQ + g] = alpha[g];
+      fence_proxy_async();
       mbar_arrive(&pfull[pb]);
       const bool seg_end = (x + 1 == te) || ((x + 1) / tpu != u);
       if (seg_end && et == 0) {
@@ -462,81 +726,67 @@ __global__ void __launch_bounds__(kAttendThreads, 1)
         for (int g = 0; g < GQ; ++g) { slot[g] = m[g]; slot[8 + g] = l[g]; }
       }
     }
-  } else {
-    // ------------------------------------- value path: u_g += p_gt A_V[t]
-    const int vt = tid - 192;
-    const int cp = vt;
-    const bool act = cp < args.rV / 2;
-    const int atom = cp >> 5, wrd = cp & 31;
-    float acc[GQ][2];
+  } else if (warp < 12) {
+    // ------------------------- value epilogue: u_g = u_g alpha + P A_V (TMEM)
+    const int lq = warp & 3;
+    float acc[4][GQ];
+#pragma unroll
+    for (int mb = 0; mb < 4; ++mb)
+#pragma unroll
+      for (int g = 0; g < GQ; ++g) acc[mb][g] = 0.f;
     int cur_u = -1, j = 0;
-    uint32_t vsn = 0;
     for (int x = tb; x < te && !*abort_flag; ++x, ++j) {
-      const int u = x / tpu, ti = x % tpu;
+      const int u = x / tpu;
       if (u != cur_u) {
         cur_u = u;
 #pragma unroll
-        for (int g = 0; g < GQ; ++g) acc[g][0] = acc[g][1] = 0.f;
+        for (int mb = 0; mb < 4; ++mb)
+#pragma unroll
+          for (int g = 0; g < GQ; ++g) acc[mb][g] = 0.f;
       }
       const int pb = j & 1;
-      if (!mbar_wait(&pfull[pb], (j >> 1) & 1, args.status)) { *abort_flag = 1; break; }
+      if (!mbar_wait(&vaccfull[pb], (j >> 1) & 1, args.status)) { *abort_flag = 1; break; }
+      tc_fence_after();
+      float al[GQ];
 #pragma unroll
-      for (int g = 0; g < GQ; ++g) {
-        const float a = alpha_s[pb * kMaxGQ + g];
-        acc[g][0] *= a;
-        acc[g][1] *= a;
-      }
-      const int nch = min(kTileChunks, k - ti * kTileChunks);
-      bool ok = true;
-      for (int v = 0; v < (nch + 1) / 2; ++v, ++vsn) {
-        const int slot = vsn % kVStages;
-        if (!mbar_wait(&vfull[slot], (vsn / kVStages) & 1, args.status)) { *abort_flag = 1; ok = false; break; }
-        const int nr = min(2, nch - 2 * v) * 8;
-        if (act) {
-          const uint8_t* base = Vs + slot * 16384;
-          const float* pr = p_s + (pb * 128 + v * 16) * kMaxGQ;
-#pragma unroll 4
-          for (int r = 0; r < nr; ++r) {
-            const int c2 = r >> 3, rr = r & 7;
-            const uint32_t w = *reinterpret_cast<const uint32_t*>(base + ((c2 * NAV + atom) * 8 + rr) * 128 + wrd * 4);
-            const float2 a = bf2_to_f2(w);
+      for (int g = 0; g < GQ; ++g) al[g] = alpha_s[pb * kMaxGQ + g];
+      const uint32_t taddr = tmem + (static_cast<uint32_t>(lq * 32) << 16) + kVAccCol + pb * 64;
 #pragma unroll
-            for (int g = 0; g < GQ; ++g) {
-              const float pg = pr[r * kMaxGQ + g];
-              acc[g][0] = fmaf(pg, a.x, acc[g][0]);
-              acc[g][1] = fmaf(pg, a.y, acc[g][1]);
-            }
-          }
+      for (int mb = 0; mb < 4; ++mb) {
+        if (mb < NMB) {
+          float v[16];
+          tmem_ld16(taddr + mb * 16, v);
+          tmem_ld_wait();
+#pragma unroll
+          for (int g = 0; g < GQ; ++g) acc[mb][g] = fmaf(acc[mb][g], al[g], v[g]);
         }
-        fence_proxy_async();
-        mbar_arrive(&vempty[slot]);
       }
-      if (!ok) break;
+      tc_fence_before();
+      mbar_arrive(&vaccempty[pb]);
       mbar_arrive(&pempty[pb]);
       const bool seg_end = (x + 1 == te) || ((x + 1) / tpu != u);
-      if (seg_end && act) {
+      if (seg_end) {
         const int u_first = tb / tpu;
         float* slot = args.part + (static_cast<int64_t>(cta) * args.max_units + (u - u_first)) * args.slot_floats;
 #pragma unroll
-        for (int g = 0; g < GQ; ++g) {
-          slot[16 + g * args.rV + 2 * cp] = acc[g][0];
-          slot[16 + g * args.rV + 2 * cp + 1] = acc[g][1];
+        for (int mb = 0; mb < 4; ++mb) {
+          const int c = mb * 128 + lq * 32 + lane;
+          if (mb < NMB && c < args.rV)
+#pragma unroll
+            for (int g = 0; g < GQ; ++g) slot[16 + g * args.rV + c] = acc[mb][g];
         }
       }
     }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == 14) {
     tc_fence_after();
-    tmem_dealloc(tmem, 256);
+    tmem_dealloc(tmem, 512);
   }
 }
 
-size_t attend_tc_smem() {
-  return 1024 + 2 * kKStages * kAtomBytes + kVStages * 16384 + (2 * 128 * kMaxGQ + 2 * kMaxGQ + kMaxGQ * 128) * 4 +
-         64 * 8 + 64 * 4 + (2 * kKStages + 2 * kVStages + 8) * 8 + 16;
-}
+size_t attend_tc_smem() { return 1024 + kSmemEnd; }
 
 // ---------------------------------------------------- sr_attend (SIMT)
 // Same schedule and partial format; rebuilds both K and the value basis sums on
@@ -562,7 +812,7 @@ __global__ void __launch_bounds__(256) sr_attend_simt_kernel(const T* __restrict
   const int tpu = args.tiles_per_unit, k = args.k, half = hd / 2;
   const int d = args.Hkv * hd;
   const float qscale = rsqrtf(static_cast<float>(hd)) * kLog2e;
-  for (int j = tid; j < half; j += blockDim.x) ft[j] = rope_turns(static_cast<double>(args.theta), j, hd);
+  for (int j = tid; j < half; j += blockDim.x) ft[j] = args.ft[j];
   int cur_u = -1;
   for (int x = tb; x < te; ++x) {
     const int u = x / tpu, ti = x % tpu;
@@ -646,120 +896,231 @@ __global__ void __launch_bounds__(256) sr_attend_simt_kernel(const T* __restrict
 }
 
 // ----------------------------------------------------------- sr_combine
-// One block per unit: merge the partials of every CTA that covered the unit,
-// add the raw sink/recent rows, and map the value-basis sums through Bt_V:
-//   o_g = (sum_c U_g[c] Bt_V[h hd + j][c] + sum_t p_gt V_t[j]) / L_g.
+// Grid (unit, column split of kCombineSplit), 256 threads.  Each phase issues
+// all of its loads before using them (one memory round trip per phase):
+//   A  queries, the unit's raw window rows, the partial-slot statistics, and
+//      the RoPE angles of the window positions;
+//   B  window scores (thread per row x query head, padded rows: no bank
+//      conflicts);  C  M_g and L_g;  D  U_g = sum over slots of u 2^(m - M);
+//   E  o_g[j] = (U_g . Bt_V[h hd + j] + sum_t p_gt V_t[j]) / L_g for the
+//      split's columns (warp per column, 16-byte loads of the Bt_V row).
+constexpr int kCombineSplit = 4;
+constexpr int kCombineThreads = 256;
+constexpr int kMaxSlots = 64;
+
 template <typename T>
-__global__ void __launch_bounds__(256) sr_combine_kernel(const T* __restrict__ q, const T* __restrict__ BtV,
-                                                         const T* __restrict__ srK, const T* __restrict__ srV,
-                                                         const AttendArgs args, int hd, float* __restrict__ out) {
+__global__ void __launch_bounds__(kCombineThreads) sr_combine_kernel(const T* __restrict__ q, const T* __restrict__ BtV,
+                                                                     const T* __restrict__ srK,
+                                                                     const T* __restrict__ srV, const AttendArgs args,
+                                                                     int hd, float* __restrict__ out) {
   extern __shared__ double smd[];
   const int gq = args.Hq / args.Hkv;
   const int nsr = args.sink + args.recent;
   const int u = blockIdx.x, b = u / args.Hkv, h = u % args.Hkv;
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nwarps = blockDim.x >> 5;
   const int tpu = args.tiles_per_unit;
   const int d = args.Hkv * hd, half = hd / 2;
-  double* ft = smd;                        // [half]
-  float* Us = reinterpret_cast<float*>(smd + half);  // [gq][rV]
-  float* Ws = Us + gq * args.rV;           // [gq][hd]
-  float* qs = Ws + gq * hd;                // [gq][hd]
-  float* srs = qs + gq * hd;               // [nsr][gq] scores, then weights
-  float* Mg = srs + nsr * gq;              // [gq]
-  float* Lg = Mg + kMaxGQ;                 // [gq]
-  float* sc = Lg + kMaxGQ;                 // [slots][gq] partial rescale factors (slots <= 64)
+  const int hdp = hd + 1;  // padded row stride
+  const int cols = (hd + kCombineSplit - 1) / kCombineSplit, j0 = blockIdx.y * cols, j1 = min(hd, j0 + cols);
+  double* ftab = smd;                      // [128] RoPE turns (first: 8-byte aligned)
+  float* Us = reinterpret_cast<float*>(smd + 128);  // [gq][rV] (16-byte aligned)
+  float* qs = Us + gq * args.rV;           // [gq][hd]
+  float* wK = qs + gq * hd;                // [nsr][hd+1] raw window keys
+  float* wV = wK + nsr * hdp;              // [nsr][hd+1] raw window values
+  float* csn = wV + nsr * hdp;             // [nsr][half+1] cos
+  float* snn = csn + nsr * (half + 1);     // [nsr][half+1] sin
+  float* srs = snn + nsr * (half + 1);     // [nsr][gq] scores, then weights
+  float* ml = srs + nsr * gq;              // [slots][16] partial m, l
+  float* sc = ml + kMaxSlots * 16;         // [slots][8] slot factors
+  float* Mg = sc + kMaxSlots * kMaxGQ;     // [8]
+  float* Lg = Mg + kMaxGQ;                 // [8]
   const int fc = cta_of_tile(u * tpu, args.n_tiles, args.ctas);
   const int lc = cta_of_tile((u + 1) * tpu - 1, args.n_tiles, args.ctas);
   const int nslots = lc - fc + 1;
+  auto slot_ptr = [&](int c) -> const float* {
+    const int uf = tile_begin(c, args.n_tiles, args.ctas) / tpu;
+    return args.part + (static_cast<int64_t>(c) * args.max_units + (u - uf)) * args.slot_floats;
+  };
+  // ---- A: loads and the window RoPE angles
   const float qscale = rsqrtf(static_cast<float>(hd)) * kLog2e;
   for (int i = tid; i < gq * hd; i += blockDim.x)
     qs[i] = to_f(q[(static_cast<int64_t>(b) * args.Hq + h * gq) * hd + i]) * qscale;
-  for (int j = tid; j < half; j += blockDim.x) ft[j] = rope_turns(static_cast<double>(args.theta), j, hd);
+  if (sizeof(T) == 2 && hd % 8 == 0) {
+    // 16-byte vectors; every load of a thread is issued before any is used
+    const int vpr = hd / 8;  // vectors per row
+    constexpr int kV = 8;
+    for (int v0 = tid; v0 < 2 * nsr * vpr; v0 += kV * blockDim.x) {
+      uint4 w[kV];
+#pragma unroll
+      for (int t = 0; t < kV; ++t) {
+        const int v = v0 + t * blockDim.x;
+        if (v < 2 * nsr * vpr) {
+          const int mat = v / (nsr * vpr), r = (v / vpr) % nsr, c8 = v % vpr;
+          const T* src = (mat ? srV : srK) + (static_cast<int64_t>(b) * nsr + r) * d + h * hd + c8 * 8;
+          w[t] = *reinterpret_cast<const uint4*>(src);
+        }
+      }
+#pragma unroll
+      for (int t = 0; t < kV; ++t) {
+        const int v = v0 + t * blockDim.x;
+        if (v < 2 * nsr * vpr) {
+          const int mat = v / (nsr * vpr), r = (v / vpr) % nsr, c8 = v % vpr;
+          float* dst = (mat ? wV : wK) + r * hdp + c8 * 8;
+          const uint32_t ww[4] = {w[t].x, w[t].y, w[t].z, w[t].w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 f = bf2_to_f2(ww[e]);
+            dst[2 * e] = f.x;
+            dst[2 * e + 1] = f.y;
+          }
+        }
+      }
+    }
+  } else {
+    for (int i = tid; i < nsr * hd; i += blockDim.x) {
+      const int r = i / hd, jj = i % hd;
+      const int64_t off = (static_cast<int64_t>(b) * nsr + r) * d + h * hd + jj;
+      wK[r * hdp + jj] = to_f(srK[off]);
+      wV[r * hdp + jj] = to_f(srV[off]);
+    }
+  }
+  for (int i = tid; i < nslots * 16; i += blockDim.x) ml[i] = slot_ptr(fc + i / 16)[i % 16];
+  for (int j = tid; j < half; j += blockDim.x) ftab[j] = args.ft[j];
   __syncthreads();
-  // scores of the raw window rows (row i < sink is token i, else T - recent + i - sink)
+  for (int i = tid; i < nsr * half; i += blockDim.x) {
+    const int r = i / half, jj = i % half;
+    const int64_t t = r < args.sink ? r : args.T - args.recent + (r - args.sink);
+    float c, sn;
+    rope_cs(ftab[jj], static_cast<double>(t), &c, &sn);
+    csn[r * (half + 1) + jj] = c;
+    snn[r * (half + 1) + jj] = sn;
+  }
+  __syncthreads();
+  // ---- B: window scores
   for (int i = tid; i < nsr * gq; i += blockDim.x) {
     const int r = i / gq, g = i % gq;
-    const int64_t t = r < args.sink ? r : args.T - args.recent + (r - args.sink);
-    const T* kr = srK + (static_cast<int64_t>(b) * nsr + r) * d + h * hd;
-    float s = 0.f;
+    const float* kr = wK + r * hdp;
+    const float* cr = csn + r * (half + 1);
+    const float* sr = snn + r * (half + 1);
+    const float* qg = qs + g * hd;
+    float s0 = 0.f, s1 = 0.f;
+#pragma unroll 8
     for (int jj = 0; jj < half; ++jj) {
-      float cs, sn;
-      rope_cs(ft[jj], static_cast<double>(t), &cs, &sn);
-      const float x0 = to_f(kr[jj]), x1 = to_f(kr[jj + half]);
-      s = fmaf(qs[g * hd + jj], x0 * cs - x1 * sn, s);
-      s = fmaf(qs[g * hd + jj + half], x1 * cs + x0 * sn, s);
+      const float x0 = kr[jj], x1 = kr[jj + half], c = cr[jj], sn = sr[jj];
+      s0 = fmaf(qg[jj], x0 * c - x1 * sn, s0);
+      s1 = fmaf(qg[jj + half], x1 * c + x0 * sn, s1);
     }
-    srs[r * gq + g] = s;
+    srs[i] = s0 + s1;
   }
   __syncthreads();
-  if (tid < gq) {
-    const int g = tid;
-    const int u_first0 = 0;
-    (void)u_first0;
-    float M = -INFINITY;
-    for (int c = fc; c <= lc; ++c) {
-      const int uf = tile_begin(c, args.n_tiles, args.ctas) / tpu;
-      const float* slot = args.part + (static_cast<int64_t>(c) * args.max_units + (u - uf)) * args.slot_floats;
-      M = fmaxf(M, slot[g]);
+  // ---- C: global max and denominator per query head
+  if (warp == 0) {
+    for (int g = 0; g < gq; ++g) {
+      float M = -INFINITY;
+      for (int i = lane; i < nslots; i += 32) M = fmaxf(M, ml[i * 16 + g]);
+      for (int r = lane; r < nsr; r += 32) M = fmaxf(M, srs[r * gq + g]);
+      M = warp_max(M);
+      float L = 0.f;
+      for (int i = lane; i < nslots; i += 32) {
+        const float f = exp2f(ml[i * 16 + g] - M);
+        sc[i * kMaxGQ + g] = f;
+        L = fmaf(ml[i * 16 + 8 + g], f, L);
+      }
+      for (int r = lane; r < nsr; r += 32) {
+        const float w = exp2f(srs[r * gq + g] - M);
+        srs[r * gq + g] = w;
+        L += w;
+      }
+      L = warp_sum(L);
+      if (lane == 0) { Mg[g] = M; Lg[g] = L; }
     }
-    for (int r = 0; r < nsr; ++r) M = fmaxf(M, srs[r * gq + g]);
-    float L = 0.f;
-    for (int c = fc; c <= lc; ++c) {
-      const int uf = tile_begin(c, args.n_tiles, args.ctas) / tpu;
-      const float* slot = args.part + (static_cast<int64_t>(c) * args.max_units + (u - uf)) * args.slot_floats;
-      const float f = exp2f(slot[g] - M);
-      sc[(c - fc) * kMaxGQ + g] = f;
-      L += slot[8 + g] * f;
-    }
-    for (int r = 0; r < nsr; ++r) {
-      const float w = exp2f(srs[r * gq + g] - M);
-      srs[r * gq + g] = w;
-      L += w;
-    }
-    Mg[g] = M;
-    Lg[g] = L;
   }
   __syncthreads();
-  for (int i = tid; i < gq * args.rV; i += blockDim.x) {
-    const int g = i / args.rV, c = i % args.rV;
-    float acc = 0.f;
-    for (int cc = fc; cc <= lc; ++cc) {
-      const int uf = tile_begin(cc, args.n_tiles, args.ctas) / tpu;
-      const float* slot = args.part + (static_cast<int64_t>(cc) * args.max_units + (u - uf)) * args.slot_floats;
-      acc = fmaf(slot[16 + g * args.rV + c], sc[(cc - fc) * kMaxGQ + g], acc);
+  // ---- D: value-basis sums over the slots (float4, 8 slots' loads in flight)
+  {
+    const int n4 = gq * args.rV / 4;
+    for (int i4 = tid; i4 < n4; i4 += blockDim.x) {
+      const int g = (4 * i4) / args.rV;
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int c0 = 0; c0 < nslots; c0 += 8) {
+        float4 v[8];
+#pragma unroll
+        for (int t = 0; t < 8; ++t)
+          v[t] = c0 + t < nslots ? reinterpret_cast<const float4*>(slot_ptr(fc + c0 + t) + 16)[i4]
+                                 : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+          if (c0 + t < nslots) {
+            const float f = sc[(c0 + t) * kMaxGQ + g];
+            acc.x = fmaf(v[t].x, f, acc.x);
+            acc.y = fmaf(v[t].y, f, acc.y);
+            acc.z = fmaf(v[t].z, f, acc.z);
+            acc.w = fmaf(v[t].w, f, acc.w);
+          }
+        }
+      }
+      reinterpret_cast<float4*>(Us)[i4] = acc;
     }
-    Us[i] = acc;
-  }
-  for (int i = tid; i < gq * hd; i += blockDim.x) {
-    const int g = i / hd, j = i % hd;
-    float acc = 0.f;
-    for (int r = 0; r < nsr; ++r)
-      acc = fmaf(srs[r * gq + g], to_f(srV[(static_cast<int64_t>(b) * nsr + r) * d + h * hd + j]), acc);
-    Ws[i] = acc;
   }
   __syncthreads();
-  for (int j = tid; j < hd; j += blockDim.x) {
+  // ---- E: output columns of this split
+  const bool vec = sizeof(T) == 2 && args.rV % 256 == 0 && args.rV <= 512;
+  for (int j = j0 + warp; j < j1; j += nwarps) {
     const T* br = BtV + b * args.sbv + static_cast<int64_t>(h * hd + j) * args.rV;
     float acc[kMaxGQ];
 #pragma unroll
     for (int g = 0; g < kMaxGQ; ++g) acc[g] = 0.f;
-    for (int c = 0; c < args.rV; ++c) {
-      const float bv = to_f(br[c]);
+    if (vec) {
+      // lane owns 8 consecutive rank columns in each 256-column half
+      const int nh = args.rV / 256;
+      uint4 w[2];
+#pragma unroll
+      for (int t = 0; t < 2; ++t)
+        w[t] = t < nh ? *reinterpret_cast<const uint4*>(br + 256 * t + 8 * lane) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+        if (t < nh) {
+          const uint32_t ww[4] = {w[t].x, w[t].y, w[t].z, w[t].w};
+          const int c0 = 256 * t + 8 * lane;
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 f = bf2_to_f2(ww[e]);
+#pragma unroll
+            for (int g = 0; g < kMaxGQ; ++g)
+              if (g < gq) {
+                acc[g] = fmaf(Us[g * args.rV + c0 + 2 * e], f.x, acc[g]);
+                acc[g] = fmaf(Us[g * args.rV + c0 + 2 * e + 1], f.y, acc[g]);
+              }
+          }
+        }
+      }
+    } else {
+      for (int c = lane; c < args.rV; c += 32) {
+        const float bv = to_f(br[c]);
+#pragma unroll
+        for (int g = 0; g < kMaxGQ; ++g)
+          if (g < gq) acc[g] = fmaf(Us[g * args.rV + c], bv, acc[g]);
+      }
+    }
+    for (int r = lane; r < nsr; r += 32) {
+      const float v = wV[r * hdp + j];
 #pragma unroll
       for (int g = 0; g < kMaxGQ; ++g)
-        if (g < gq) acc[g] = fmaf(Us[g * args.rV + c], bv, acc[g]);
+        if (g < gq) acc[g] = fmaf(srs[r * gq + g], v, acc[g]);
     }
 #pragma unroll
-    for (int g = 0; g < kMaxGQ; ++g)
-      if (g < gq)
-        out[(static_cast<int64_t>(b) * args.Hq + h * gq + g) * hd + j] = (acc[g] + Ws[g * hd + j]) / Lg[g];
+    for (int g = 0; g < kMaxGQ; ++g) {
+      if (g >= gq) break;
+      const float v = warp_sum(acc[g]);
+      if (lane == 0) out[(static_cast<int64_t>(b) * args.Hq + h * gq + g) * hd + j] = v / Lg[g];
+    }
   }
-  (void)nslots;
 }
 
 size_t combine_smem(int gq, int rV, int hd, int nsr) {
-  return (static_cast<size_t>(gq) * rV + 2 * gq * hd + nsr * gq + 2 * kMaxGQ + 64 * kMaxGQ + 8) * 4 +
-         (hd / 2) * 8 + 16;
+  return (static_cast<size_t>(gq) * rV + static_cast<size_t>(gq) * hd + 2 * static_cast<size_t>(nsr) * (hd + 1) +
+          2 * static_cast<size_t>(nsr) * (hd / 2 + 1) + static_cast<size_t>(nsr) * gq + kMaxSlots * 16 +
+          kMaxSlots * kMaxGQ + 2 * kMaxGQ + 8) * 4 + 128 * 8 + 32;
 }
 
 size_t simt_smem(int gq, int rV, int hd) {
@@ -768,7 +1129,7 @@ size_t simt_smem(int gq, int rV, int hd) {
 
 bool tc_shape_ok(const xkv_sr_params* p) {
   const int gq = p->n_q_heads / p->n_kv_heads;
-  return p->dtype == XKV_BF16 && p->head_dim == 128 && p->chunk == 8 && p->rank_k % 64 == 0 &&
+  return p->dtype == XKV_BF16 && p->head_dim == 128 && p->chunk == 8 && p->rank_k % (64 * kKAtoms) == 0 &&
          p->rank_v % 64 == 0 && p->rank_k <= 2048 && p->rank_v <= 512 && gq <= kMaxGQ &&
          p->a_k_batch_stride % 8 == 0 && p->a_v_batch_stride % 8 == 0 && p->bt_k_batch_stride % 8 == 0 &&
          !force_simt();
@@ -823,10 +1184,11 @@ static xkv_status sr_launch_t(const xkv_sr_params* p, const SRPlan& plan, const 
   }
   // 2. exact top-k
   {
-    const size_t smem = static_cast<size_t>(n_mid) * 4;
+    const int64_t per = (n_mid + kTopkThreads - 1) / kTopkThreads;
+    const size_t smem = static_cast<size_t>(per * kTopkThreads + n_mid) * 4;
     if (smem > 48 * 1024)
       cudaFuncSetAttribute(sr_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-    sr_topk_kernel<<<plan.units, 1024, smem, st>>>(scores, sel, sel_out, n_mid, p->topk);
+    sr_topk_kernel<<<plan.units, kTopkThreads, smem, st>>>(scores, sel, sel_out, n_mid, p->topk);
   }
   AttendArgs a;
   a.sel = sel;
@@ -849,16 +1211,18 @@ static xkv_status sr_launch_t(const xkv_sr_params* p, const SRPlan& plan, const 
   a.max_units = plan.max_units_per_cta;
   a.slot_floats = static_cast<int>(plan.slot_floats);
   a.theta = p->rope_theta;
+  for (int j = 0; j < 128; ++j) a.ft[j] = j < p->head_dim / 2 ? rope_turns(p->rope_theta, j, p->head_dim) : 0.0;
   // 3. selective reconstruction + attention partials
   if (plan.tc) {
     CUtensorMap mAK, mBK, mAV;
     const int d = p->n_kv_heads * p->head_dim;
     {
-      const uint64_t dims[3] = {static_cast<uint64_t>(p->rank_k), static_cast<uint64_t>(p->T),
+      // (64 columns, token rows, 64-column atoms, batch): one box = 8 rows x kKAtoms atoms
+      const uint64_t dims[4] = {64, static_cast<uint64_t>(p->T), static_cast<uint64_t>(p->rank_k / 64),
                                 static_cast<uint64_t>(p->batch)};
-      const uint64_t str[2] = {static_cast<uint64_t>(p->rank_k) * 2, static_cast<uint64_t>(p->a_k_batch_stride) * 2};
-      const uint32_t box[3] = {64, 8, 1};
-      if (!make_tmap(&mAK, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, A_K, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B))
+      const uint64_t str[3] = {static_cast<uint64_t>(p->rank_k) * 2, 128, static_cast<uint64_t>(p->a_k_batch_stride) * 2};
+      const uint32_t box[4] = {64, 8, static_cast<uint32_t>(kKAtoms), 1};
+      if (!make_tmap(&mAK, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, A_K, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B))
         return XKV_ERR_CUDA;
     }
     {
@@ -872,11 +1236,12 @@ static xkv_status sr_launch_t(const xkv_sr_params* p, const SRPlan& plan, const 
         return XKV_ERR_CUDA;
     }
     {
-      const uint64_t dims[3] = {static_cast<uint64_t>(p->rank_v), static_cast<uint64_t>(p->T),
+      // (64 columns, token rows, atoms, batch): one box = 8 rows x the full rank
+      const uint64_t dims[4] = {64, static_cast<uint64_t>(p->T), static_cast<uint64_t>(p->rank_v / 64),
                                 static_cast<uint64_t>(p->batch)};
-      const uint64_t str[2] = {static_cast<uint64_t>(p->rank_v) * 2, static_cast<uint64_t>(p->a_v_batch_stride) * 2};
-      const uint32_t box[3] = {64, 8, 1};
-      if (!make_tmap(&mAV, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, A_V, dims, str, box, CU_TENSOR_MAP_SWIZZLE_NONE))
+      const uint64_t str[3] = {static_cast<uint64_t>(p->rank_v) * 2, 128, static_cast<uint64_t>(p->a_v_batch_stride) * 2};
+      const uint32_t box[4] = {64, 8, static_cast<uint32_t>(p->rank_v / 64), 1};
+      if (!make_tmap(&mAV, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, A_V, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B))
         return XKV_ERR_CUDA;
     }
     const size_t smem = attend_tc_smem();
@@ -908,7 +1273,8 @@ static xkv_status sr_launch_t(const xkv_sr_params* p, const SRPlan& plan, const 
     if (smem > 48 * 1024)
       cudaFuncSetAttribute(sr_combine_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(smem));
-    sr_combine_kernel<T><<<plan.units, 256, smem, st>>>(static_cast<const T*>(q), static_cast<const T*>(Bt_V),
+    sr_combine_kernel<T><<<dim3(plan.units, kCombineSplit), kCombineThreads, smem, st>>>(
+        static_cast<const T*>(q), static_cast<const T*>(Bt_V),
                                                          static_cast<const T*>(sr_K), static_cast<const T*>(sr_V),
                                                          a, p->head_dim, out);
   }

@@ -222,7 +222,7 @@ static xkv_status check_sr(const xkv_sr_params* p) {
   if (p->dtype != XKV_F32 && p->dtype != XKV_BF16) return XKV_ERR_INVALID_ARG;
   if (!(p->rope_theta > 1.0f)) return XKV_ERR_INVALID_ARG;
   const int gq = p->n_q_heads / p->n_kv_heads;
-  if (gq > 8 || p->head_dim > 256 || p->sink + p->recent > 64 || n_mid * 4 > 200 * 1024 || p->rank_v > 4096 ||
+  if (gq > 8 || p->head_dim > 256 || p->sink + p->recent > 64 || n_mid * 8 > 200 * 1024 || p->rank_v > 4096 ||
       p->topk > 1024)
     return XKV_ERR_UNSUPPORTED;
   if (p->T > (int64_t(1) << 30)) return XKV_ERR_UNSUPPORTED;

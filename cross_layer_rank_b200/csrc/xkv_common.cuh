@@ -134,26 +134,42 @@ __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
 
 // ------------------------------------------------------------ tcgen05
 // Shared-memory matrix descriptor for a K-major operand tile stored with the
-// 128-byte swizzle: rows of 64 bf16 (128 B), 8-row core groups 1024 B apart.
+// 128-byte swizzle: rows of 64 bf16 (128 B), 8-row core groups `sbo` bytes
+// apart (1024 when the groups are packed).
 // Fields: start address >> 4 [0,14), leading byte offset >> 4 [16,30) (unused
 // for swizzled K-major, set to 1), stride byte offset >> 4 [32,46), descriptor
 // version 1 [46,48), swizzle mode [61,64) = 2 (128B).
-__device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t smem_addr) {
+__device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t smem_addr, uint32_t sbo = 1024u) {
   uint64_t d = 0;
   d |= static_cast<uint64_t>((smem_addr >> 4) & 0x3FFFu);
   d |= static_cast<uint64_t>(1u) << 16;
-  d |= static_cast<uint64_t>(1024u >> 4) << 32;
+  d |= static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32;
   d |= static_cast<uint64_t>(1u) << 46;
   d |= static_cast<uint64_t>(2u) << 61;
   return d;
 }
 
-// Instruction descriptor of kind::f16 with bf16 A/B, f32 accumulator, both
-// operands K-major, tile M x N.
-__host__ __device__ constexpr uint32_t umma_idesc_bf16(int M, int N) {
+// Descriptor of an MN-major operand in the 128-byte swizzle: atoms of 8 K-rows
+// x 64 bf16 (128 B) contiguous along M/N; `lbo` = bytes between atoms along
+// M/N, `sbo` = bytes between 8-row groups along K.
+__device__ __forceinline__ uint64_t umma_desc_sw128_mn(uint32_t smem_addr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((smem_addr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16;
+  d |= static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32;
+  d |= static_cast<uint64_t>(1u) << 46;
+  d |= static_cast<uint64_t>(2u) << 61;
+  return d;
+}
+
+// Instruction descriptor of kind::f16 with bf16 A/B, f32 accumulator, tile
+// M x N; operands K-major unless a_mn / b_mn select MN-major.
+__host__ __device__ constexpr uint32_t umma_idesc_bf16(int M, int N, bool a_mn = false, bool b_mn = false) {
   return (1u << 4)                                   // D format: f32
          | (1u << 7)                                 // A format: bf16
          | (1u << 10)                                // B format: bf16
+         | (static_cast<uint32_t>(a_mn) << 15)       // A major
+         | (static_cast<uint32_t>(b_mn) << 16)       // B major
          | (static_cast<uint32_t>(N >> 3) << 17)     // N / 8
          | (static_cast<uint32_t>(M >> 4) << 24);    // M / 16
 }
