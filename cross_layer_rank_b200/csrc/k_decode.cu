@@ -107,7 +107,7 @@ __global__ void __launch_bounds__(256) sr_score_kernel(const T* __restrict__ q, 
   const int64_t c1 = min(c0 + chunks_per_block, n_mid);
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const T* base = lm + static_cast<int64_t>(unit) * n_mid * hd;
-  float* out = scores + static_cast<int64_t>(unit) * n_mid;
+  float* out = scores + static_cast<int64_t>(unit) * ((n_mid + 3) & ~int64_t(3));
   if (sizeof(T) == 2 && hd == 128) {
     // 16 lanes x 16 B cover one 256-B landmark row; a warp scores 2 rows per
     // load and keeps 8 rows (4 loads per lane) in flight.
@@ -151,14 +151,17 @@ __global__ void __launch_bounds__(256) sr_score_kernel(const T* __restrict__ q, 
 
 // ------------------------------------------------------------- sr_topk
 // Exact top-k of one unit's chunk scores (1024 threads, one CTA per unit).
-//   1. scores -> order-preserving 32-bit keys; their range [lo, hi];
+//   1. scores -> order-preserving 32-bit keys (coalesced 16-byte loads of the
+//      padded score row) and their range [lo, hi];
 //   2. a 1024-bucket histogram of floor((key - lo) * 1024 / (hi - lo + 1))
 //      (fp32 arithmetic: a monotone map, so every key of a higher bucket is
 //      larger than every key of a lower one);
 //   3. a suffix scan finds the boundary bucket B holding the k-th largest key;
 //      keys above B are kept, `need` more come from B;
 //   4. the keys of B are compacted in ascending index order and the `need`
-//      largest of them found bit by bit (ties -> lower index);
+//      largest of them chosen (ties -> lower index): up to 1024 candidates by
+//      counting, per candidate (one warp each), the candidates ranked above it;
+//      more by 8-bit radix passes and an ordered scan of the equal keys;
 //   5. an ordered compaction writes the selection ascending by chunk.
 // Thread t owns the contiguous index segment [t per, (t+1) per), stored
 // transposed (element j of every thread's segment is contiguous) so that the
@@ -171,33 +174,175 @@ __device__ __forceinline__ uint32_t topk_bucket(uint32_t key, uint32_t lo, float
   return min(static_cast<uint32_t>(x), static_cast<uint32_t>(kBuckets - 1));
 }
 
-__global__ void __launch_bounds__(kTopkThreads) sr_topk_kernel(const float* __restrict__ scores, int32_t* __restrict__ sel,
-                                                               int32_t* __restrict__ sel_out, int64_t n_mid, int k) {
-  extern __shared__ uint32_t ksm[];  // [per][1024] keys (transposed), then [n] candidate indices
+// ------------------------------------------------------------ sr_window
+// Raw sink/recent window of one unit, computed by extra blocks of the top-k
+// grid (the top-k itself occupies one SM per unit): the uncompressed rows are
+// staged in shared memory with one round of loads, RoPE is applied in place at
+// their true positions, then the scores, their softmax statistics and the
+// unnormalised weighted value sum o_g = sum_t 2^(s_gt - m_g) V_t.
+// Window slot layout: [0..7] m_g (log2 domain), [8..15] l_g, [16 + g hd + j] o_g[j].
+struct WinArgs {
+  const void* q;
+  const void* srK;
+  const void* srV;
+  float* win;
+  int64_t T;
+  int Hq, Hkv, hd, sink, recent;
+  double ft[128];  // RoPE frequency of pair j in turns per position
+};
+
+inline size_t window_smem(int gq, int hd, int nsr) {
+  return 128 * 8 + (static_cast<size_t>(nsr) * (2 * hd + 1) + static_cast<size_t>(gq) * hd + nsr * kMaxGQ) * 4;
+}
+
+template <typename T>
+__device__ void window_partial(const WinArgs& wa, int unit, uint8_t* smem) {
+  const int hd = wa.hd, gq = wa.Hq / wa.Hkv, half = hd / 2, nsr = wa.sink + wa.recent, d = wa.Hkv * hd;
+  const int b = unit / wa.Hkv, h = unit % wa.Hkv;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nt = blockDim.x, nwarps = nt >> 5;
+  const int ks = hd + 1;  // padded key row stride
+  double* fts = reinterpret_cast<double*>(smem);  // [128]
+  float* wK = reinterpret_cast<float*>(fts + 128);  // [nsr][hd + 1]
+  float* wV = wK + nsr * ks;                        // [nsr][hd]
+  float* qs = wV + nsr * hd;                        // [gq][hd]
+  float* ws = qs + gq * hd;                         // [nsr][8] scores, then weights
+  const T* q = static_cast<const T*>(wa.q);
+  const T* srK = static_cast<const T*>(wa.srK);
+  const T* srV = static_cast<const T*>(wa.srV);
+  float* slot = wa.win + static_cast<int64_t>(unit) * (16 + gq * hd);
+  const float qscale = rsqrtf(static_cast<float>(hd)) * kLog2e;
+  // 1. loads
+  for (int i = tid; i < gq * hd; i += nt) qs[i] = ldf(q + (static_cast<int64_t>(b) * wa.Hq + h * gq) * hd + i) * qscale;
+  for (int j = tid; j < half; j += nt) fts[j] = wa.ft[j];
+  if (sizeof(T) == 2 && hd % 8 == 0) {
+    const int vpr = hd / 8;
+    for (int v = tid; v < 2 * nsr * vpr; v += nt) {
+      const int mat = v / (nsr * vpr), r = (v / vpr) % nsr, c8 = v % vpr;
+      const T* src = (mat ? srV : srK) + (static_cast<int64_t>(b) * nsr + r) * d + h * hd + c8 * 8;
+      const uint4 w = *reinterpret_cast<const uint4*>(src);
+      float* dst = mat ? wV + r * hd + c8 * 8 : wK + r * ks + c8 * 8;
+      const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 f = bf2_to_f2(ww[e]);
+        dst[2 * e] = f.x;
+        dst[2 * e + 1] = f.y;
+      }
+    }
+  } else {
+    for (int i = tid; i < nsr * hd; i += nt) {
+      const int r = i / hd, j = i % hd;
+      const int64_t off = (static_cast<int64_t>(b) * nsr + r) * d + h * hd + j;
+      wK[r * ks + j] = ldf(srK + off);
+      wV[r * hd + j] = ldf(srV + off);
+    }
+  }
+  __syncthreads();
+  // 2. RoPE of the window keys at their positions
+  for (int i = tid; i < nsr * half; i += nt) {
+    const int r = i / half, jj = i % half;
+    const int64_t t = r < wa.sink ? r : wa.T - wa.recent + (r - wa.sink);
+    float c, sn;
+    rope_cs(fts[jj], static_cast<double>(t), &c, &sn);
+    float* kr = wK + r * ks;
+    const float x0 = kr[jj], x1 = kr[jj + half];
+    kr[jj] = x0 * c - x1 * sn;
+    kr[jj + half] = x1 * c + x0 * sn;
+  }
+  __syncthreads();
+  // 3. scores: warp per row
+  for (int r = warp; r < nsr; r += nwarps) {
+    float acc[kMaxGQ];
+#pragma unroll
+    for (int g = 0; g < kMaxGQ; ++g) acc[g] = 0.f;
+    for (int j = lane; j < hd; j += 32) {
+      const float kv = wK[r * ks + j];
+#pragma unroll
+      for (int g = 0; g < kMaxGQ; ++g)
+        if (g < gq) acc[g] = fmaf(qs[g * hd + j], kv, acc[g]);
+    }
+#pragma unroll
+    for (int g = 0; g < kMaxGQ; ++g) {
+      if (g >= gq) break;
+      const float v = warp_sum(acc[g]);
+      if (lane == 0) ws[r * kMaxGQ + g] = v;
+    }
+  }
+  __syncthreads();
+  // 4. softmax statistics: warp per query head
+  for (int g = warp; g < gq; g += nwarps) {
+    float m = -INFINITY;
+    for (int r = lane; r < nsr; r += 32) m = fmaxf(m, ws[r * kMaxGQ + g]);
+    m = warp_max(m);
+    float l = 0.f;
+    for (int r = lane; r < nsr; r += 32) {
+      const float w = exp2f(ws[r * kMaxGQ + g] - m);
+      ws[r * kMaxGQ + g] = w;
+      l += w;
+    }
+    l = warp_sum(l);
+    if (lane == 0) { slot[g] = m; slot[8 + g] = l; }
+  }
+  __syncthreads();
+  // 5. o_g[j]: thread per (g, j)
+  for (int i = tid; i < gq * hd; i += nt) {
+    const int g = i / hd, j = i % hd;
+    float acc = 0.f;
+    for (int r = 0; r < nsr; ++r) acc = fmaf(ws[r * kMaxGQ + g], wV[r * hd + j], acc);
+    slot[16 + i] = acc;
+  }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kTopkThreads) sr_topk_kernel(const float* __restrict__ scores, int64_t ld,
+                                                               int32_t* __restrict__ sel,
+                                                               int32_t* __restrict__ sel_out, int64_t n_mid, int k,
+                                                               int units, const __grid_constant__ WinArgs wa) {
+  extern __shared__ uint32_t ksm[];  // [per][1024] keys (transposed), [n] candidate keys, [n] decisions
+  if (static_cast<int>(blockIdx.x) >= units) {
+    window_partial<T>(wa, blockIdx.x - units, reinterpret_cast<uint8_t*>(ksm));
+    return;
+  }
   __shared__ uint32_t hist[kBuckets];
   __shared__ uint32_t warp_tot[32];
-  __shared__ uint32_t s_wcnt[3 * 64];
-  __shared__ uint32_t s_lo, s_hi, s_total, s_bucket, s_need;
+  __shared__ uint32_t s_lo, s_hi, s_total, s_bucket, s_need, s_all, s_digit, s_kk, s_eq;
   const int unit = blockIdx.x;
   const int n = static_cast<int>(n_mid);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int nt = static_cast<int>(blockDim.x), nwarps = nt >> 5;
   const int per = (n + nt - 1) / nt;
+  const float inv_per = 1.0f / static_cast<float>(per);
   uint32_t* ckey = ksm + per * nt;
-  const float* sc = scores + static_cast<int64_t>(unit) * n_mid;
-  // 1. keys and their range
-  uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
-  for (int j = 0; j < per; ++j) {
-    const int i = tid * per + j;
-    const uint32_t key = i < n ? order_key(sc[i]) : 0u;
-    ksm[j * nt + tid] = key;
-    if (i < n) { kmin = min(kmin, key); kmax = max(kmax, key); }
-  }
+  uint8_t* ckeep = reinterpret_cast<uint8_t*>(ckey + n);
   hist[tid] = 0u;
   if (tid == 0) { s_lo = 0xFFFFFFFFu; s_hi = 0u; }
-  __syncthreads();
+  // 1. keys (row start 16-byte aligned: ld is a multiple of 4) and their range
+  uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
+  {
+    const float4* row = reinterpret_cast<const float4*>(scores + static_cast<int64_t>(unit) * ld);
+    const int n4 = (n + 3) / 4;
+    for (int i4 = tid; i4 < n4; i4 += nt) {
+      const float4 v = row[i4];
+      const float vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int i = 4 * i4 + e;
+        if (i < n) {
+          const uint32_t key = order_key(vv[e]);
+          // i / per by a float product: exact, since (i + 0.5) / per lies at
+          // least 0.5 / per from an integer, i + 0.5 is exact (n < 2^23) and
+          // the product's relative error is below 2^-23 (per <= 32 here)
+          const int t = static_cast<int>((static_cast<float>(i) + 0.5f) * inv_per);
+          ksm[(i - t * per) * nt + t] = key;
+          kmin = min(kmin, key);
+          kmax = max(kmax, key);
+        }
+      }
+    }
+  }
   kmin = __reduce_min_sync(0xffffffffu, kmin);
   kmax = __reduce_max_sync(0xffffffffu, kmax);
+  __syncthreads();
   if (lane == 0) { atomicMin(&s_lo, kmin); atomicMax(&s_hi, kmax); }
   __syncthreads();
   const uint32_t lo = s_lo;
@@ -222,101 +367,110 @@ __global__ void __launch_bounds__(kTopkThreads) sr_topk_kernel(const float* __re
   for (int j = 0; j < cnt; ++j) nc += topk_bucket(ksm[j * nt + tid], lo, scale) == B;
   uint32_t cpos = block_exclusive_scan(nc, warp_tot, &s_total);
   const uint32_t m = s_total;
+  const uint32_t cbase = cpos;
   for (int j = 0; j < cnt; ++j) {
     const uint32_t key = ksm[j * nt + tid];
     if (topk_bucket(key, lo, scale) == B) ckey[cpos++] = key;
   }
   __syncthreads();
-  // bit-serial selection of the `need` largest candidate keys: warp 0 runs the
-  // passes when the list is short, the whole block otherwise
-  __shared__ uint32_t s_prefix, s_himask, s_kk, s_all;
-  const bool block_wide = m > 2048;
   if (m == need) {
-    if (tid == 0) { s_prefix = 0u; s_himask = 0u; s_kk = need; s_all = 1u; }
-  } else if (!block_wide) {
-    if (warp == 0) {
-      uint32_t prefix = 0u, himask = 0u, kk = need, all = 0u;
-      for (int bit = 31; bit >= 0; --bit) {
-        uint32_t c = 0, cm = 0;
-        for (uint32_t i = lane; i < m; i += 32) {
-          const uint32_t key = ckey[i];
-          const uint32_t match = (key & himask) == prefix;
-          cm += match;
-          c += match & (key >> bit);
-        }
-        const uint32_t c1 = __reduce_add_sync(0xffffffffu, c);
-        const uint32_t cand = __reduce_add_sync(0xffffffffu, cm);
-        if (cand == kk) { all = 1u; break; }
-        if (c1 >= kk) prefix |= 1u << bit;
-        else kk -= c1;
-        himask |= 1u << bit;
+    if (tid == 0) s_all = 1u;
+  } else if (m <= static_cast<uint32_t>(nt)) {
+    // rank of candidate c: candidates with a larger key, or an equal key and
+    // a lower index; the `need` lowest ranks are kept
+    if (tid == 0) s_all = 0u;
+    for (uint32_t c = warp; c < m; c += nwarps) {
+      const uint32_t key = ckey[c];
+      uint32_t r = 0;
+      for (uint32_t o = lane; o < m; o += 32) {
+        const uint32_t ko = ckey[o];
+        r += (ko > key) || (ko == key && o < c);
       }
-      if (lane == 0) { s_prefix = prefix; s_himask = himask; s_kk = kk; s_all = all; }
+      r = __reduce_add_sync(0xffffffffu, r);
+      if (lane == 0) ckeep[c] = r < need;
     }
   } else {
-    uint32_t prefix = 0u, himask = 0u, kk = need, all = 0u;
-    int pass = 0;
-    for (int bit = 31; bit >= 0; --bit, ++pass) {
-      uint32_t c = 0, cm = 0;
-      for (uint32_t i = tid; i < m; i += nt) {
-        const uint32_t key = ckey[i];
-        const uint32_t match = (key & himask) == prefix;
-        cm += match;
-        c += match & (key >> bit);
-      }
-      c = __reduce_add_sync(0xffffffffu, c);
-      cm = __reduce_add_sync(0xffffffffu, cm);
-      uint32_t* slot = s_wcnt + (pass % 3) * 64;
-      if (lane == 0) { slot[warp] = c; slot[32 + warp] = cm; }
+    // 8-bit radix passes over the candidates: the k-th key's digits top down
+    uint32_t prefix = 0u, mask = 0u, kk = need;
+    bool all = false;
+    for (int shift = 24; shift >= 0 && !all; shift -= 8) {
+      if (tid < 256) hist[tid] = 0u;
       __syncthreads();
-      const uint32_t c1 = __reduce_add_sync(0xffffffffu, lane < nwarps ? slot[lane] : 0u);
-      const uint32_t cand = __reduce_add_sync(0xffffffffu, lane < nwarps ? slot[32 + lane] : 0u);
-      if (cand == kk) { all = 1u; break; }
-      if (c1 >= kk) prefix |= 1u << bit;
-      else kk -= c1;
-      himask |= 1u << bit;
+      for (uint32_t c = tid; c < m; c += nt) {
+        const uint32_t key = ckey[c];
+        if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
+      }
+      __syncthreads();
+      if (warp == 0) {
+        // lane l holds digits 255 - 8l .. 248 - 8l (descending)
+        uint32_t h[8], sum = 0;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) { h[e] = hist[255 - 8 * lane - e]; sum += h[e]; }
+        uint32_t incl = sum;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += y;
+        }
+        uint32_t above = incl - sum;
+        if (above < kk && incl >= kk) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            if (above < kk && above + h[e] >= kk) {
+              s_digit = 255 - 8 * lane - e;
+              s_kk = kk - above;
+              s_eq = h[e];
+            }
+            above += h[e];
+          }
+        }
+      }
+      __syncthreads();
+      prefix |= s_digit << shift;
+      mask |= 255u << shift;
+      kk = s_kk;
+      all = s_eq == kk;  // every candidate with this prefix is kept
     }
-    if (tid == 0) { s_prefix = prefix; s_himask = himask; s_kk = kk; s_all = all; }
+    // decisions: above the prefix kept; equal to it kept when all are, else
+    // the first kk in index order (ordered scan over contiguous candidate runs)
+    const uint32_t cpt = (m + nt - 1) / nt, c0 = min(m, tid * cpt), c1 = min(m, c0 + cpt);
+    uint32_t eq = 0;
+    for (uint32_t c = c0; c < c1; ++c) eq += (ckey[c] & mask) == prefix;
+    uint32_t rank = block_exclusive_scan(eq, warp_tot, &s_total);
+    for (uint32_t c = c0; c < c1; ++c) {
+      const uint32_t km = ckey[c] & mask;
+      bool keep;
+      if (km > prefix) keep = true;
+      else if (km < prefix) keep = false;
+      else keep = all || rank++ < kk;
+      ckeep[c] = keep;
+    }
+    if (tid == 0) s_all = 0u;
   }
   __syncthreads();
-  const uint32_t prefix = s_prefix, himask = s_himask, kk = s_kk;
   const bool all_taken = s_all != 0u;
-  // inside B: keep keys above tau and the first need_eq keys equal to it, or
-  // every candidate whose top bits reach the prefix (all_taken)
-  const uint32_t tau = prefix;
-  const uint32_t need_eq = all_taken ? 0xFFFFFFFFu : kk;
-  auto in_b_keep = [&](uint32_t key, uint32_t& e) -> bool {
-    if (all_taken) return (key & himask) >= prefix;
-    if (key > tau) return true;
-    if (key == tau) { const bool t = e < need_eq; ++e; return t; }
-    return false;
-  };
-  // 5. ordered compaction of the selection
-  uint32_t n_eq = 0;
-  if (!all_taken)
-    for (int j = 0; j < cnt; ++j) {
-      const uint32_t key = ksm[j * nt + tid];
-      n_eq += (key == tau && topk_bucket(key, lo, scale) == B);
-    }
-  const uint32_t eq_before = block_exclusive_scan(n_eq, warp_tot, &s_total);
+  // 5. ordered compaction of the selection: a key of B is kept when its
+  // candidate decision says so (candidates are numbered in index order)
   uint32_t n_sel = 0;
   {
-    uint32_t e = eq_before;
+    uint32_t ci = cbase;
     for (int j = 0; j < cnt; ++j) {
-      const uint32_t key = ksm[j * nt + tid];
-      const uint32_t bk = topk_bucket(key, lo, scale);
-      n_sel += bk > B || (bk == B && in_b_keep(key, e));
+      const uint32_t bk = topk_bucket(ksm[j * nt + tid], lo, scale);
+      if (bk == B) n_sel += all_taken || ckeep[ci++];
+      else n_sel += bk > B;
     }
   }
   uint32_t pos = block_exclusive_scan(n_sel, warp_tot, &s_total);
   {
-    uint32_t e = eq_before;
+    uint32_t ci = cbase;
     int32_t* o = sel + static_cast<int64_t>(unit) * k;
     int32_t* o2 = sel_out ? sel_out + static_cast<int64_t>(unit) * k : nullptr;
     for (int j = 0; j < cnt; ++j) {
-      const uint32_t key = ksm[j * nt + tid];
-      const uint32_t bk = topk_bucket(key, lo, scale);
-      if (bk > B || (bk == B && in_b_keep(key, e))) {
+      const uint32_t bk = topk_bucket(ksm[j * nt + tid], lo, scale);
+      bool take;
+      if (bk == B) take = all_taken || ckeep[ci++];
+      else take = bk > B;
+      if (take) {
         o[pos] = i0 + j;
         if (o2) o2[pos] = i0 + j;
         ++pos;
@@ -394,6 +548,7 @@ __global__ void __launch_bounds__(kAttendThreads, 1)
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int NKA = args.rK / 64;
+  const int NKS = (NKA + kKAtoms - 1) / kKAtoms;  // key stages per tile
   const int NMB = (args.rV + 127) / 128;  // value M-blocks of 128 rank columns
   const int NAVp = 2 * NMB;               // 64-column atoms per value slab (zero-padded)
   const int NAV = args.rV / 64;           // atoms actually loaded
@@ -483,15 +638,18 @@ __global__ void __launch_bounds__(kAttendThreads, 1)
         for (int ch = 0; ch < kTileChunks; ++ch) rows[ch] = ch < nch ? args.sink + su[ch] * 8 : 0;
         // one 4-D box per chunk covers kKAtoms atoms (8 rows x 128 columns);
         // the Bt_K atoms of the stage follow on their own ring (L2 hits)
+        // (an odd atom count leaves the last box half out of range: TMA fills
+        // it with zeros and still delivers the whole box; it gets no MMA)
         bool ok = true;
-        for (int sk = 0; sk < NKA / kKAtoms && ok; ++sk, ++ks) {
+        for (int sk = 0; sk < NKS && ok; ++sk, ++ks) {
           const int slot = ks % kKStages;
           if (!mbar_wait(&kempty[slot], ((ks / kKStages) & 1) ^ 1, args.status)) { *abort_flag = 1; ok = false; break; }
           mbar_arrive_expect_tx(&kfull[slot], nch * kKAtoms * 1024);
           for (int ch = 0; ch < nch; ++ch)
             tma_load_4d(Ka + slot * kKStageBytes + ch * kKAtoms * 1024, &mapAK, &kfull[slot], 0, rows[ch],
                         sk * kKAtoms, b);
-          for (int a = 0; a < kKAtoms; ++a, ++bs) {
+          const int na = min(kKAtoms, NKA - sk * kKAtoms);
+          for (int a = 0; a < na; ++a, ++bs) {
             const int bslot = bs % kBStages;
             if (!mbar_wait(&bempty[bslot], ((bs / kBStages) & 1) ^ 1, args.status)) { *abort_flag = 1; ok = false; break; }
             mbar_arrive_expect_tx(&bfull[bslot], kAtomBytes);
@@ -537,10 +695,11 @@ __global__ void __launch_bounds__(kAttendThreads, 1)
         if (!mbar_wait(&accempty[buf], ((j >> 1) & 1) ^ 1, args.status)) return false;
         tc_fence_after();
         const uint32_t dtm = tmem + buf * 128;
-        for (int sk = 0; sk < NKA / kKAtoms; ++sk, ++ks) {
+        for (int sk = 0; sk < NKS; ++sk, ++ks) {
           const int slot = ks % kKStages;
           if (!mbar_wait(&kfull[slot], (ks / kKStages) & 1, args.status)) return false;
-          for (int a = 0; a < kKAtoms; ++a, ++bs) {
+          const int na = min(kKAtoms, NKA - sk * kKAtoms);
+          for (int a = 0; a < na; ++a, ++bs) {
             const int bslot = bs % kBStages;
             if (!mbar_wait(&bfull[bslot], (bs / kBStages) & 1, args.status)) return false;
             tc_fence_after();
@@ -898,42 +1057,40 @@ __global__ void __launch_bounds__(256) sr_attend_simt_kernel(const T* __restrict
 // ----------------------------------------------------------- sr_combine
 // Grid (unit, column split of kCombineSplit), 256 threads.  Each phase issues
 // all of its loads before using them (one memory round trip per phase):
-//   A  queries, the unit's raw window rows, the partial-slot statistics, and
-//      the RoPE angles of the window positions;
-//   B  window scores (thread per row x query head, padded rows: no bank
-//      conflicts);  C  M_g and L_g;  D  U_g = sum over slots of u 2^(m - M);
-//   E  o_g[j] = (U_g . Bt_V[h hd + j] + sum_t p_gt V_t[j]) / L_g for the
-//      split's columns (warp per column, 16-byte loads of the Bt_V row).
+//   A  (m, l) of the unit's partial slots and of its window partial;
+//   C  M_g, the slot factors 2^(m - M_g) and L_g (warp per query head);
+//   D  U_g = sum over slots of u 2^(m - M_g), kept in shared memory in an
+//      order where lane-consecutive 8-column groups are word-consecutive;
+//   E  o_g[j] = (U_g . Bt_V[h hd + j] + 2^(m_w - M_g) o_w,g[j]) / L_g for the
+//      split's columns (warp per column, 16-byte loads of the Bt_V rows of
+//      all of the warp's columns issued first).
 constexpr int kCombineSplit = 4;
 constexpr int kCombineThreads = 256;
 constexpr int kMaxSlots = 64;
+constexpr int kCombineColsPerWarp = 4;
 
 template <typename T>
-__global__ void __launch_bounds__(kCombineThreads) sr_combine_kernel(const T* __restrict__ q, const T* __restrict__ BtV,
-                                                                     const T* __restrict__ srK,
-                                                                     const T* __restrict__ srV, const AttendArgs args,
-                                                                     int hd, float* __restrict__ out) {
-  extern __shared__ double smd[];
+__global__ void __launch_bounds__(kCombineThreads) sr_combine_kernel(const T* __restrict__ BtV,
+                                                                     const float* __restrict__ win,
+                                                                     const AttendArgs args, int hd,
+                                                                     float* __restrict__ out) {
+  extern __shared__ float4 smf4[];
   const int gq = args.Hq / args.Hkv;
-  const int nsr = args.sink + args.recent;
   const int u = blockIdx.x, b = u / args.Hkv, h = u % args.Hkv;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nwarps = blockDim.x >> 5;
   const int tpu = args.tiles_per_unit;
-  const int d = args.Hkv * hd, half = hd / 2;
-  const int hdp = hd + 1;  // padded row stride
+  const int rV = args.rV;
   const int cols = (hd + kCombineSplit - 1) / kCombineSplit, j0 = blockIdx.y * cols, j1 = min(hd, j0 + cols);
-  double* ftab = smd;                      // [128] RoPE turns (first: 8-byte aligned)
-  float* Us = reinterpret_cast<float*>(smd + 128);  // [gq][rV] (16-byte aligned)
-  float* qs = Us + gq * args.rV;           // [gq][hd]
-  float* wK = qs + gq * hd;                // [nsr][hd+1] raw window keys
-  float* wV = wK + nsr * hdp;              // [nsr][hd+1] raw window values
-  float* csn = wV + nsr * hdp;             // [nsr][half+1] cos
-  float* snn = csn + nsr * (half + 1);     // [nsr][half+1] sin
-  float* srs = snn + nsr * (half + 1);     // [nsr][gq] scores, then weights
-  float* ml = srs + nsr * gq;              // [slots][16] partial m, l
-  float* sc = ml + kMaxSlots * 16;         // [slots][8] slot factors
-  float* Mg = sc + kMaxSlots * kMaxGQ;     // [8]
-  float* Lg = Mg + kMaxGQ;                 // [8]
+  // bf16 rows with 8-column groups: U stored as [g][e][v] for column 8v + e
+  const bool vec = sizeof(T) == 2 && rV % 8 == 0;
+  const int nv = rV / 8;
+  float* Us = reinterpret_cast<float*>(smf4);   // [gq][rV] (permuted when vec)
+  float* ml = Us + gq * rV;                     // [slots][16] partial m, l
+  float* sc = ml + kMaxSlots * 16;              // [slots][8] slot factors
+  float* wml = sc + kMaxSlots * kMaxGQ;         // [16] window m, l
+  float* Lg = wml + 16;                         // [8] 1 / L_g
+  float* fw = Lg + kMaxGQ;                      // [8] window factors
+  const float* wslot = win + static_cast<int64_t>(u) * (16 + gq * hd);
   const int fc = cta_of_tile(u * tpu, args.n_tiles, args.ctas);
   const int lc = cta_of_tile((u + 1) * tpu - 1, args.n_tiles, args.ctas);
   const int nslots = lc - fc + 1;
@@ -941,106 +1098,34 @@ __global__ void __launch_bounds__(kCombineThreads) sr_combine_kernel(const T* __
     const int uf = tile_begin(c, args.n_tiles, args.ctas) / tpu;
     return args.part + (static_cast<int64_t>(c) * args.max_units + (u - uf)) * args.slot_floats;
   };
-  // ---- A: loads and the window RoPE angles
-  const float qscale = rsqrtf(static_cast<float>(hd)) * kLog2e;
-  for (int i = tid; i < gq * hd; i += blockDim.x)
-    qs[i] = to_f(q[(static_cast<int64_t>(b) * args.Hq + h * gq) * hd + i]) * qscale;
-  if (sizeof(T) == 2 && hd % 8 == 0) {
-    // 16-byte vectors; every load of a thread is issued before any is used
-    const int vpr = hd / 8;  // vectors per row
-    constexpr int kV = 8;
-    for (int v0 = tid; v0 < 2 * nsr * vpr; v0 += kV * blockDim.x) {
-      uint4 w[kV];
-#pragma unroll
-      for (int t = 0; t < kV; ++t) {
-        const int v = v0 + t * blockDim.x;
-        if (v < 2 * nsr * vpr) {
-          const int mat = v / (nsr * vpr), r = (v / vpr) % nsr, c8 = v % vpr;
-          const T* src = (mat ? srV : srK) + (static_cast<int64_t>(b) * nsr + r) * d + h * hd + c8 * 8;
-          w[t] = *reinterpret_cast<const uint4*>(src);
-        }
-      }
-#pragma unroll
-      for (int t = 0; t < kV; ++t) {
-        const int v = v0 + t * blockDim.x;
-        if (v < 2 * nsr * vpr) {
-          const int mat = v / (nsr * vpr), r = (v / vpr) % nsr, c8 = v % vpr;
-          float* dst = (mat ? wV : wK) + r * hdp + c8 * 8;
-          const uint32_t ww[4] = {w[t].x, w[t].y, w[t].z, w[t].w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float2 f = bf2_to_f2(ww[e]);
-            dst[2 * e] = f.x;
-            dst[2 * e + 1] = f.y;
-          }
-        }
-      }
-    }
-  } else {
-    for (int i = tid; i < nsr * hd; i += blockDim.x) {
-      const int r = i / hd, jj = i % hd;
-      const int64_t off = (static_cast<int64_t>(b) * nsr + r) * d + h * hd + jj;
-      wK[r * hdp + jj] = to_f(srK[off]);
-      wV[r * hdp + jj] = to_f(srV[off]);
-    }
-  }
+  // ---- A
   for (int i = tid; i < nslots * 16; i += blockDim.x) ml[i] = slot_ptr(fc + i / 16)[i % 16];
-  for (int j = tid; j < half; j += blockDim.x) ftab[j] = args.ft[j];
+  if (tid < 16) wml[tid] = wslot[tid];
   __syncthreads();
-  for (int i = tid; i < nsr * half; i += blockDim.x) {
-    const int r = i / half, jj = i % half;
-    const int64_t t = r < args.sink ? r : args.T - args.recent + (r - args.sink);
-    float c, sn;
-    rope_cs(ftab[jj], static_cast<double>(t), &c, &sn);
-    csn[r * (half + 1) + jj] = c;
-    snn[r * (half + 1) + jj] = sn;
-  }
-  __syncthreads();
-  // ---- B: window scores
-  for (int i = tid; i < nsr * gq; i += blockDim.x) {
-    const int r = i / gq, g = i % gq;
-    const float* kr = wK + r * hdp;
-    const float* cr = csn + r * (half + 1);
-    const float* sr = snn + r * (half + 1);
-    const float* qg = qs + g * hd;
-    float s0 = 0.f, s1 = 0.f;
-#pragma unroll 8
-    for (int jj = 0; jj < half; ++jj) {
-      const float x0 = kr[jj], x1 = kr[jj + half], c = cr[jj], sn = sr[jj];
-      s0 = fmaf(qg[jj], x0 * c - x1 * sn, s0);
-      s1 = fmaf(qg[jj + half], x1 * c + x0 * sn, s1);
+  // ---- C
+  for (int g = warp; g < gq; g += nwarps) {
+    float M = lane == 0 ? wml[g] : -INFINITY;
+    for (int i = lane; i < nslots; i += 32) M = fmaxf(M, ml[i * 16 + g]);
+    M = warp_max(M);
+    float L = 0.f;
+    for (int i = lane; i < nslots; i += 32) {
+      const float f = exp2f(ml[i * 16 + g] - M);
+      sc[i * kMaxGQ + g] = f;
+      L = fmaf(ml[i * 16 + 8 + g], f, L);
     }
-    srs[i] = s0 + s1;
-  }
-  __syncthreads();
-  // ---- C: global max and denominator per query head
-  if (warp == 0) {
-    for (int g = 0; g < gq; ++g) {
-      float M = -INFINITY;
-      for (int i = lane; i < nslots; i += 32) M = fmaxf(M, ml[i * 16 + g]);
-      for (int r = lane; r < nsr; r += 32) M = fmaxf(M, srs[r * gq + g]);
-      M = warp_max(M);
-      float L = 0.f;
-      for (int i = lane; i < nslots; i += 32) {
-        const float f = exp2f(ml[i * 16 + g] - M);
-        sc[i * kMaxGQ + g] = f;
-        L = fmaf(ml[i * 16 + 8 + g], f, L);
-      }
-      for (int r = lane; r < nsr; r += 32) {
-        const float w = exp2f(srs[r * gq + g] - M);
-        srs[r * gq + g] = w;
-        L += w;
-      }
-      L = warp_sum(L);
-      if (lane == 0) { Mg[g] = M; Lg[g] = L; }
+    L = warp_sum(L);
+    if (lane == 0) {
+      const float f = exp2f(wml[g] - M);
+      fw[g] = f;
+      Lg[g] = 1.f / fmaf(wml[8 + g], f, L);
     }
   }
   __syncthreads();
-  // ---- D: value-basis sums over the slots (float4, 8 slots' loads in flight)
+  // ---- D (float4 over rank columns, 8 slots' loads in flight)
   {
-    const int n4 = gq * args.rV / 4;
+    const int n4 = gq * rV / 4;
     for (int i4 = tid; i4 < n4; i4 += blockDim.x) {
-      const int g = (4 * i4) / args.rV;
+      const int g = (4 * i4) / rV;
       float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
       for (int c0 = 0; c0 < nslots; c0 += 8) {
         float4 v[8];
@@ -1059,68 +1144,87 @@ __global__ void __launch_bounds__(kCombineThreads) sr_combine_kernel(const T* __
           }
         }
       }
-      reinterpret_cast<float4*>(Us)[i4] = acc;
+      if (vec) {
+        const int c = 4 * i4 - g * rV, vv = c >> 3, e = c & 7;
+        float* dst = Us + (g * 8 + e) * nv + vv;
+        dst[0] = acc.x;
+        dst[nv] = acc.y;
+        dst[2 * nv] = acc.z;
+        dst[3 * nv] = acc.w;
+      } else {
+        reinterpret_cast<float4*>(Us)[i4] = acc;
+      }
     }
   }
   __syncthreads();
-  // ---- E: output columns of this split
-  const bool vec = sizeof(T) == 2 && args.rV % 256 == 0 && args.rV <= 512;
-  for (int j = j0 + warp; j < j1; j += nwarps) {
-    const T* br = BtV + b * args.sbv + static_cast<int64_t>(h * hd + j) * args.rV;
-    float acc[kMaxGQ];
+  // ---- E
+  for (int jb = j0 + warp * kCombineColsPerWarp; jb < j1; jb += nwarps * kCombineColsPerWarp) {
+    const int ncol = min(kCombineColsPerWarp, j1 - jb);
+    float acc[kCombineColsPerWarp][kMaxGQ];
 #pragma unroll
-    for (int g = 0; g < kMaxGQ; ++g) acc[g] = 0.f;
+    for (int cc = 0; cc < kCombineColsPerWarp; ++cc)
+#pragma unroll
+      for (int g = 0; g < kMaxGQ; ++g) acc[cc][g] = 0.f;
     if (vec) {
-      // lane owns 8 consecutive rank columns in each 256-column half
-      const int nh = args.rV / 256;
-      uint4 w[2];
+      for (int v0 = 0; v0 < nv; v0 += 32) {
+        const int v = v0 + lane;
+        uint4 w[kCombineColsPerWarp];
 #pragma unroll
-      for (int t = 0; t < 2; ++t)
-        w[t] = t < nh ? *reinterpret_cast<const uint4*>(br + 256 * t + 8 * lane) : make_uint4(0, 0, 0, 0);
+        for (int cc = 0; cc < kCombineColsPerWarp; ++cc) {
+          const T* br = BtV + b * args.sbv + static_cast<int64_t>(h * hd + jb + cc) * rV;
+          w[cc] = cc < ncol && v < nv ? *reinterpret_cast<const uint4*>(br + 8 * v) : make_uint4(0, 0, 0, 0);
+        }
+        if (v < nv) {
 #pragma unroll
-      for (int t = 0; t < 2; ++t) {
-        if (t < nh) {
-          const uint32_t ww[4] = {w[t].x, w[t].y, w[t].z, w[t].w};
-          const int c0 = 256 * t + 8 * lane;
+          for (int e2 = 0; e2 < 4; ++e2) {
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float2 f = bf2_to_f2(ww[e]);
-#pragma unroll
-            for (int g = 0; g < kMaxGQ; ++g)
+            for (int g = 0; g < kMaxGQ; ++g) {
               if (g < gq) {
-                acc[g] = fmaf(Us[g * args.rV + c0 + 2 * e], f.x, acc[g]);
-                acc[g] = fmaf(Us[g * args.rV + c0 + 2 * e + 1], f.y, acc[g]);
+                const float u0 = Us[(g * 8 + 2 * e2) * nv + v], u1 = Us[(g * 8 + 2 * e2 + 1) * nv + v];
+#pragma unroll
+                for (int cc = 0; cc < kCombineColsPerWarp; ++cc) {
+                  const uint32_t word = e2 == 0 ? w[cc].x : e2 == 1 ? w[cc].y : e2 == 2 ? w[cc].z : w[cc].w;
+                  const float2 f = bf2_to_f2(word);
+                  acc[cc][g] = fmaf(u0, f.x, fmaf(u1, f.y, acc[cc][g]));
+                }
               }
+            }
           }
         }
       }
     } else {
-      for (int c = lane; c < args.rV; c += 32) {
-        const float bv = to_f(br[c]);
+      for (int c = lane; c < rV; c += 32) {
+        float bv[kCombineColsPerWarp];
+#pragma unroll
+        for (int cc = 0; cc < kCombineColsPerWarp; ++cc)
+          bv[cc] = cc < ncol ? to_f(BtV[b * args.sbv + static_cast<int64_t>(h * hd + jb + cc) * rV + c]) : 0.f;
 #pragma unroll
         for (int g = 0; g < kMaxGQ; ++g)
-          if (g < gq) acc[g] = fmaf(Us[g * args.rV + c], bv, acc[g]);
+          if (g < gq) {
+            const float uu = Us[g * rV + c];
+#pragma unroll
+            for (int cc = 0; cc < kCombineColsPerWarp; ++cc) acc[cc][g] = fmaf(uu, bv[cc], acc[cc][g]);
+          }
       }
     }
-    for (int r = lane; r < nsr; r += 32) {
-      const float v = wV[r * hdp + j];
 #pragma unroll
-      for (int g = 0; g < kMaxGQ; ++g)
-        if (g < gq) acc[g] = fmaf(srs[r * gq + g], v, acc[g]);
-    }
+    for (int cc = 0; cc < kCombineColsPerWarp; ++cc) {
 #pragma unroll
-    for (int g = 0; g < kMaxGQ; ++g) {
-      if (g >= gq) break;
-      const float v = warp_sum(acc[g]);
-      if (lane == 0) out[(static_cast<int64_t>(b) * args.Hq + h * gq + g) * hd + j] = v / Lg[g];
+      for (int g = 0; g < kMaxGQ; ++g) {
+        if (g >= gq) break;
+        const float v = warp_sum(acc[cc][g]);
+        if (lane == 0 && cc < ncol) {
+          const int j = jb + cc;
+          out[(static_cast<int64_t>(b) * args.Hq + h * gq + g) * hd + j] =
+              fmaf(fw[g], wslot[16 + g * hd + j], v) * Lg[g];
+        }
+      }
     }
   }
 }
 
-size_t combine_smem(int gq, int rV, int hd, int nsr) {
-  return (static_cast<size_t>(gq) * rV + static_cast<size_t>(gq) * hd + 2 * static_cast<size_t>(nsr) * (hd + 1) +
-          2 * static_cast<size_t>(nsr) * (hd / 2 + 1) + static_cast<size_t>(nsr) * gq + kMaxSlots * 16 +
-          kMaxSlots * kMaxGQ + 2 * kMaxGQ + 8) * 4 + 128 * 8 + 32;
+size_t combine_smem(int gq, int rV) {
+  return (static_cast<size_t>(gq) * rV + kMaxSlots * 16 + kMaxSlots * kMaxGQ + 16 + 2 * kMaxGQ) * 4 + 16;
 }
 
 size_t simt_smem(int gq, int rV, int hd) {
@@ -1129,7 +1233,7 @@ size_t simt_smem(int gq, int rV, int hd) {
 
 bool tc_shape_ok(const xkv_sr_params* p) {
   const int gq = p->n_q_heads / p->n_kv_heads;
-  return p->dtype == XKV_BF16 && p->head_dim == 128 && p->chunk == 8 && p->rank_k % (64 * kKAtoms) == 0 &&
+  return p->dtype == XKV_BF16 && p->head_dim == 128 && p->chunk == 8 && p->rank_k % 64 == 0 &&
          p->rank_v % 64 == 0 && p->rank_k <= 2048 && p->rank_v <= 512 && gq <= kMaxGQ &&
          p->a_k_batch_stride % 8 == 0 && p->a_v_batch_stride % 8 == 0 && p->bt_k_batch_stride % 8 == 0 &&
          !force_simt();
@@ -1154,12 +1258,14 @@ xkv_status sr_plan(const xkv_sr_params* p, SRPlan* plan) {
   plan->max_units_per_cta = mx;
   plan->slot_floats = 16 + static_cast<size_t>(std::max(gq, 1)) * p->rank_v;
   size_t off = 0;
-  plan->off_scores = off;
-  off = align_up(off + static_cast<size_t>(plan->units) * n_mid * 4);
+  plan->off_scores = off;  // rows padded to a multiple of 4 floats
+  off = align_up(off + static_cast<size_t>(plan->units) * ((n_mid + 3) & ~int64_t(3)) * 4);
   plan->off_sel = off;
   off = align_up(off + static_cast<size_t>(plan->units) * p->topk * 4);
   plan->off_part = off;
   off = align_up(off + static_cast<size_t>(plan->ctas) * mx * plan->slot_floats * 4);
+  plan->off_win = off;
+  off = align_up(off + static_cast<size_t>(plan->units) * (16 + static_cast<size_t>(gq) * p->head_dim) * 4);
   plan->bytes = off;
   return XKV_OK;
 }
@@ -1175,20 +1281,38 @@ static xkv_status sr_launch_t(const xkv_sr_params* p, const SRPlan& plan, const 
   float* scores = reinterpret_cast<float*>(w + plan.off_scores);
   int32_t* sel = reinterpret_cast<int32_t*>(w + plan.off_sel);
   float* part = reinterpret_cast<float*>(w + plan.off_part);
+  float* win = reinterpret_cast<float*>(w + plan.off_win);
   // 1. chunk scores
   {
     const int cpb = 512;
     dim3 grid(static_cast<unsigned>((n_mid + cpb - 1) / cpb), static_cast<unsigned>(plan.units));
     sr_score_kernel<T><<<grid, 256, 0, st>>>(static_cast<const T*>(q), static_cast<const T*>(lm), scores,
                                              p->n_q_heads, p->n_kv_heads, p->head_dim, n_mid, cpb);
+    if (cudaPeekAtLastError() != cudaSuccess) return XKV_ERR_CUDA;
   }
-  // 2. exact top-k
+  // 2. exact top-k (blocks [0, units)) and the raw window partials (blocks [units, 2 units))
   {
+    WinArgs wa;
+    wa.q = q;
+    wa.srK = sr_K;
+    wa.srV = sr_V;
+    wa.win = win;
+    wa.T = p->T;
+    wa.Hq = p->n_q_heads;
+    wa.Hkv = p->n_kv_heads;
+    wa.hd = p->head_dim;
+    wa.sink = p->sink;
+    wa.recent = p->recent;
+    for (int j = 0; j < 128; ++j) wa.ft[j] = j < p->head_dim / 2 ? rope_turns(p->rope_theta, j, p->head_dim) : 0.0;
+    const int nsr = p->sink + p->recent;
     const int64_t per = (n_mid + kTopkThreads - 1) / kTopkThreads;
-    const size_t smem = static_cast<size_t>(per * kTopkThreads + n_mid) * 4;
-    if (smem > 48 * 1024)
-      cudaFuncSetAttribute(sr_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-    sr_topk_kernel<<<plan.units, kTopkThreads, smem, st>>>(scores, sel, sel_out, n_mid, p->topk);
+    const size_t smem = std::max(static_cast<size_t>(per * kTopkThreads + n_mid) * 4 + static_cast<size_t>(n_mid) + 16,
+                                 window_smem(gq, p->head_dim, nsr));
+    // the opt-in covers static + dynamic shared memory above 48 KiB
+    cudaFuncSetAttribute(sr_topk_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    sr_topk_kernel<T><<<2 * plan.units, kTopkThreads, smem, st>>>(scores, (n_mid + 3) & ~int64_t(3), sel, sel_out, n_mid,
+                                                                   p->topk, plan.units, wa);
+    if (cudaPeekAtLastError() != cudaSuccess) return XKV_ERR_CUDA;
   }
   AttendArgs a;
   a.sel = sel;
@@ -1260,23 +1384,20 @@ static xkv_status sr_launch_t(const xkv_sr_params* p, const SRPlan& plan, const 
     kern<<<plan.ctas, kAttendThreads, smem, st>>>(mAK, mBK, mAV, a);
   } else {
     const size_t smem = simt_smem(gq, p->rank_v, p->head_dim);
-    if (smem > 48 * 1024)
-      cudaFuncSetAttribute(sr_attend_simt_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(smem));
+    cudaFuncSetAttribute(sr_attend_simt_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         static_cast<int>(smem));
     sr_attend_simt_kernel<T><<<plan.ctas, 256, smem, st>>>(
         static_cast<const T*>(q), static_cast<const T*>(A_K), static_cast<const T*>(Bt_K),
         static_cast<const T*>(A_V), a, p->head_dim, p->chunk, p->a_k_batch_stride, p->a_v_batch_stride);
   }
+  if (cudaPeekAtLastError() != cudaSuccess) return XKV_ERR_CUDA;
   // 4. combine
   {
-    const size_t smem = combine_smem(gq, p->rank_v, p->head_dim, p->sink + p->recent);
-    if (smem > 48 * 1024)
-      cudaFuncSetAttribute(sr_combine_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(smem));
+    const size_t smem = combine_smem(gq, p->rank_v);
+    cudaFuncSetAttribute(sr_combine_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         static_cast<int>(smem));
     sr_combine_kernel<T><<<dim3(plan.units, kCombineSplit), kCombineThreads, smem, st>>>(
-        static_cast<const T*>(q), static_cast<const T*>(Bt_V),
-                                                         static_cast<const T*>(sr_K), static_cast<const T*>(sr_V),
-                                                         a, p->head_dim, out);
+        static_cast<const T*>(Bt_V), win, a, p->head_dim, out);
   }
   return cudaPeekAtLastError() == cudaSuccess ? XKV_OK : XKV_ERR_CUDA;
 }

@@ -174,12 +174,10 @@ void cholqr_pass(const float* Y, float* Q, int n, int b, double shift_rel, doubl
   gemm_simt<float, float, double, double>(Y, 1, b, Y, b, 1, W, b, b, b, n, 1.0, 0.0, st);
   if (shift_rel > 0.0) trace_kernel<<<1, 256, 0, st>>>(W, b, scal);
   const size_t smem = static_cast<size_t>(b) * 8;
-  if (smem > 48 * 1024)
-    cudaFuncSetAttribute(cholesky_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  cudaFuncSetAttribute(cholesky_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   cholesky_kernel<<<1, 1024, smem, st>>>(W, b, shift_rel, shift_rel > 0.0 ? scal : nullptr, status);
   const size_t smem2 = static_cast<size_t>(8) * b * 8;
-  if (smem2 > 48 * 1024)
-    cudaFuncSetAttribute(tri_inverse_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem2));
+  cudaFuncSetAttribute(tri_inverse_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem2));
   tri_inverse_kernel<<<(b + 7) / 8, 256, smem2, st>>>(W, Linv, b);
   // Q(m, j) = sum_k Y(m, k) Linv(j, k)
   gemm_simt<float, double, float, double>(Y, b, 1, Linv, 1, b, Q, b, n, b, b, 1.0, 0.0, st);

@@ -299,8 +299,7 @@ static xkv_status dense_launch_t(const xkv_dense_params* p, const void* q, const
   const int units = p->batch * p->n_kv_heads;
   const size_t smem = (static_cast<size_t>(gq) * hd + 256 * gq + 8 * kMaxGQ + 3 * kMaxGQ +
                        static_cast<size_t>(256 / (hd / 2)) * gq * hd) * 4;
-  if (smem > 48 * 1024)
-    cudaFuncSetAttribute(dense_partial_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  cudaFuncSetAttribute(dense_partial_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   dense_partial_kernel<T><<<dim3(splits, units), 256, smem, st>>>(static_cast<const T*>(q), static_cast<const T*>(K),
                                                                   static_cast<const T*>(V), p->T, p->n_q_heads,
                                                                   p->n_kv_heads, hd, per, static_cast<float*>(ws));

@@ -30,7 +30,7 @@ struct SRPlan {
   int ctas;         // attention CTAs (persistent ranges of tiles)
   int max_units_per_cta;
   bool tc;          // tcgen05 path
-  size_t off_scores, off_sel, off_part, slot_floats, bytes;
+  size_t off_scores, off_sel, off_part, off_win, slot_floats, bytes;
 };
 xkv_status sr_plan(const xkv_sr_params* p, SRPlan* plan);
 xkv_status sr_launch(const xkv_sr_params* p, const SRPlan& plan, const void* q, const void* A_K,

@@ -5,7 +5,8 @@ Selection: the GPU's top-k set must equal the exact one except chunks whose
 score lies within 1e-3 (relative) of the k-th score.  Output: max-abs error
 <= 1e-2 against the oracle run on the GPU's own (valid) selection; the f32
 path is held to 2e-4.  Shapes cover the tiny f32 workload, small bf16 cases on
-the tensor-core path (ragged last tile, GQA group of 7, every chunk kept) and,
+the tensor-core path (ragged last tile, GQA group of 7, odd atom counts,
+every chunk kept) and,
 at full size, one layer launch of the Llama-3.1-8B group (16K), the 32-layer
 Llama-3.1-8B shape (64K, batch 4, sampled units) and the Qwen2.5-7B shape
 (128K, batch 2).
@@ -53,6 +54,47 @@ def test_sr_bf16_tensor_core_ragged_tile(xkv):
 def test_sr_bf16_gqa7_single_tile(xkv):
     w = synth.Workload("sr_bf16_gq7", 1, 4, 4, 2, 128, 14, 8 + 32 + 8 * 100, 96, 1.0, 64, 128, topk=16)
     _parity(xkv, w)
+
+
+def test_sr_bf16_odd_key_atom_count(xkv):
+    # key rank 192 = three 64-column atoms: the last key stage is half empty;
+    # value rank 320 leaves the last 128-column value block half empty
+    w = synth.Workload("sr_bf16_odd_atoms", 1, 4, 4, 2, 128, 8, 8 + 32 + 8 * 120, 96, 0.8, 192, 320, topk=33)
+    _parity(xkv, w)
+
+
+@pytest.mark.parametrize("n_tied", [800, 2000])
+def test_sr_topk_tied_boundary_bucket(xkv, n_tied):
+    # landmarks l_c = a_c u with u = sign(qbar) / 16 and a_c in {2, 1, 1/2}
+    # (all bf16-exact), so the scores take three exact values.  300 chunks
+    # score highest, n_tied share the boundary score and the rest score lower;
+    # with k = 600 the selection is the 300 high chunks plus the 300 tied
+    # chunks of lowest index (ties go to the lower index).  800 tied chunks
+    # are ranked by counting, 2000 by the radix passes.
+    n_mid = 3000
+    w = synth.Workload("sr_topk_ties", 1, 4, 4, 2, 128, 8, 8 + 32 + 8 * n_mid, 96, 0.8, 64, 64, topk=600)
+    inp = synth.compressed_cache(w, 0)
+    rng = np.random.default_rng(5)
+    q = inp["q"].reshape(1, w.n_kv_heads, w.gq, w.head_dim)
+    lm = np.empty_like(inp["landmarks"])
+    expect = []
+    for h in range(w.n_kv_heads):
+        qbar = q[0, h].astype(np.float64).sum(axis=0)
+        u = np.where(qbar >= 0, 1.0, -1.0) / 16.0
+        perm = rng.permutation(n_mid)
+        high, tied = np.sort(perm[:300]), np.sort(perm[300:300 + n_tied])
+        a = np.full(n_mid, 0.5)
+        a[high] = 2.0
+        a[tied] = 1.0
+        lm[0, h] = (a[:, None] * u[None, :]).astype(np.float32)
+        expect.append(np.sort(np.concatenate([high, tied[:300]])))
+    inp["landmarks"] = lm
+    out_g, sel_g = run_sr(xkv, w, sr_inputs_on_device(w, inp))
+    sel_g = sel_g.cpu().numpy()
+    for h in range(w.n_kv_heads):
+        assert np.array_equal(sel_g[0, h], expect[h])
+    ref, _, _ = oracle.sr_decode(w, sel_in=sel_g, **inp)
+    assert np.abs(host(out_g) - ref).max() <= 1e-2
 
 
 def test_sr_f32_general_shape(xkv):
