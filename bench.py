@@ -21,6 +21,7 @@ ranks of the device-timed region.
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import math
 import os
@@ -56,6 +57,14 @@ def sr_bytes_per_unit(w) -> int:
             + (w.rank_k + w.rank_v) * w.head_dim * el                # Bt slices
             + (w.sink + w.recent) * w.head_dim * 2 * el              # raw sink/recent K and V
             + 2 * w.gq * w.head_dim * el)                            # queries in, outputs out
+
+
+def attend_bytes_per_unit(w) -> int:
+    """Algorithmic HBM bytes of the attend stage for one unit: the selected
+    A_K and A_V chunk rows, the head's Bt_K slice and the group's queries."""
+    el = 2 if w.dtype == "bf16" else 4
+    return (w.topk * w.chunk * (w.rank_k + w.rank_v) * el + w.rank_k * w.head_dim * el
+            + w.gq * w.head_dim * el)
 
 
 def sr_flops_per_unit(w) -> int:
@@ -261,7 +270,9 @@ def run_cuda(args, rank, world, log):
             e1.record(stream)
             e1.synchronize()
         ms_total = e0.elapsed_time(e1)
-        # per-call timing of the dominant call (one layer of SR decode), live
+        if world > 1:
+            dist.barrier()
+        # per-call timing of one layer of SR decode (graph of one call), live
         with torch.cuda.stream(stream):
             ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(20)]
             for a, b_ in ev:
@@ -270,7 +281,18 @@ def run_cuda(args, rank, world, log):
                 b_.record(stream)
             torch.cuda.synchronize()
         call_ms = statistics.median(a.elapsed_time(b_) for a, b_ in ev)
-        # end to end: per step, pinned-host queries in, outputs out, around the same graph
+        # per-launch durations of the four stages (CUDA events recorded by the
+        # library on the launching stream), layers in turn so caches are cold
+        xkv.xkv_sr_profile_enable(True)
+        stages = []
+        with torch.cuda.stream(stream):
+            for i in range(2 * L):
+                layer_call(i % L, stream)
+                stages.append(xkv.xkv_sr_profile_read())
+        xkv.xkv_sr_profile_enable(False)
+        stage_ms = [statistics.median(s_[j] for s_ in stages) for j in range(4)]
+        # end to end through the C ABI: per step, pinned-host queries in, one
+        # library call per layer, outputs back to pinned host memory
         q_host = [model["q"][l].cpu().pin_memory() for l in range(L)]
         o_host = [torch.empty_like(outs[l], device="cpu").pin_memory() for l in range(L)]
         with torch.cuda.stream(stream):
@@ -280,7 +302,8 @@ def run_cuda(args, rank, world, log):
             for _ in range(args.steps):
                 for l in range(L):
                     model["q"][l].copy_(q_host[l], non_blocking=True)
-                graph.replay()
+                for l in range(L):
+                    layer_call(l, stream)
                 for l in range(L):
                     o_host[l].copy_(outs[l], non_blocking=True)
             e3.record(stream)
@@ -302,11 +325,19 @@ def run_cuda(args, rank, world, log):
     achieved_step = bytes_step / (ms_step / 1e3) / 1e9
     bytes_call = sr_bytes_per_unit(w) * w.batch * w.n_kv_heads
     achieved_call = bytes_call / (call_ms / 1e3) / 1e9
+    # dominant kernel: selective reconstruction + attention (sr_attend)
+    bytes_attend = attend_bytes_per_unit(w) * w.batch * w.n_kv_heads
+    achieved_attend = bytes_attend / (stage_ms[2] / 1e3) / 1e9
+    # DRAM traffic per launch from the committed ncu summary, valid only while
+    # the kernel source is the one that was profiled
     traffic = None
     tp = os.path.join(ROOT, "profiles", "traffic.json")
     if os.path.exists(tp):
         try:
-            traffic = json.load(open(tp)).get(args.workload)
+            ent = json.load(open(tp)).get(args.workload)
+            src = open(os.path.join(ROOT, ent["source"]), "rb").read()
+            if ent and hashlib.sha1(src).hexdigest() == ent["source_sha1"]:
+                traffic = ent["bytes_per_launch"]
         except Exception:
             traffic = None
     q_bytes = sum(t.numel() * t.element_size() for t in model["q"])
@@ -322,11 +353,15 @@ def run_cuda(args, rank, world, log):
                    "l2": "inputs larger than L2 (%.1f GB touched per step)" % (bytes_step / 1e9)},
         "hbm_gbs": round(achieved_step, 1),
         "hbm_frac_of_peak": round(achieved_step / hbm_gbs_peak, 4),
-        "roofline": {"bound": "hbm", "kernel": "xkv_sr_attention_decode (one layer: score, top-k, attend, combine)",
-                     "achieved": round(achieved_call, 1), "peak": hbm_gbs_peak, "unit": "GB/s",
-                     "frac": round(achieved_call / hbm_gbs_peak, 4), "traffic": traffic,
-                     "peak_source": f"{peak_kind} hbm_gbs", "bytes_per_launch": bytes_call,
-                     "launch_ms": round(call_ms, 5)},
+        "roofline": {"bound": "hbm", "kernel": "sr_attend_tc (selective reconstruction + attention partials)",
+                     "achieved": round(achieved_attend, 1), "peak": hbm_gbs_peak, "unit": "GB/s",
+                     "frac": round(achieved_attend / hbm_gbs_peak, 4), "traffic": traffic,
+                     "peak_source": f"{peak_kind} hbm_gbs (burst copy)", "bytes_per_launch": bytes_attend,
+                     "launch_ms": round(stage_ms[2], 5)},
+        "stages_ms": {"score": round(stage_ms[0], 5), "topk_window": round(stage_ms[1], 5),
+                      "attend": round(stage_ms[2], 5), "combine": round(stage_ms[3], 5)},
+        "layer_call": {"ms": round(call_ms, 5), "bytes": bytes_call, "achieved_gbs": round(achieved_call, 1),
+                       "frac": round(achieved_call / hbm_gbs_peak, 4)},
         "e2e": {"value": round(tokens / (e2e_ms / args.steps / 1e3), 2), "unit": "tokens/s",
                 "h2d_bytes_per_step": q_bytes, "d2h_bytes_per_step": o_bytes},
         "gpu_launches": 4 * L * args.steps,

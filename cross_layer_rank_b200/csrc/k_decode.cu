@@ -1270,6 +1270,22 @@ xkv_status sr_plan(const xkv_sr_params* p, SRPlan* plan) {
   return XKV_OK;
 }
 
+// stage-timing events (see xkv_sr_profile_enable)
+struct SRProfile {
+  bool on = false, recorded = false;
+  int device = -1;
+  cudaEvent_t ev[5] = {};
+};
+SRProfile g_prof;
+
+inline void prof_mark(int i, cudaStream_t st) {
+  int dev = -1;
+  if (g_prof.on && cudaGetDevice(&dev) == cudaSuccess && dev == g_prof.device) {
+    cudaEventRecord(g_prof.ev[i], st);
+    if (i == 4) g_prof.recorded = true;
+  }
+}
+
 template <typename T>
 static xkv_status sr_launch_t(const xkv_sr_params* p, const SRPlan& plan, const void* q, const void* A_K,
                               const void* Bt_K, const void* A_V, const void* Bt_V, const void* lm,
@@ -1282,6 +1298,7 @@ static xkv_status sr_launch_t(const xkv_sr_params* p, const SRPlan& plan, const 
   int32_t* sel = reinterpret_cast<int32_t*>(w + plan.off_sel);
   float* part = reinterpret_cast<float*>(w + plan.off_part);
   float* win = reinterpret_cast<float*>(w + plan.off_win);
+  prof_mark(0, st);
   // 1. chunk scores
   {
     const int cpb = 512;
@@ -1290,6 +1307,7 @@ static xkv_status sr_launch_t(const xkv_sr_params* p, const SRPlan& plan, const 
                                              p->n_q_heads, p->n_kv_heads, p->head_dim, n_mid, cpb);
     if (cudaPeekAtLastError() != cudaSuccess) return XKV_ERR_CUDA;
   }
+  prof_mark(1, st);
   // 2. exact top-k (blocks [0, units)) and the raw window partials (blocks [units, 2 units))
   {
     WinArgs wa;
@@ -1314,6 +1332,7 @@ static xkv_status sr_launch_t(const xkv_sr_params* p, const SRPlan& plan, const 
                                                                    p->topk, plan.units, wa);
     if (cudaPeekAtLastError() != cudaSuccess) return XKV_ERR_CUDA;
   }
+  prof_mark(2, st);
   AttendArgs a;
   a.sel = sel;
   a.q = q;
@@ -1391,6 +1410,7 @@ static xkv_status sr_launch_t(const xkv_sr_params* p, const SRPlan& plan, const 
         static_cast<const T*>(A_V), a, p->head_dim, p->chunk, p->a_k_batch_stride, p->a_v_batch_stride);
   }
   if (cudaPeekAtLastError() != cudaSuccess) return XKV_ERR_CUDA;
+  prof_mark(3, st);
   // 4. combine
   {
     const size_t smem = combine_smem(gq, p->rank_v);
@@ -1399,7 +1419,37 @@ static xkv_status sr_launch_t(const xkv_sr_params* p, const SRPlan& plan, const 
     sr_combine_kernel<T><<<dim3(plan.units, kCombineSplit), kCombineThreads, smem, st>>>(
         static_cast<const T*>(Bt_V), win, a, p->head_dim, out);
   }
+  prof_mark(4, st);
   return cudaPeekAtLastError() == cudaSuccess ? XKV_OK : XKV_ERR_CUDA;
+}
+
+xkv_status sr_profile_enable(int enable) {
+  if (!enable) {
+    g_prof.on = false;
+    return XKV_OK;
+  }
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return XKV_ERR_CUDA;
+  if (g_prof.device != dev) {
+    for (cudaEvent_t& e : g_prof.ev) {
+      if (e) cudaEventDestroy(e);
+      e = nullptr;
+    }
+    for (cudaEvent_t& e : g_prof.ev)
+      if (cudaEventCreate(&e) != cudaSuccess) return XKV_ERR_CUDA;
+    g_prof.device = dev;
+  }
+  g_prof.recorded = false;
+  g_prof.on = true;
+  return XKV_OK;
+}
+
+xkv_status sr_profile_read(float* stage_ms) {
+  if (!stage_ms || !g_prof.recorded) return XKV_ERR_INVALID_ARG;
+  if (cudaEventSynchronize(g_prof.ev[4]) != cudaSuccess) return XKV_ERR_CUDA;
+  for (int i = 0; i < 4; ++i)
+    if (cudaEventElapsedTime(&stage_ms[i], g_prof.ev[i], g_prof.ev[i + 1]) != cudaSuccess) return XKV_ERR_CUDA;
+  return XKV_OK;
 }
 
 xkv_status sr_launch(const xkv_sr_params* p, const SRPlan& plan, const void* q, const void* A_K, const void* Bt_K,

@@ -222,12 +222,16 @@ static xkv_status check_sr(const xkv_sr_params* p) {
   if (p->dtype != XKV_F32 && p->dtype != XKV_BF16) return XKV_ERR_INVALID_ARG;
   if (!(p->rope_theta > 1.0f)) return XKV_ERR_INVALID_ARG;
   const int gq = p->n_q_heads / p->n_kv_heads;
-  if (gq > 8 || p->head_dim > 256 || p->sink + p->recent > 64 || n_mid * 8 > 200 * 1024 || p->rank_v > 4096 ||
+  if (gq > 8 || p->head_dim > 256 || p->sink + p->recent > 64 || n_mid > kMaxMidChunks || p->rank_v > 4096 ||
       p->topk > 1024)
     return XKV_ERR_UNSUPPORTED;
   if (p->T > (int64_t(1) << 30)) return XKV_ERR_UNSUPPORTED;
   return XKV_OK;
 }
+
+xkv_status xkv_sr_profile_enable(int enable) { return sr_profile_enable(enable); }
+
+xkv_status xkv_sr_profile_read(float* stage_ms) { return sr_profile_read(stage_ms); }
 
 xkv_status xkv_sr_workspace_size(const xkv_sr_params* p, size_t* bytes) {
   if (!bytes) return XKV_ERR_INVALID_ARG;

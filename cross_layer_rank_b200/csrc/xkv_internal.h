@@ -32,7 +32,12 @@ struct SRPlan {
   bool tc;          // tcgen05 path
   size_t off_scores, off_sel, off_part, off_win, slot_floats, bytes;
 };
+// top-k shared memory: 9 bytes per chunk (+ padding) must stay under the
+// 227 KiB opt-in with the kernel's static arrays
+constexpr int64_t kMaxMidChunks = 24576;
 xkv_status sr_plan(const xkv_sr_params* p, SRPlan* plan);
+xkv_status sr_profile_enable(int enable);
+xkv_status sr_profile_read(float* stage_ms);
 xkv_status sr_launch(const xkv_sr_params* p, const SRPlan& plan, const void* q, const void* A_K,
                      const void* Bt_K, const void* A_V, const void* Bt_V, const void* landmarks,
                      const void* sr_K, const void* sr_V, float* out, int32_t* sel_out, void* ws,

@@ -132,7 +132,8 @@ typedef struct xkv_sr_params {
   int64_t T;              /* cached tokens; the query sits at position T */
   int rank_k, rank_v;     /* columns of A_K, A_V */
   int chunk;              /* tokens per chunk */
-  int topk;               /* chunks kept per (batch, KV head), <= n_mid */
+  int topk;               /* chunks kept per (batch, KV head), <= n_mid and <= 1024;
+                             n_mid = (T - sink - recent) / chunk <= 24576 */
   int sink, recent;       /* raw windows [0, sink) and [T - recent, T) */
   float rope_theta;
   xkv_dtype dtype;        /* of q, A, Bt, landmarks, sink/recent */
@@ -160,6 +161,19 @@ XKV_API xkv_status xkv_sr_attention_decode(const xkv_sr_params* p, const void* q
                                    const void* landmarks, const void* sr_K, const void* sr_V,
                                    float* out, int32_t* sel_out, void* workspace, size_t ws_bytes,
                                    void* stream);
+
+/* Stage timing (measurement aid; the method has no counterpart).  While
+ * enabled, every xkv_sr_attention_decode call records CUDA events on its
+ * stream around its four launches: chunk scores, top-k (+ raw window
+ * partials), selective reconstruction + attention partials, combine.
+ * xkv_sr_profile_read waits for the most recent call's last event and writes
+ * the four durations in milliseconds to stage_ms[0..3].  The events belong to
+ * the device current at enable time; calls on another device are not timed.
+ * Not for use while a stream is being captured.  Process-wide state, not
+ * thread-safe.  Errors: XKV_ERR_CUDA (event creation or query failed),
+ * XKV_ERR_INVALID_ARG (stage_ms NULL, or nothing recorded yet). */
+XKV_API xkv_status xkv_sr_profile_enable(int enable);
+XKV_API xkv_status xkv_sr_profile_read(float* stage_ms);
 
 /* -------------------------------------------------- full reconstruction */
 /* The comparison path of [xKV-blog] Fig. 6: rebuild every row,
