@@ -37,6 +37,7 @@ EXPORTS = (
     "xkv_compress_workspace_size", "xkv_compress_group",
     "xkv_build_landmarks",
     "xkv_sr_workspace_size", "xkv_sr_attention_decode",
+    "xkv_sr_attention_decode_noalloc",
     "xkv_sr_profile_enable", "xkv_sr_profile_read",
     "xkv_full_reconstruct",
     "xkv_dense_workspace_size", "xkv_dense_attention_decode",
@@ -85,6 +86,8 @@ def _load():
         "xkv_sr_workspace_size": (C.c_int, [C.POINTER(SRParams), C.POINTER(sz)]),
         "xkv_sr_attention_decode": (C.c_int, [C.POINTER(SRParams), vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz,
                                               vp]),
+        "xkv_sr_attention_decode_noalloc": (C.c_int, [C.POINTER(SRParams), vp, vp, vp, vp, vp, vp, vp, vp, vp, vp,
+                                                      vp]),
         "xkv_sr_profile_enable": (C.c_int, [C.c_int]),
         "xkv_sr_profile_read": (C.c_int, [C.POINTER(C.c_float)]),
         "xkv_full_reconstruct": (C.c_int, [vp, vp, i64, C.c_int, C.c_int, C.c_int, C.c_int, C.c_int, C.c_float,
@@ -232,6 +235,18 @@ def xkv_sr_attention_decode(p: SRParams, q, A_K, Bt_K, A_V, Bt_V, landmarks, sr_
     _check(lib.xkv_sr_attention_decode(C.byref(p), _ptr(q), _ptr(A_K), _ptr(Bt_K), _ptr(A_V), _ptr(Bt_V),
                                        _ptr(landmarks), _ptr(sr_K), _ptr(sr_V), _ptr(out), _ptr(sel_out), _ptr(ws),
                                        ws.numel(), _stream(stream)), "xkv_sr_attention_decode")
+
+
+SR_STATIC_SCRATCH_BYTES = 8 << 20
+
+
+def xkv_sr_attention_decode_noalloc(p: SRParams, q, A_K, Bt_K, A_V, Bt_V, landmarks, sr_K, sr_V, out,
+                                    sel_out=None, stream=None):
+    """One SR decode step with the library's fixed scratch array (no workspace,
+    no allocation); calls that overlap in time race on that array."""
+    _check(lib.xkv_sr_attention_decode_noalloc(C.byref(p), _ptr(q), _ptr(A_K), _ptr(Bt_K), _ptr(A_V), _ptr(Bt_V),
+                                               _ptr(landmarks), _ptr(sr_K), _ptr(sr_V), _ptr(out), _ptr(sel_out),
+                                               _stream(stream)), "xkv_sr_attention_decode_noalloc")
 
 
 def xkv_sr_profile_enable(enable: bool = True) -> None:

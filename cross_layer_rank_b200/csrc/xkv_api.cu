@@ -15,6 +15,10 @@ namespace xkv {
 
 static __device__ int g_device_status;
 
+// Scratch of xkv_sr_attention_decode_noalloc: a fixed device array that is part
+// of the loaded module, so that entry point never allocates.
+static __device__ __align__(256) unsigned char g_sr_static_scratch[XKV_SR_STATIC_SCRATCH_BYTES];
+
 namespace {
 constexpr int kMaxDevices = 64;
 int* g_status_ptr[kMaxDevices] = {nullptr};
@@ -40,6 +44,22 @@ int* device_status_ptr() {
     g_status_ptr[dev] = static_cast<int*>(p);
   }
   return g_status_ptr[dev];
+}
+
+void* g_scratch_ptr[kMaxDevices] = {nullptr};
+
+// Device address of g_sr_static_scratch on the current device, looked up once
+// per device (with that device current) and cached.
+void* static_scratch_ptr() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_scratch_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_sr_static_scratch) != cudaSuccess) return nullptr;
+    g_scratch_ptr[dev] = p;
+  }
+  return g_scratch_ptr[dev];
 }
 
 int num_sms() {
@@ -258,6 +278,26 @@ xkv_status xkv_sr_attention_decode(const xkv_sr_params* p, const void* q, const 
   sr_plan(p, &plan);
   if (!workspace || ws_bytes < plan.bytes || !aligned256(workspace)) return XKV_ERR_WORKSPACE;
   return sr_launch(p, plan, q, A_K, Bt_K, A_V, Bt_V, landmarks, sr_K, sr_V, out, sel_out, workspace,
+                   static_cast<cudaStream_t>(stream));
+}
+
+xkv_status xkv_sr_attention_decode_noalloc(const xkv_sr_params* p, const void* q, const void* A_K,
+                                           const void* Bt_K, const void* A_V, const void* Bt_V, const void* landmarks,
+                                           const void* sr_K, const void* sr_V, float* out, int32_t* sel_out,
+                                           void* stream) {
+  xkv_status s = check_sr(p);
+  if (s != XKV_OK) return s;
+  const void* ptrs[] = {q, A_K, Bt_K, A_V, Bt_V, landmarks, out};
+  for (const void* x : ptrs)
+    if (!x || !aligned16(x)) return XKV_ERR_INVALID_ARG;
+  if (p->sink + p->recent > 0 && (!sr_K || !sr_V || !aligned16(sr_K) || !aligned16(sr_V))) return XKV_ERR_INVALID_ARG;
+  if (sel_out && !aligned16(sel_out)) return XKV_ERR_INVALID_ARG;
+  SRPlan plan;
+  sr_plan(p, &plan);
+  if (plan.bytes > static_cast<size_t>(XKV_SR_STATIC_SCRATCH_BYTES)) return XKV_ERR_UNSUPPORTED;
+  void* scratch = static_scratch_ptr();
+  if (!scratch) return XKV_ERR_CUDA;
+  return sr_launch(p, plan, q, A_K, Bt_K, A_V, Bt_V, landmarks, sr_K, sr_V, out, sel_out, scratch,
                    static_cast<cudaStream_t>(stream));
 }
 

@@ -162,6 +162,29 @@ XKV_API xkv_status xkv_sr_attention_decode(const xkv_sr_params* p, const void* q
                                    float* out, int32_t* sel_out, void* workspace, size_t ws_bytes,
                                    void* stream);
 
+/* The same decode step without a caller workspace (an interface convenience;
+ * the pages have no counterpart).  Its scratch is a fixed device array of
+ * XKV_SR_STATIC_SCRATCH_BYTES inside the loaded library, so the call performs
+ * no device allocation of any kind; it serves callers that cannot allocate or
+ * hold a workspace, e.g. a plain C host program without a device allocator of
+ * its own, or a decode loop that must run under a fixed memory budget.
+ *   - Requests whose scratch (xkv_sr_workspace_size) exceeds the array return
+ *     XKV_ERR_UNSUPPORTED and launch nothing.
+ *   - The array's device address is looked up once per device, on the first
+ *     call made with that device current; make that first call before any
+ *     stream capture that includes this entry point.
+ *   - Nothing in the scratch needs to start at zero: every word the kernels
+ *     read is written earlier in the same call.
+ *   - Every call on a device shares the one array: calls that overlap in time
+ *     (on different streams or from different host threads) race on it and
+ *     corrupt each other's results.  Order them, e.g. on one stream.
+ * Arguments, layouts and errors are otherwise those of xkv_sr_attention_decode. */
+#define XKV_SR_STATIC_SCRATCH_BYTES (8u << 20)
+XKV_API xkv_status xkv_sr_attention_decode_noalloc(const xkv_sr_params* p, const void* q, const void* A_K,
+                                           const void* Bt_K, const void* A_V, const void* Bt_V,
+                                           const void* landmarks, const void* sr_K, const void* sr_V,
+                                           float* out, int32_t* sel_out, void* stream);
+
 /* Stage timing (measurement aid; the method has no counterpart).  While
  * enabled, every xkv_sr_attention_decode call records CUDA events on its
  * stream around its four launches: chunk scores, top-k (+ raw window
