@@ -119,10 +119,10 @@ __global__ void emit_factors_kernel(const float* __restrict__ Vr, int n, int r, 
 // operands from the K-major transposed shard Xt.  The tensor cores accumulate
 // only kGramChunk rows into a TMEM buffer (two buffers, double-buffered); the
 // epilogue warps add each chunk's tile into fp32 registers with IEEE adds.
-// Keeping the in-MMA accumulation chain short (8 MMAs of 16 rows) removes the
+// Keeping the in-MMA accumulation chain short (16 MMAs of 16 rows) removes the
 // drift a long chain of tensor-core accumulations shows over thousands of
 // rows; the outer sum is an ordinary round-to-nearest fp32 chain.
-constexpr int kGramChunkStages = 2;  // 2 x 64 rows per TMEM chunk
+constexpr int kGramChunkStages = 4;  // 4 x 64 rows per TMEM chunk
 constexpr int kGramStages = 4;
 constexpr int kGramThreads = 192;
 
@@ -202,28 +202,49 @@ __global__ void __launch_bounds__(kGramThreads, 1)
       if (!mbar_wait(&accfull[buf], (c >> 1) & 1, status)) { ok = false; break; }
       tc_fence_after();
 #pragma unroll
-      for (int jb = 0; jb < 8; ++jb) {
-        float v[16];
+      for (int jb = 0; jb < 8; jb += 2) {
+        float v[32];
         tmem_ld16(tbase + buf * 128 + jb * 16, v);
+        tmem_ld16(tbase + buf * 128 + jb * 16 + 16, v + 16);
         tmem_ld_wait();
 #pragma unroll
-        for (int i = 0; i < 16; ++i) acc[jb * 16 + i] += v[i];
+        for (int i = 0; i < 32; ++i) acc[jb * 16 + i] += v[i];
       }
       tc_fence_before();
       mbar_arrive(&accempty[buf]);
     }
     if (ok) {
+      // read-modify-write of C in batches whose loads are all issued before
+      // any of their stores (C is read and written through one pointer, so a
+      // plain += loop would wait for every load in turn)
       const int m = m0 + row;
       float* crow = C + static_cast<int64_t>(m) * ldc + n0;
 #pragma unroll
-      for (int i = 0; i < 128; i += 4) {
-        float4 cv = *reinterpret_cast<float4*>(crow + i);
-        cv.x += acc[i]; cv.y += acc[i + 1]; cv.z += acc[i + 2]; cv.w += acc[i + 3];
-        *reinterpret_cast<float4*>(crow + i) = cv;
+      for (int i0 = 0; i0 < 128; i0 += 32) {
+        float4 cv[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) cv[u] = *reinterpret_cast<const float4*>(crow + i0 + 4 * u);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int i = i0 + 4 * u;
+          cv[u].x += acc[i];
+          cv[u].y += acc[i + 1];
+          cv[u].z += acc[i + 2];
+          cv[u].w += acc[i + 3];
+          *reinterpret_cast<float4*>(crow + i) = cv[u];
+        }
       }
       if (tm != tn) {
+        // the mirrored tile: lanes hold consecutive m, so each access is one
+        // 128-byte row segment per warp
 #pragma unroll
-        for (int i = 0; i < 128; ++i) C[static_cast<int64_t>(n0 + i) * ldc + m] += acc[i];
+        for (int i0 = 0; i0 < 128; i0 += 16) {
+          float v[16];
+#pragma unroll
+          for (int u = 0; u < 16; ++u) v[u] = C[static_cast<int64_t>(n0 + i0 + u) * ldc + m];
+#pragma unroll
+          for (int u = 0; u < 16; ++u) C[static_cast<int64_t>(n0 + i0 + u) * ldc + m] = v[u] + acc[i0 + u];
+        }
       }
     }
   }

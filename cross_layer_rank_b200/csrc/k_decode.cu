@@ -35,7 +35,7 @@ constexpr int kKAtoms = 2;
 constexpr int kBStages = 2;   // Bt_K atoms (128 rows x 64 columns)
 constexpr int kVStages = 4;   // value stages: 2 chunks x full rank
 constexpr int kAtomBytes = 16384;  // 128 rows x 64 bf16
-constexpr int kAttendThreads = 480;  // 15 warps: 8 key epilogue, 4 value epilogue, 2 TMA, 1 MMA
+constexpr int kAttendThreads = 512;  // 16 warps: 8 key epilogue, 4 value epilogue, 2 TMA, 2 MMA
 
 // ----------------------------------------------------------------- helpers
 __host__ __device__ inline int tile_begin(int c, int n_tiles, int ctas) {
@@ -168,6 +168,7 @@ __global__ void __launch_bounds__(256) sr_score_kernel(const T* __restrict__ q, 
 // segment loops are free of shared-memory bank conflicts.
 constexpr int kTopkThreads = 1024;
 constexpr int kBuckets = 1024;
+constexpr uint32_t kRefineMin = 64;  // boundary buckets above this size get a second histogram
 
 __device__ __forceinline__ uint32_t topk_bucket(uint32_t key, uint32_t lo, float scale) {
   const float x = static_cast<float>(key - lo) * scale;
@@ -351,26 +352,67 @@ __global__ void __launch_bounds__(kTopkThreads) sr_topk_kernel(const float* __re
   // 2. histogram
   for (int j = 0; j < cnt; ++j) atomicAdd(&hist[topk_bucket(ksm[j * nt + tid], lo, scale)], 1u);
   __syncthreads();
-  // 3. suffix scan: thread t owns bucket kBuckets - 1 - t
-  {
+  // 3. suffix scan: thread t owns bucket kBuckets - 1 - t; the bucket where
+  // the running count reaches kk, and how many keys it must still give
+  auto find_boundary = [&](uint32_t kk) {
     const uint32_t hv = hist[kBuckets - 1 - tid];
     const uint32_t excl = block_exclusive_scan(hv, warp_tot, &s_total);  // keys in higher buckets
-    if (excl < static_cast<uint32_t>(k) && excl + hv >= static_cast<uint32_t>(k)) {
+    if (excl < kk && excl + hv >= kk) {
       s_bucket = kBuckets - 1 - tid;
-      s_need = static_cast<uint32_t>(k) - excl;
+      s_need = kk - excl;
     }
+    __syncthreads();
+  };
+  find_boundary(static_cast<uint32_t>(k));
+  const uint32_t B = s_bucket, need1 = s_need;
+  const uint32_t m1 = hist[B];
+  // 4. a crowded boundary bucket is refined by a second histogram over its own
+  // key range (same monotone map), so few keys remain to be ranked one by one
+  const bool two = m1 > kRefineMin;
+  uint32_t lo2 = 0u, B2 = 0u, need = need1;
+  float scale2 = 0.f;
+  if (two) {
+    uint32_t bmin = 0xFFFFFFFFu, bmax = 0u;
+    for (int j = 0; j < cnt; ++j) {
+      const uint32_t key = ksm[j * nt + tid];
+      if (topk_bucket(key, lo, scale) == B) { bmin = min(bmin, key); bmax = max(bmax, key); }
+    }
+    bmin = __reduce_min_sync(0xffffffffu, bmin);
+    bmax = __reduce_max_sync(0xffffffffu, bmax);
+    __syncthreads();  // every thread has read hist[B]
+    hist[tid] = 0u;
+    if (tid == 0) { s_lo = 0xFFFFFFFFu; s_hi = 0u; }
+    __syncthreads();
+    if (lane == 0) { atomicMin(&s_lo, bmin); atomicMax(&s_hi, bmax); }
+    __syncthreads();
+    lo2 = s_lo;
+    scale2 = static_cast<float>(kBuckets) / (static_cast<float>(s_hi - lo2) + 1.0f);
+    for (int j = 0; j < cnt; ++j) {
+      const uint32_t key = ksm[j * nt + tid];
+      if (topk_bucket(key, lo, scale) == B) atomicAdd(&hist[topk_bucket(key, lo2, scale2)], 1u);
+    }
+    __syncthreads();
+    find_boundary(need1);
+    B2 = s_bucket;
+    need = s_need;
   }
-  __syncthreads();
-  const uint32_t B = s_bucket, need = s_need;
-  // 4. candidates of the boundary bucket (their keys, ascending index)
+  // key classes: 2 = kept outright, 1 = final candidate, 0 = dropped
+  auto klass = [&](uint32_t key) -> int {
+    const uint32_t b1 = topk_bucket(key, lo, scale);
+    if (b1 != B) return b1 > B ? 2 : 0;
+    if (!two) return 1;
+    const uint32_t b2 = topk_bucket(key, lo2, scale2);
+    return b2 > B2 ? 2 : (b2 == B2 ? 1 : 0);
+  };
+  // 5. final candidates (their keys, ascending index)
   uint32_t nc = 0;
-  for (int j = 0; j < cnt; ++j) nc += topk_bucket(ksm[j * nt + tid], lo, scale) == B;
+  for (int j = 0; j < cnt; ++j) nc += klass(ksm[j * nt + tid]) == 1;
   uint32_t cpos = block_exclusive_scan(nc, warp_tot, &s_total);
   const uint32_t m = s_total;
   const uint32_t cbase = cpos;
   for (int j = 0; j < cnt; ++j) {
     const uint32_t key = ksm[j * nt + tid];
-    if (topk_bucket(key, lo, scale) == B) ckey[cpos++] = key;
+    if (klass(key) == 1) ckey[cpos++] = key;
   }
   __syncthreads();
   if (m == need) {
@@ -449,15 +491,15 @@ __global__ void __launch_bounds__(kTopkThreads) sr_topk_kernel(const float* __re
   }
   __syncthreads();
   const bool all_taken = s_all != 0u;
-  // 5. ordered compaction of the selection: a key of B is kept when its
-  // candidate decision says so (candidates are numbered in index order)
+  // 6. ordered compaction of the selection: a final candidate is kept when
+  // its decision says so (candidates are numbered in index order)
   uint32_t n_sel = 0;
   {
     uint32_t ci = cbase;
     for (int j = 0; j < cnt; ++j) {
-      const uint32_t bk = topk_bucket(ksm[j * nt + tid], lo, scale);
-      if (bk == B) n_sel += all_taken || ckeep[ci++];
-      else n_sel += bk > B;
+      const int c = klass(ksm[j * nt + tid]);
+      if (c == 1) n_sel += all_taken || ckeep[ci++];
+      else n_sel += c == 2;
     }
   }
   uint32_t pos = block_exclusive_scan(n_sel, warp_tot, &s_total);
@@ -466,10 +508,10 @@ __global__ void __launch_bounds__(kTopkThreads) sr_topk_kernel(const float* __re
     int32_t* o = sel + static_cast<int64_t>(unit) * k;
     int32_t* o2 = sel_out ? sel_out + static_cast<int64_t>(unit) * k : nullptr;
     for (int j = 0; j < cnt; ++j) {
-      const uint32_t bk = topk_bucket(ksm[j * nt + tid], lo, scale);
+      const int c = klass(ksm[j * nt + tid]);
       bool take;
-      if (bk == B) take = all_taken || ckeep[ci++];
-      else take = bk > B;
+      if (c == 1) take = all_taken || ckeep[ci++];
+      else take = c == 2;
       if (take) {
         o[pos] = i0 + j;
         if (o2) o2[pos] = i0 + j;
@@ -540,7 +582,9 @@ constexpr int kVAccCol = 256;  // TMEM columns of the value accumulators (2 x 64
 
 // Warp roles: 0-7 key epilogue (warp w reads TMEM lane quarter w % 4 and the
 // frequency pairs of half w / 4), 8-11 value epilogue, 12 key TMA producer,
-// 13 value TMA producer, 14 MMA issuer (TMEM owner).
+// 13 value TMA producer, 14 key MMA issuer (TMEM owner), 15 value MMA issuer.
+// The two issuers run independently, so the key gathers of later tiles never
+// wait behind the value products of earlier ones.
 template <int GQ>
 __global__ void __launch_bounds__(kAttendThreads, 1)
     sr_attend_tc_kernel(const __grid_constant__ CUtensorMap mapAK, const __grid_constant__ CUtensorMap mapBK,
@@ -685,11 +729,10 @@ __global__ void __launch_bounds__(kAttendThreads, 1)
       }
     }
   } else if (warp == 14) {
-    // ------------------------------------------------------------ MMA issuer
+    // -------------------------------------------------------- key MMA issuer
     if (lane == 0) {
       const uint32_t idk = umma_idesc_bf16(128, 128);
-      const uint32_t idv = umma_idesc_bf16(128, 16, true, false);
-      uint32_t ks = 0, bs = 0, vsn = 0;
+      uint32_t ks = 0, bs = 0;
       auto issue_keys = [&](int j) -> bool {
         const int buf = j & 1;
         if (!mbar_wait(&accempty[buf], ((j >> 1) & 1) ^ 1, args.status)) return false;
@@ -715,6 +758,16 @@ __global__ void __launch_bounds__(kAttendThreads, 1)
         umma_commit(&accfull[buf]);
         return true;
       };
+      bool ok = true;
+      int j = 0;
+      for (int x = tb; x < te && ok && !*abort_flag; ++x, ++j) ok = issue_keys(j);
+      if (!ok) *abort_flag = 1;
+    }
+  } else if (warp == 15) {
+    // ------------------------------------------------------ value MMA issuer
+    if (lane == 0) {
+      const uint32_t idv = umma_idesc_bf16(128, 16, true, false);
+      uint32_t vsn = 0;
       auto issue_values = [&](int j, int x) -> bool {
         const int pb = j & 1;
         const int ti = x % tpu;
@@ -738,12 +791,9 @@ __global__ void __launch_bounds__(kAttendThreads, 1)
         umma_commit(&pempty[pb]);
         return true;
       };
-      bool ok = tb < te ? issue_keys(0) : true;
+      bool ok = true;
       int j = 0;
-      for (int x = tb; x < te && ok && !*abort_flag; ++x, ++j) {
-        if (x + 1 < te) ok = issue_keys(j + 1);
-        if (ok) ok = issue_values(j, x);
-      }
+      for (int x = tb; x < te && ok && !*abort_flag; ++x, ++j) ok = issue_values(j, x);
       if (!ok) *abort_flag = 1;
     }
   } else if (warp < 8) {
@@ -1098,6 +1148,21 @@ __global__ void __launch_bounds__(kCombineThreads) sr_combine_kernel(const T* __
     const int uf = tile_begin(c, args.n_tiles, args.ctas) / tpu;
     return args.part + (static_cast<int64_t>(c) * args.max_units + (u - uf)) * args.slot_floats;
   };
+  // E's first Bt_V rows depend on nothing: their loads are issued first and
+  // land while the slot statistics are merged
+  const int jb0 = j0 + warp * kCombineColsPerWarp;
+  uint4 pre[2][kCombineColsPerWarp];
+  if (vec) {
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+      const int v = 32 * t + lane;
+#pragma unroll
+      for (int cc = 0; cc < kCombineColsPerWarp; ++cc) {
+        const T* br = BtV + b * args.sbv + static_cast<int64_t>(h * hd + jb0 + cc) * rV;
+        pre[t][cc] = jb0 + cc < j1 && v < nv ? *reinterpret_cast<const uint4*>(br + 8 * v) : make_uint4(0, 0, 0, 0);
+      }
+    }
+  }
   // ---- A
   for (int i = tid; i < nslots * 16; i += blockDim.x) ml[i] = slot_ptr(fc + i / 16)[i % 16];
   if (tid < 16) wml[tid] = wslot[tid];
@@ -1127,14 +1192,14 @@ __global__ void __launch_bounds__(kCombineThreads) sr_combine_kernel(const T* __
     for (int i4 = tid; i4 < n4; i4 += blockDim.x) {
       const int g = (4 * i4) / rV;
       float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int c0 = 0; c0 < nslots; c0 += 8) {
-        float4 v[8];
+      for (int c0 = 0; c0 < nslots; c0 += 16) {
+        float4 v[16];
 #pragma unroll
-        for (int t = 0; t < 8; ++t)
+        for (int t = 0; t < 16; ++t)
           v[t] = c0 + t < nslots ? reinterpret_cast<const float4*>(slot_ptr(fc + c0 + t) + 16)[i4]
                                  : make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-        for (int t = 0; t < 8; ++t) {
+        for (int t = 0; t < 16; ++t) {
           if (c0 + t < nslots) {
             const float f = sc[(c0 + t) * kMaxGQ + g];
             acc.x = fmaf(v[t].x, f, acc.x);
@@ -1166,31 +1231,49 @@ __global__ void __launch_bounds__(kCombineThreads) sr_combine_kernel(const T* __
 #pragma unroll
       for (int g = 0; g < kMaxGQ; ++g) acc[cc][g] = 0.f;
     if (vec) {
-      for (int v0 = 0; v0 < nv; v0 += 32) {
-        const int v = v0 + lane;
-        uint4 w[kCombineColsPerWarp];
+      auto fold = [&](const uint4* w, int v) {
+#pragma unroll
+        for (int e2 = 0; e2 < 4; ++e2) {
+#pragma unroll
+          for (int g = 0; g < kMaxGQ; ++g) {
+            if (g < gq) {
+              const float u0 = Us[(g * 8 + 2 * e2) * nv + v], u1 = Us[(g * 8 + 2 * e2 + 1) * nv + v];
+#pragma unroll
+              for (int cc = 0; cc < kCombineColsPerWarp; ++cc) {
+                const uint32_t word = e2 == 0 ? w[cc].x : e2 == 1 ? w[cc].y : e2 == 2 ? w[cc].z : w[cc].w;
+                const float2 f = bf2_to_f2(word);
+                acc[cc][g] = fmaf(u0, f.x, fmaf(u1, f.y, acc[cc][g]));
+              }
+            }
+          }
+        }
+      };
+      auto load_w = [&](uint4* w, int v) {
 #pragma unroll
         for (int cc = 0; cc < kCombineColsPerWarp; ++cc) {
           const T* br = BtV + b * args.sbv + static_cast<int64_t>(h * hd + jb + cc) * rV;
           w[cc] = cc < ncol && v < nv ? *reinterpret_cast<const uint4*>(br + 8 * v) : make_uint4(0, 0, 0, 0);
         }
-        if (v < nv) {
+      };
+      // rank-column groups v0 = 0 and 32 (all of rV <= 512): prefetched rows
+      // for the warp's first columns
 #pragma unroll
-          for (int e2 = 0; e2 < 4; ++e2) {
+      for (int t = 0; t < 2; ++t) {
+        const int v = 32 * t + lane;
+        uint4 w[kCombineColsPerWarp];
+        if (jb == jb0) {
 #pragma unroll
-            for (int g = 0; g < kMaxGQ; ++g) {
-              if (g < gq) {
-                const float u0 = Us[(g * 8 + 2 * e2) * nv + v], u1 = Us[(g * 8 + 2 * e2 + 1) * nv + v];
-#pragma unroll
-                for (int cc = 0; cc < kCombineColsPerWarp; ++cc) {
-                  const uint32_t word = e2 == 0 ? w[cc].x : e2 == 1 ? w[cc].y : e2 == 2 ? w[cc].z : w[cc].w;
-                  const float2 f = bf2_to_f2(word);
-                  acc[cc][g] = fmaf(u0, f.x, fmaf(u1, f.y, acc[cc][g]));
-                }
-              }
-            }
-          }
+          for (int cc = 0; cc < kCombineColsPerWarp; ++cc) w[cc] = pre[t][cc];
+        } else {
+          load_w(w, v);
         }
+        if (v < nv) fold(w, v);
+      }
+      for (int v0 = 64; v0 < nv; v0 += 32) {
+        const int v = v0 + lane;
+        uint4 w[kCombineColsPerWarp];
+        load_w(w, v);
+        if (v < nv) fold(w, v);
       }
     } else {
       for (int c = lane; c < rV; c += 32) {
