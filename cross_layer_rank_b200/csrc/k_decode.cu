@@ -404,16 +404,19 @@ __global__ void __launch_bounds__(kTopkThreads) sr_topk_kernel(const float* __re
     const uint32_t b2 = topk_bucket(key, lo2, scale2);
     return b2 > B2 ? 2 : (b2 == B2 ? 1 : 0);
   };
-  // 5. final candidates (their keys, ascending index)
-  uint32_t nc = 0;
-  for (int j = 0; j < cnt; ++j) nc += klass(ksm[j * nt + tid]) == 1;
-  uint32_t cpos = block_exclusive_scan(nc, warp_tot, &s_total);
+  // 5. every key's class once, as bit masks over the thread's segment
+  // (per <= 32): kmask = kept outright, cmask = final candidates
+  uint32_t kmask = 0u, cmask = 0u;
+  for (int j = 0; j < cnt; ++j) {
+    const int c = klass(ksm[j * nt + tid]);
+    kmask |= static_cast<uint32_t>(c == 2) << j;
+    cmask |= static_cast<uint32_t>(c == 1) << j;
+  }
+  // final candidates (their keys, ascending index)
+  uint32_t cpos = block_exclusive_scan(__popc(cmask), warp_tot, &s_total);
   const uint32_t m = s_total;
   const uint32_t cbase = cpos;
-  for (int j = 0; j < cnt; ++j) {
-    const uint32_t key = ksm[j * nt + tid];
-    if (klass(key) == 1) ckey[cpos++] = key;
-  }
+  for (uint32_t bits = cmask; bits; bits &= bits - 1) ckey[cpos++] = ksm[(__ffs(bits) - 1) * nt + tid];
   __syncthreads();
   if (m == need) {
     if (tid == 0) s_all = 1u;
@@ -493,30 +496,20 @@ __global__ void __launch_bounds__(kTopkThreads) sr_topk_kernel(const float* __re
   const bool all_taken = s_all != 0u;
   // 6. ordered compaction of the selection: a final candidate is kept when
   // its decision says so (candidates are numbered in index order)
-  uint32_t n_sel = 0;
+  uint32_t take = kmask;
   {
     uint32_t ci = cbase;
-    for (int j = 0; j < cnt; ++j) {
-      const int c = klass(ksm[j * nt + tid]);
-      if (c == 1) n_sel += all_taken || ckeep[ci++];
-      else n_sel += c == 2;
-    }
+    for (uint32_t bits = cmask; bits; bits &= bits - 1, ++ci)
+      if (all_taken || ckeep[ci]) take |= 1u << (__ffs(bits) - 1);
   }
-  uint32_t pos = block_exclusive_scan(n_sel, warp_tot, &s_total);
+  uint32_t pos = block_exclusive_scan(__popc(take), warp_tot, &s_total);
   {
-    uint32_t ci = cbase;
     int32_t* o = sel + static_cast<int64_t>(unit) * k;
     int32_t* o2 = sel_out ? sel_out + static_cast<int64_t>(unit) * k : nullptr;
-    for (int j = 0; j < cnt; ++j) {
-      const int c = klass(ksm[j * nt + tid]);
-      bool take;
-      if (c == 1) take = all_taken || ckeep[ci++];
-      else take = c == 2;
-      if (take) {
-        o[pos] = i0 + j;
-        if (o2) o2[pos] = i0 + j;
-        ++pos;
-      }
+    for (uint32_t bits = take; bits; bits &= bits - 1, ++pos) {
+      const int idx = i0 + __ffs(bits) - 1;
+      o[pos] = idx;
+      if (o2) o2[pos] = idx;
     }
   }
 }
@@ -585,6 +578,217 @@ constexpr int kVAccCol = 256;  // TMEM columns of the value accumulators (2 x 64
 // 13 value TMA producer, 14 key MMA issuer (TMEM owner), 15 value MMA issuer.
 // The two issuers run independently, so the key gathers of later tiles never
 // wait behind the value products of earlier ones.
+// ------------------------------------------------------ merge of a unit
+// Final output of one unit (the combine step) by one CTA, for output columns
+// [j0, j1).  Each phase issues all of its loads before using them (one memory
+// round trip per phase):
+//   A  (m, l) of the unit's partial slots and of its window partial;
+//   C  M_g, the slot factors 2^(m - M_g) and L_g (warp per query head);
+//   D  U_g = sum over slots of u 2^(m - M_g), kept in shared memory in an
+//      order where lane-consecutive 8-column groups are word-consecutive;
+//   E  o_g[j] = (U_g . Bt_V[h hd + j] + 2^(m_w - M_g) o_w,g[j]) / L_g for the
+//      split's columns (warp per column, 16-byte loads of the Bt_V rows of
+//      all of the warp's columns issued first).
+constexpr int kCombineSplit = 4;
+constexpr int kCombineThreads = 256;
+constexpr int kMaxSlots = 64;
+constexpr int kCombineColsPerWarp = 4;
+
+// Partials are read through L2 (__ldcg): they may have been written by other
+// CTAs of the same launch.  smf: (gq rV + 64 * 24 + 32 + gq (j1 - j0) + 2 + 128)
+// floats, 16-byte aligned.
+template <typename T>
+__device__ void merge_unit(const T* __restrict__ BtV, const float* __restrict__ win, const AttendArgs& args, int hd,
+                           float* __restrict__ out, int u, int j0, int j1, float* smf) {
+  const int gq = args.Hq / args.Hkv;
+  const int b = u / args.Hkv, h = u % args.Hkv;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nwarps = blockDim.x >> 5;
+  const int tpu = args.tiles_per_unit;
+  const int rV = args.rV;
+  // bf16 rows with 8-column groups: U stored as [g][e][v] for column 8v + e
+  const bool vec = sizeof(T) == 2 && rV % 8 == 0;
+  const int nv = rV / 8;
+  float* Us = smf;                              // [gq][rV] (permuted when vec)
+  float* ml = Us + gq * rV;                     // [slots][16] partial m, l
+  float* sc = ml + kMaxSlots * 16;              // [slots][8] slot factors
+  float* wml = sc + kMaxSlots * kMaxGQ;         // [16] window m, l
+  float* Lg = wml + 16;                         // [8] 1 / L_g
+  float* fw = Lg + kMaxGQ;                      // [8] window factors
+  float* wo = fw + kMaxGQ;                      // [gq][j1 - j0] window value sums of the columns
+  const float* wslot = win + static_cast<int64_t>(u) * (16 + gq * hd);
+  const int fc = cta_of_tile(u * tpu, args.n_tiles, args.ctas);
+  const int lc = cta_of_tile((u + 1) * tpu - 1, args.n_tiles, args.ctas);
+  const int nslots = lc - fc + 1;
+  // slot i of the unit belongs to CTA fc + i; its offset is computed once
+  int64_t* soff = reinterpret_cast<int64_t*>(wo + gq * (j1 - j0) + 1) ;
+  soff = reinterpret_cast<int64_t*>((reinterpret_cast<uintptr_t>(soff) + 7) & ~uintptr_t(7));
+  for (int i = tid; i < nslots; i += blockDim.x) {
+    const int c = fc + i;
+    const int uf = tile_begin(c, args.n_tiles, args.ctas) / tpu;
+    soff[i] = (static_cast<int64_t>(c) * args.max_units + (u - uf)) * args.slot_floats;
+  }
+  __syncthreads();
+  auto slot_ptr = [&](int c) -> const float* { return args.part + soff[c - fc]; };
+  // E's first Bt_V rows depend on nothing: their loads are issued first and
+  // land while the slot statistics are merged
+  const int jb0 = j0 + warp * kCombineColsPerWarp;
+  uint4 pre[2][kCombineColsPerWarp];
+  if (vec) {
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+      const int v = 32 * t + lane;
+#pragma unroll
+      for (int cc = 0; cc < kCombineColsPerWarp; ++cc) {
+        const T* br = BtV + b * args.sbv + static_cast<int64_t>(h * hd + jb0 + cc) * rV;
+        pre[t][cc] = jb0 + cc < j1 && v < nv ? *reinterpret_cast<const uint4*>(br + 8 * v) : make_uint4(0, 0, 0, 0);
+      }
+    }
+  }
+  // ---- A
+  for (int i = tid; i < nslots * 16; i += blockDim.x) ml[i] = __ldcg(slot_ptr(fc + i / 16) + i % 16);
+  if (tid < 16) wml[tid] = __ldcg(wslot + tid);
+  for (int i = tid; i < gq * (j1 - j0); i += blockDim.x)
+    wo[i] = __ldcg(wslot + 16 + (i / (j1 - j0)) * hd + j0 + i % (j1 - j0));
+  __syncthreads();
+  // ---- C
+  for (int g = warp; g < gq; g += nwarps) {
+    float M = lane == 0 ? wml[g] : -INFINITY;
+    for (int i = lane; i < nslots; i += 32) M = fmaxf(M, ml[i * 16 + g]);
+    M = warp_max(M);
+    float L = 0.f;
+    for (int i = lane; i < nslots; i += 32) {
+      const float f = exp2f(ml[i * 16 + g] - M);
+      sc[i * kMaxGQ + g] = f;
+      L = fmaf(ml[i * 16 + 8 + g], f, L);
+    }
+    L = warp_sum(L);
+    if (lane == 0) {
+      const float f = exp2f(wml[g] - M);
+      fw[g] = f;
+      Lg[g] = 1.f / fmaf(wml[8 + g], f, L);
+    }
+  }
+  __syncthreads();
+  // ---- D (float4 over rank columns, 8 slots' loads in flight)
+  {
+    const int n4 = gq * rV / 4;
+    for (int i4 = tid; i4 < n4; i4 += blockDim.x) {
+      const int g = (4 * i4) / rV;
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int c0 = 0; c0 < nslots; c0 += 16) {
+        float4 v[16];
+#pragma unroll
+        for (int t = 0; t < 16; ++t)
+          v[t] = c0 + t < nslots ? __ldcg(reinterpret_cast<const float4*>(slot_ptr(fc + c0 + t) + 16) + i4)
+                                 : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int t = 0; t < 16; ++t) {
+          if (c0 + t < nslots) {
+            const float f = sc[(c0 + t) * kMaxGQ + g];
+            acc.x = fmaf(v[t].x, f, acc.x);
+            acc.y = fmaf(v[t].y, f, acc.y);
+            acc.z = fmaf(v[t].z, f, acc.z);
+            acc.w = fmaf(v[t].w, f, acc.w);
+          }
+        }
+      }
+      if (vec) {
+        const int c = 4 * i4 - g * rV, vv = c >> 3, e = c & 7;
+        float* dst = Us + (g * 8 + e) * nv + vv;
+        dst[0] = acc.x;
+        dst[nv] = acc.y;
+        dst[2 * nv] = acc.z;
+        dst[3 * nv] = acc.w;
+      } else {
+        reinterpret_cast<float4*>(Us)[i4] = acc;
+      }
+    }
+  }
+  __syncthreads();
+  // ---- E
+  for (int jb = j0 + warp * kCombineColsPerWarp; jb < j1; jb += nwarps * kCombineColsPerWarp) {
+    const int ncol = min(kCombineColsPerWarp, j1 - jb);
+    float acc[kCombineColsPerWarp][kMaxGQ];
+#pragma unroll
+    for (int cc = 0; cc < kCombineColsPerWarp; ++cc)
+#pragma unroll
+      for (int g = 0; g < kMaxGQ; ++g) acc[cc][g] = 0.f;
+    if (vec) {
+      auto fold = [&](const uint4* w, int v) {
+#pragma unroll
+        for (int e2 = 0; e2 < 4; ++e2) {
+#pragma unroll
+          for (int g = 0; g < kMaxGQ; ++g) {
+            if (g < gq) {
+              const float u0 = Us[(g * 8 + 2 * e2) * nv + v], u1 = Us[(g * 8 + 2 * e2 + 1) * nv + v];
+#pragma unroll
+              for (int cc = 0; cc < kCombineColsPerWarp; ++cc) {
+                const uint32_t word = e2 == 0 ? w[cc].x : e2 == 1 ? w[cc].y : e2 == 2 ? w[cc].z : w[cc].w;
+                const float2 f = bf2_to_f2(word);
+                acc[cc][g] = fmaf(u0, f.x, fmaf(u1, f.y, acc[cc][g]));
+              }
+            }
+          }
+        }
+      };
+      auto load_w = [&](uint4* w, int v) {
+#pragma unroll
+        for (int cc = 0; cc < kCombineColsPerWarp; ++cc) {
+          const T* br = BtV + b * args.sbv + static_cast<int64_t>(h * hd + jb + cc) * rV;
+          w[cc] = cc < ncol && v < nv ? *reinterpret_cast<const uint4*>(br + 8 * v) : make_uint4(0, 0, 0, 0);
+        }
+      };
+      // rank-column groups v0 = 0 and 32 (all of rV <= 512): prefetched rows
+      // for the warp's first columns
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+        const int v = 32 * t + lane;
+        uint4 w[kCombineColsPerWarp];
+        if (jb == jb0) {
+#pragma unroll
+          for (int cc = 0; cc < kCombineColsPerWarp; ++cc) w[cc] = pre[t][cc];
+        } else {
+          load_w(w, v);
+        }
+        if (v < nv) fold(w, v);
+      }
+      for (int v0 = 64; v0 < nv; v0 += 32) {
+        const int v = v0 + lane;
+        uint4 w[kCombineColsPerWarp];
+        load_w(w, v);
+        if (v < nv) fold(w, v);
+      }
+    } else {
+      for (int c = lane; c < rV; c += 32) {
+        float bv[kCombineColsPerWarp];
+#pragma unroll
+        for (int cc = 0; cc < kCombineColsPerWarp; ++cc)
+          bv[cc] = cc < ncol ? to_f(BtV[b * args.sbv + static_cast<int64_t>(h * hd + jb + cc) * rV + c]) : 0.f;
+#pragma unroll
+        for (int g = 0; g < kMaxGQ; ++g)
+          if (g < gq) {
+            const float uu = Us[g * rV + c];
+#pragma unroll
+            for (int cc = 0; cc < kCombineColsPerWarp; ++cc) acc[cc][g] = fmaf(uu, bv[cc], acc[cc][g]);
+          }
+      }
+    }
+#pragma unroll
+    for (int cc = 0; cc < kCombineColsPerWarp; ++cc) {
+#pragma unroll
+      for (int g = 0; g < kMaxGQ; ++g) {
+        if (g >= gq) break;
+        const float v = warp_sum(acc[cc][g]);
+        if (lane == 0 && cc < ncol) {
+          const int j = jb + cc;
+          out[(static_cast<int64_t>(b) * args.Hq + h * gq + g) * hd + j] =
+              fmaf(fw[g], wo[g * (j1 - j0) + j - j0], v) * Lg[g];
+        }
+      }
+    }
+  }
+}
+
 template <int GQ>
 __global__ void __launch_bounds__(kAttendThreads, 1)
     sr_attend_tc_kernel(const __grid_constant__ CUtensorMap mapAK, const __grid_constant__ CUtensorMap mapBK,
@@ -997,6 +1201,19 @@ __global__ void __launch_bounds__(kAttendThreads, 1)
 
 size_t attend_tc_smem() { return 1024 + kSmemEnd; }
 
+// ----------------------------------------------------------- sr_combine
+// Grid (unit, column split of kCombineSplit), 256 threads.
+template <typename T>
+__global__ void __launch_bounds__(kCombineThreads) sr_combine_kernel(const T* __restrict__ BtV,
+                                                                     const float* __restrict__ win,
+                                                                     const AttendArgs args, int hd,
+                                                                     float* __restrict__ out) {
+  extern __shared__ float4 smf4[];
+  const int cols = (hd + kCombineSplit - 1) / kCombineSplit, j0 = blockIdx.y * cols, j1 = min(hd, j0 + cols);
+  merge_unit<T>(BtV, win, args, hd, out, blockIdx.x, j0, j1, reinterpret_cast<float*>(smf4));
+}
+
+
 // ---------------------------------------------------- sr_attend (SIMT)
 // Same schedule and partial format; rebuilds both K and the value basis sums on
 // CUDA cores.  Tiles are 16 chunks of `chunk` rows, handled 32 rows at a time.
@@ -1104,210 +1321,11 @@ __global__ void __launch_bounds__(256) sr_attend_simt_kernel(const T* __restrict
   (void)d;
 }
 
-// ----------------------------------------------------------- sr_combine
-// Grid (unit, column split of kCombineSplit), 256 threads.  Each phase issues
-// all of its loads before using them (one memory round trip per phase):
-//   A  (m, l) of the unit's partial slots and of its window partial;
-//   C  M_g, the slot factors 2^(m - M_g) and L_g (warp per query head);
-//   D  U_g = sum over slots of u 2^(m - M_g), kept in shared memory in an
-//      order where lane-consecutive 8-column groups are word-consecutive;
-//   E  o_g[j] = (U_g . Bt_V[h hd + j] + 2^(m_w - M_g) o_w,g[j]) / L_g for the
-//      split's columns (warp per column, 16-byte loads of the Bt_V rows of
-//      all of the warp's columns issued first).
-constexpr int kCombineSplit = 4;
-constexpr int kCombineThreads = 256;
-constexpr int kMaxSlots = 64;
-constexpr int kCombineColsPerWarp = 4;
 
-template <typename T>
-__global__ void __launch_bounds__(kCombineThreads) sr_combine_kernel(const T* __restrict__ BtV,
-                                                                     const float* __restrict__ win,
-                                                                     const AttendArgs args, int hd,
-                                                                     float* __restrict__ out) {
-  extern __shared__ float4 smf4[];
-  const int gq = args.Hq / args.Hkv;
-  const int u = blockIdx.x, b = u / args.Hkv, h = u % args.Hkv;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nwarps = blockDim.x >> 5;
-  const int tpu = args.tiles_per_unit;
-  const int rV = args.rV;
-  const int cols = (hd + kCombineSplit - 1) / kCombineSplit, j0 = blockIdx.y * cols, j1 = min(hd, j0 + cols);
-  // bf16 rows with 8-column groups: U stored as [g][e][v] for column 8v + e
-  const bool vec = sizeof(T) == 2 && rV % 8 == 0;
-  const int nv = rV / 8;
-  float* Us = reinterpret_cast<float*>(smf4);   // [gq][rV] (permuted when vec)
-  float* ml = Us + gq * rV;                     // [slots][16] partial m, l
-  float* sc = ml + kMaxSlots * 16;              // [slots][8] slot factors
-  float* wml = sc + kMaxSlots * kMaxGQ;         // [16] window m, l
-  float* Lg = wml + 16;                         // [8] 1 / L_g
-  float* fw = Lg + kMaxGQ;                      // [8] window factors
-  const float* wslot = win + static_cast<int64_t>(u) * (16 + gq * hd);
-  const int fc = cta_of_tile(u * tpu, args.n_tiles, args.ctas);
-  const int lc = cta_of_tile((u + 1) * tpu - 1, args.n_tiles, args.ctas);
-  const int nslots = lc - fc + 1;
-  auto slot_ptr = [&](int c) -> const float* {
-    const int uf = tile_begin(c, args.n_tiles, args.ctas) / tpu;
-    return args.part + (static_cast<int64_t>(c) * args.max_units + (u - uf)) * args.slot_floats;
-  };
-  // E's first Bt_V rows depend on nothing: their loads are issued first and
-  // land while the slot statistics are merged
-  const int jb0 = j0 + warp * kCombineColsPerWarp;
-  uint4 pre[2][kCombineColsPerWarp];
-  if (vec) {
-#pragma unroll
-    for (int t = 0; t < 2; ++t) {
-      const int v = 32 * t + lane;
-#pragma unroll
-      for (int cc = 0; cc < kCombineColsPerWarp; ++cc) {
-        const T* br = BtV + b * args.sbv + static_cast<int64_t>(h * hd + jb0 + cc) * rV;
-        pre[t][cc] = jb0 + cc < j1 && v < nv ? *reinterpret_cast<const uint4*>(br + 8 * v) : make_uint4(0, 0, 0, 0);
-      }
-    }
-  }
-  // ---- A
-  for (int i = tid; i < nslots * 16; i += blockDim.x) ml[i] = slot_ptr(fc + i / 16)[i % 16];
-  if (tid < 16) wml[tid] = wslot[tid];
-  __syncthreads();
-  // ---- C
-  for (int g = warp; g < gq; g += nwarps) {
-    float M = lane == 0 ? wml[g] : -INFINITY;
-    for (int i = lane; i < nslots; i += 32) M = fmaxf(M, ml[i * 16 + g]);
-    M = warp_max(M);
-    float L = 0.f;
-    for (int i = lane; i < nslots; i += 32) {
-      const float f = exp2f(ml[i * 16 + g] - M);
-      sc[i * kMaxGQ + g] = f;
-      L = fmaf(ml[i * 16 + 8 + g], f, L);
-    }
-    L = warp_sum(L);
-    if (lane == 0) {
-      const float f = exp2f(wml[g] - M);
-      fw[g] = f;
-      Lg[g] = 1.f / fmaf(wml[8 + g], f, L);
-    }
-  }
-  __syncthreads();
-  // ---- D (float4 over rank columns, 8 slots' loads in flight)
-  {
-    const int n4 = gq * rV / 4;
-    for (int i4 = tid; i4 < n4; i4 += blockDim.x) {
-      const int g = (4 * i4) / rV;
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int c0 = 0; c0 < nslots; c0 += 16) {
-        float4 v[16];
-#pragma unroll
-        for (int t = 0; t < 16; ++t)
-          v[t] = c0 + t < nslots ? reinterpret_cast<const float4*>(slot_ptr(fc + c0 + t) + 16)[i4]
-                                 : make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-        for (int t = 0; t < 16; ++t) {
-          if (c0 + t < nslots) {
-            const float f = sc[(c0 + t) * kMaxGQ + g];
-            acc.x = fmaf(v[t].x, f, acc.x);
-            acc.y = fmaf(v[t].y, f, acc.y);
-            acc.z = fmaf(v[t].z, f, acc.z);
-            acc.w = fmaf(v[t].w, f, acc.w);
-          }
-        }
-      }
-      if (vec) {
-        const int c = 4 * i4 - g * rV, vv = c >> 3, e = c & 7;
-        float* dst = Us + (g * 8 + e) * nv + vv;
-        dst[0] = acc.x;
-        dst[nv] = acc.y;
-        dst[2 * nv] = acc.z;
-        dst[3 * nv] = acc.w;
-      } else {
-        reinterpret_cast<float4*>(Us)[i4] = acc;
-      }
-    }
-  }
-  __syncthreads();
-  // ---- E
-  for (int jb = j0 + warp * kCombineColsPerWarp; jb < j1; jb += nwarps * kCombineColsPerWarp) {
-    const int ncol = min(kCombineColsPerWarp, j1 - jb);
-    float acc[kCombineColsPerWarp][kMaxGQ];
-#pragma unroll
-    for (int cc = 0; cc < kCombineColsPerWarp; ++cc)
-#pragma unroll
-      for (int g = 0; g < kMaxGQ; ++g) acc[cc][g] = 0.f;
-    if (vec) {
-      auto fold = [&](const uint4* w, int v) {
-#pragma unroll
-        for (int e2 = 0; e2 < 4; ++e2) {
-#pragma unroll
-          for (int g = 0; g < kMaxGQ; ++g) {
-            if (g < gq) {
-              const float u0 = Us[(g * 8 + 2 * e2) * nv + v], u1 = Us[(g * 8 + 2 * e2 + 1) * nv + v];
-#pragma unroll
-              for (int cc = 0; cc < kCombineColsPerWarp; ++cc) {
-                const uint32_t word = e2 == 0 ? w[cc].x : e2 == 1 ? w[cc].y : e2 == 2 ? w[cc].z : w[cc].w;
-                const float2 f = bf2_to_f2(word);
-                acc[cc][g] = fmaf(u0, f.x, fmaf(u1, f.y, acc[cc][g]));
-              }
-            }
-          }
-        }
-      };
-      auto load_w = [&](uint4* w, int v) {
-#pragma unroll
-        for (int cc = 0; cc < kCombineColsPerWarp; ++cc) {
-          const T* br = BtV + b * args.sbv + static_cast<int64_t>(h * hd + jb + cc) * rV;
-          w[cc] = cc < ncol && v < nv ? *reinterpret_cast<const uint4*>(br + 8 * v) : make_uint4(0, 0, 0, 0);
-        }
-      };
-      // rank-column groups v0 = 0 and 32 (all of rV <= 512): prefetched rows
-      // for the warp's first columns
-#pragma unroll
-      for (int t = 0; t < 2; ++t) {
-        const int v = 32 * t + lane;
-        uint4 w[kCombineColsPerWarp];
-        if (jb == jb0) {
-#pragma unroll
-          for (int cc = 0; cc < kCombineColsPerWarp; ++cc) w[cc] = pre[t][cc];
-        } else {
-          load_w(w, v);
-        }
-        if (v < nv) fold(w, v);
-      }
-      for (int v0 = 64; v0 < nv; v0 += 32) {
-        const int v = v0 + lane;
-        uint4 w[kCombineColsPerWarp];
-        load_w(w, v);
-        if (v < nv) fold(w, v);
-      }
-    } else {
-      for (int c = lane; c < rV; c += 32) {
-        float bv[kCombineColsPerWarp];
-#pragma unroll
-        for (int cc = 0; cc < kCombineColsPerWarp; ++cc)
-          bv[cc] = cc < ncol ? to_f(BtV[b * args.sbv + static_cast<int64_t>(h * hd + jb + cc) * rV + c]) : 0.f;
-#pragma unroll
-        for (int g = 0; g < kMaxGQ; ++g)
-          if (g < gq) {
-            const float uu = Us[g * rV + c];
-#pragma unroll
-            for (int cc = 0; cc < kCombineColsPerWarp; ++cc) acc[cc][g] = fmaf(uu, bv[cc], acc[cc][g]);
-          }
-      }
-    }
-#pragma unroll
-    for (int cc = 0; cc < kCombineColsPerWarp; ++cc) {
-#pragma unroll
-      for (int g = 0; g < kMaxGQ; ++g) {
-        if (g >= gq) break;
-        const float v = warp_sum(acc[cc][g]);
-        if (lane == 0 && cc < ncol) {
-          const int j = jb + cc;
-          out[(static_cast<int64_t>(b) * args.Hq + h * gq + g) * hd + j] =
-              fmaf(fw[g], wslot[16 + g * hd + j], v) * Lg[g];
-        }
-      }
-    }
-  }
-}
-
-size_t combine_smem(int gq, int rV) {
-  return (static_cast<size_t>(gq) * rV + kMaxSlots * 16 + kMaxSlots * kMaxGQ + 16 + 2 * kMaxGQ) * 4 + 16;
+size_t combine_smem(int gq, int rV, int hd) {
+  const int cols = (hd + kCombineSplit - 1) / kCombineSplit;
+  return (static_cast<size_t>(gq) * rV + kMaxSlots * 16 + kMaxSlots * kMaxGQ + 16 + 2 * kMaxGQ +
+          static_cast<size_t>(gq) * cols + 2 + 2 * kMaxSlots) * 4 + 16;
 }
 
 size_t simt_smem(int gq, int rV, int hd) {
@@ -1496,7 +1514,7 @@ static xkv_status sr_launch_t(const xkv_sr_params* p, const SRPlan& plan, const 
   prof_mark(3, st);
   // 4. combine
   {
-    const size_t smem = combine_smem(gq, p->rank_v);
+    const size_t smem = combine_smem(gq, p->rank_v, p->head_dim);
     cudaFuncSetAttribute(sr_combine_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          static_cast<int>(smem));
     sr_combine_kernel<T><<<dim3(plan.units, kCombineSplit), kCombineThreads, smem, st>>>(

@@ -89,43 +89,115 @@ XKV_GEMM_INST(__nv_bfloat16, __nv_bfloat16, __nv_bfloat16, float)
 XKV_GEMM_INST(float, double, float, double)
 XKV_GEMM_INST(float, float, double, double)
 XKV_GEMM_INST(float, double, double, double)
+XKV_GEMM_INST(double, double, double, double)
 #undef XKV_GEMM_INST
 
 // ---------------------------------------------------- Cholesky QR pieces
-// In-place lower Cholesky factor of (W + shift I), b x b fp64 (row-major; only
-// the lower triangle is read and written), one CTA.  shift = shift_rel *
-// trace(W) when a device trace is given.  A non-positive pivot is recorded as
-// a numerical fault and replaced by a tiny positive one so results stay finite.
-__global__ void __launch_bounds__(1024) cholesky_kernel(double* __restrict__ W, int b, double shift_rel,
-                                                        const double* __restrict__ trace, int* status) {
-  extern __shared__ double colj[];
-  __shared__ double s_piv;
+// Lower Cholesky factor of (W + shift I), b x b fp64 row-major, in place (only
+// the lower triangle is meaningful afterwards), right-looking and blocked by
+// kCholNB: per block column k
+//   1. chol_diag_kernel  factors the diagonal block in shared memory (one CTA)
+//      and writes its inverse to a scratch block;
+//   2. chol_panel_kernel  L_ik = W_ik L_kk^{-T} for the rows below (64 rows a CTA);
+//   3. the trailing update W_ij -= L_ik L_jk^T as an fp64 GEMM over the whole
+//      trailing square (the upper part of W is scratch).
+// shift = shift_rel * trace(W) when a device trace is given; it is added to
+// each diagonal element when its block is factored.  A non-positive pivot is
+// recorded as a numerical fault and replaced by a tiny positive one so that
+// results stay finite.
+constexpr int kCholNB = 64;
+
+__global__ void __launch_bounds__(256) chol_diag_kernel(double* __restrict__ W, int b, int k0, double shift_rel,
+                                                        const double* __restrict__ trace, int* status,
+                                                        double* __restrict__ dinv) {
+  extern __shared__ double chol_sm[];
+  double(*a)[kCholNB + 1] = reinterpret_cast<double(*)[kCholNB + 1]>(chol_sm);
+  double(*x)[kCholNB + 1] = reinterpret_cast<double(*)[kCholNB + 1]>(chol_sm + kCholNB * (kCholNB + 1));
+  const int tid = threadIdx.x;
+  const int nb = min(kCholNB, b - k0);
   const double shift = trace ? shift_rel * (*trace) : 0.0;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  for (int j = 0; j < b; ++j) {
+  for (int e = tid; e < nb * nb; e += blockDim.x) {
+    const int i = e / nb, j = e % nb;
+    double v = j <= i ? W[static_cast<int64_t>(k0 + i) * b + k0 + j] : 0.0;
+    if (i == j) v += shift;
+    a[i][j] = v;
+  }
+  __syncthreads();
+  for (int j = 0; j < nb; ++j) {
     if (tid == 0) {
-      double d = W[static_cast<int64_t>(j) * b + j] + shift;
+      double d = a[j][j];
       if (!(d > 0.0) || !isfinite(d)) {
         record_status(status, kDevNumerical);
         d = 1e-300;
       }
-      s_piv = sqrt(d);
-      W[static_cast<int64_t>(j) * b + j] = s_piv;
+      a[j][j] = sqrt(d);
     }
     __syncthreads();
-    const double piv = s_piv;
-    for (int i = j + 1 + tid; i < b; i += blockDim.x) {
-      const double v = W[static_cast<int64_t>(i) * b + j] / piv;
-      W[static_cast<int64_t>(i) * b + j] = v;
-      colj[i] = v;
+    const double piv = a[j][j];
+    for (int i = j + 1 + tid; i < nb; i += blockDim.x) a[i][j] /= piv;
+    __syncthreads();
+    // trailing update of the block: pairs (i, l), j < l <= i < nb
+    const int m = nb - j - 1;
+    for (int e = tid; e < m * m; e += blockDim.x) {
+      const int i = j + 1 + e / m, l = j + 1 + e % m;
+      if (l <= i) a[i][l] -= a[i][j] * a[l][j];
     }
     __syncthreads();
-    for (int i = j + 1 + warp; i < b; i += 32) {
-      const double wij = colj[i];
-      double* wi = W + static_cast<int64_t>(i) * b;
-      for (int l = j + 1 + lane; l <= i; l += 32) wi[l] -= wij * colj[l];
+  }
+  // inverse of the factor: column c of X = L^{-1} by forward substitution
+  for (int c = tid; c < nb; c += blockDim.x) {
+    for (int i = 0; i < nb; ++i) {
+      double s = i == c ? 1.0 : 0.0;
+      for (int k = c; k < i; ++k) s -= a[i][k] * x[k][c];
+      x[i][c] = i < c ? 0.0 : s / a[i][i];
     }
-    __syncthreads();
+  }
+  __syncthreads();
+  for (int e = tid; e < nb * nb; e += blockDim.x) {
+    const int i = e / nb, j = e % nb;
+    if (j <= i) W[static_cast<int64_t>(k0 + i) * b + k0 + j] = a[i][j];
+    dinv[i * kCholNB + j] = x[i][j];
+  }
+}
+
+// Rows [k0 + nb + 64 blockIdx.x, +64) of block column k: L_ik = W_ik Linv_kk^T.
+__global__ void __launch_bounds__(256) chol_panel_kernel(double* __restrict__ W, int b, int k0,
+                                                         const double* __restrict__ dinv) {
+  extern __shared__ double chol_sm[];
+  double(*w)[kCholNB + 1] = reinterpret_cast<double(*)[kCholNB + 1]>(chol_sm);
+  double(*x)[kCholNB + 1] = reinterpret_cast<double(*)[kCholNB + 1]>(chol_sm + 64 * (kCholNB + 1));
+  const int tid = threadIdx.x;
+  const int nb = min(kCholNB, b - k0);
+  const int r0 = k0 + nb + 64 * blockIdx.x;
+  const int rows = min(64, b - r0);
+  for (int e = tid; e < rows * nb; e += blockDim.x) {
+    const int i = e / nb, j = e % nb;
+    w[i][j] = W[static_cast<int64_t>(r0 + i) * b + k0 + j];
+  }
+  for (int e = tid; e < nb * nb; e += blockDim.x) x[e / nb][e % nb] = dinv[(e / nb) * kCholNB + e % nb];
+  __syncthreads();
+  for (int e = tid; e < rows * nb; e += blockDim.x) {
+    const int i = e / nb, j = e % nb;
+    double s = 0.0;
+    for (int k = 0; k <= j; ++k) s += w[i][k] * x[j][k];
+    W[static_cast<int64_t>(r0 + i) * b + k0 + j] = s;
+  }
+}
+
+void cholesky_blocked(double* W, int b, double shift_rel, const double* trace, int* status, double* dinv,
+                      cudaStream_t st) {
+  const int smem = 2 * 64 * (kCholNB + 1) * 8;
+  cudaFuncSetAttribute(chol_diag_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  cudaFuncSetAttribute(chol_panel_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  for (int k0 = 0; k0 < b; k0 += kCholNB) {
+    chol_diag_kernel<<<1, 256, smem, st>>>(W, b, k0, shift_rel, trace, status, dinv);
+    const int nb = std::min(kCholNB, b - k0);
+    const int rem = b - k0 - nb;
+    if (rem <= 0) break;
+    chol_panel_kernel<<<(rem + 63) / 64, 256, smem, st>>>(W, b, k0, dinv);
+    double* P = W + static_cast<int64_t>(k0 + nb) * b + k0;  // rem x nb panel, row stride b
+    gemm_simt<double, double, double, double>(P, b, 1, P, 1, b, W + static_cast<int64_t>(k0 + nb) * b + k0 + nb,
+                                              b, rem, rem, nb, -1.0, 1.0, st);
   }
 }
 
@@ -173,9 +245,8 @@ void cholqr_pass(const float* Y, float* Q, int n, int b, double shift_rel, doubl
                  int* status, cudaStream_t st) {
   gemm_simt<float, float, double, double>(Y, 1, b, Y, b, 1, W, b, b, b, n, 1.0, 0.0, st);
   if (shift_rel > 0.0) trace_kernel<<<1, 256, 0, st>>>(W, b, scal);
-  const size_t smem = static_cast<size_t>(b) * 8;
-  cudaFuncSetAttribute(cholesky_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-  cholesky_kernel<<<1, 1024, smem, st>>>(W, b, shift_rel, shift_rel > 0.0 ? scal : nullptr, status);
+  // Linv is free until the inverse below: its first block holds the diagonal inverses
+  cholesky_blocked(W, b, shift_rel, shift_rel > 0.0 ? scal : nullptr, status, Linv, st);
   const size_t smem2 = static_cast<size_t>(8) * b * 8;
   cudaFuncSetAttribute(tri_inverse_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem2));
   tri_inverse_kernel<<<(b + 7) / 8, 256, smem2, st>>>(W, Linv, b);
