@@ -20,6 +20,7 @@
 #include <float.h>
 
 #include <algorithm>
+#include <utility>
 
 #include "xkv_common.cuh"
 #include "xkv_internal.h"
@@ -38,6 +39,14 @@ constexpr int kAtomBytes = 16384;  // 128 rows x 64 bf16
 constexpr int kAttendThreads = 512;  // 16 warps: 8 key epilogue, 4 value epilogue, 2 TMA, 2 MMA
 
 // ----------------------------------------------------------------- helpers
+// Programmatic dependent launch: the later kernels of a decode step may start
+// while the previous one drains; each waits here before its first read of the
+// previous kernel's output (a no-op when launched without the attribute).
+__device__ __forceinline__ void wait_prior_grid() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// lets the next kernel of the step be scheduled once every CTA of this grid
+// has started (its CTAs then wait in wait_prior_grid for this grid's end)
+__device__ __forceinline__ void allow_next_grid() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 __host__ __device__ inline int tile_begin(int c, int n_tiles, int ctas) {
   return static_cast<int>((static_cast<int64_t>(c) * n_tiles) / ctas);
 }
@@ -94,6 +103,7 @@ template <typename T>
 __global__ void __launch_bounds__(256) sr_score_kernel(const T* __restrict__ q, const T* __restrict__ lm,
                                                        float* __restrict__ scores, int Hq, int Hkv, int hd,
                                                        int64_t n_mid, int chunks_per_block) {
+  allow_next_grid();
   __shared__ float qbar[256];
   const int unit = blockIdx.y;
   const int b = unit / Hkv, h = unit % Hkv, gq = Hq / Hkv;
@@ -300,6 +310,7 @@ __global__ void __launch_bounds__(kTopkThreads) sr_topk_kernel(const float* __re
                                                                int32_t* __restrict__ sel_out, int64_t n_mid, int k,
                                                                int units, const __grid_constant__ WinArgs wa) {
   extern __shared__ uint32_t ksm[];  // [per][1024] keys (transposed), [n] candidate keys, [n] decisions
+  allow_next_grid();
   if (static_cast<int>(blockIdx.x) >= units) {
     window_partial<T>(wa, blockIdx.x - units, reinterpret_cast<uint8_t*>(ksm));
     return;
@@ -317,6 +328,7 @@ __global__ void __launch_bounds__(kTopkThreads) sr_topk_kernel(const float* __re
   uint8_t* ckeep = reinterpret_cast<uint8_t*>(ckey + n);
   hist[tid] = 0u;
   if (tid == 0) { s_lo = 0xFFFFFFFFu; s_hi = 0u; }
+  wait_prior_grid();  // the chunk scores
   // 1. keys (row start 16-byte aligned: ld is a multiple of 4) and their range
   uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
   {
@@ -644,6 +656,7 @@ __device__ void merge_unit(const T* __restrict__ BtV, const float* __restrict__ 
       }
     }
   }
+  wait_prior_grid();  // the partial slots (and, through the attend grid's own wait, the window partials)
   // ---- A
   for (int i = tid; i < nslots * 16; i += blockDim.x) ml[i] = __ldcg(slot_ptr(fc + i / 16) + i % 16);
   if (tid < 16) wml[tid] = __ldcg(wslot + tid);
@@ -871,6 +884,8 @@ __global__ void __launch_bounds__(kAttendThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  allow_next_grid();
+  wait_prior_grid();  // the selection
 
   if (warp == 12) {
     // ------------------------------------------------------ TMA producer (keys)
@@ -1239,6 +1254,7 @@ __global__ void __launch_bounds__(256) sr_attend_simt_kernel(const T* __restrict
   const int d = args.Hkv * hd;
   const float qscale = rsqrtf(static_cast<float>(hd)) * kLog2e;
   for (int j = tid; j < half; j += blockDim.x) ft[j] = args.ft[j];
+  wait_prior_grid();  // the selection
   int cur_u = -1;
   for (int x = tb; x < te; ++x) {
     const int u = x / tpu, ti = x % tpu;
@@ -1371,6 +1387,25 @@ xkv_status sr_plan(const xkv_sr_params* p, SRPlan* plan) {
   return XKV_OK;
 }
 
+// Launch with programmatic stream serialization: the kernel may start while
+// the previous kernel in the stream drains and waits for it in
+// wait_prior_grid before reading its output.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_after_prior(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                               Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
 // stage-timing events (see xkv_sr_profile_enable)
 struct SRProfile {
   bool on = false, recorded = false;
@@ -1429,9 +1464,11 @@ static xkv_status sr_launch_t(const xkv_sr_params* p, const SRPlan& plan, const 
                                  window_smem(gq, p->head_dim, nsr));
     // the opt-in covers static + dynamic shared memory above 48 KiB
     cudaFuncSetAttribute(sr_topk_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-    sr_topk_kernel<T><<<2 * plan.units, kTopkThreads, smem, st>>>(scores, (n_mid + 3) & ~int64_t(3), sel, sel_out, n_mid,
-                                                                   p->topk, plan.units, wa);
-    if (cudaPeekAtLastError() != cudaSuccess) return XKV_ERR_CUDA;
+    const int64_t ld = (n_mid + 3) & ~int64_t(3);
+    if (launch_after_prior(sr_topk_kernel<T>, dim3(2 * plan.units), dim3(kTopkThreads), smem, st,
+                           static_cast<const float*>(scores), ld, sel, sel_out, n_mid, static_cast<int>(p->topk),
+                           static_cast<int>(plan.units), wa) != cudaSuccess)
+      return XKV_ERR_CUDA;
   }
   prof_mark(2, st);
   AttendArgs a;
@@ -1501,14 +1538,17 @@ static xkv_status sr_launch_t(const xkv_sr_params* p, const SRPlan& plan, const 
       default: kern = sr_attend_tc_kernel<8>; break;
     }
     cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-    kern<<<plan.ctas, kAttendThreads, smem, st>>>(mAK, mBK, mAV, a);
+    if (launch_after_prior(kern, dim3(plan.ctas), dim3(kAttendThreads), smem, st, mAK, mBK, mAV, a) != cudaSuccess)
+      return XKV_ERR_CUDA;
   } else {
     const size_t smem = simt_smem(gq, p->rank_v, p->head_dim);
     cudaFuncSetAttribute(sr_attend_simt_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          static_cast<int>(smem));
-    sr_attend_simt_kernel<T><<<plan.ctas, 256, smem, st>>>(
-        static_cast<const T*>(q), static_cast<const T*>(A_K), static_cast<const T*>(Bt_K),
-        static_cast<const T*>(A_V), a, p->head_dim, p->chunk, p->a_k_batch_stride, p->a_v_batch_stride);
+    if (launch_after_prior(sr_attend_simt_kernel<T>, dim3(plan.ctas), dim3(256), smem, st, static_cast<const T*>(q),
+                           static_cast<const T*>(A_K), static_cast<const T*>(Bt_K), static_cast<const T*>(A_V), a,
+                           static_cast<int>(p->head_dim), static_cast<int>(p->chunk), p->a_k_batch_stride,
+                           p->a_v_batch_stride) != cudaSuccess)
+      return XKV_ERR_CUDA;
   }
   if (cudaPeekAtLastError() != cudaSuccess) return XKV_ERR_CUDA;
   prof_mark(3, st);
@@ -1517,8 +1557,10 @@ static xkv_status sr_launch_t(const xkv_sr_params* p, const SRPlan& plan, const 
     const size_t smem = combine_smem(gq, p->rank_v, p->head_dim);
     cudaFuncSetAttribute(sr_combine_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          static_cast<int>(smem));
-    sr_combine_kernel<T><<<dim3(plan.units, kCombineSplit), kCombineThreads, smem, st>>>(
-        static_cast<const T*>(Bt_V), win, a, p->head_dim, out);
+    if (launch_after_prior(sr_combine_kernel<T>, dim3(plan.units, kCombineSplit), dim3(kCombineThreads), smem, st,
+                           static_cast<const T*>(Bt_V), static_cast<const float*>(win), a,
+                           static_cast<int>(p->head_dim), out) != cudaSuccess)
+      return XKV_ERR_CUDA;
   }
   prof_mark(4, st);
   return cudaPeekAtLastError() == cudaSuccess ? XKV_OK : XKV_ERR_CUDA;
