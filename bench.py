@@ -212,6 +212,26 @@ def measure_gram(xkv, w, device):
     return ms, flops
 
 
+# --------------------------------------------------------- multi-rank
+def max_over_ranks(values, world: int, device=None):
+    """Element-wise maximum over all ranks of per-rank device times (every
+    rank calls it, in the same order); the identity for one rank."""
+    if world <= 1:
+        return list(values)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.cpu()]
+
+
+def job_throughput(batch_per_rank: int, world: int, ms_step: float):
+    """Whole-job tokens per step and tokens/s: every rank decodes its own
+    batch (independent sequences), the step lasts as long as the slowest rank."""
+    tokens = batch_per_rank * world
+    return tokens, tokens / (ms_step / 1e3)
+
+
 # ------------------------------------------------------------------- arms
 def run_cuda(args, rank, world, log):
     import torch
@@ -312,13 +332,9 @@ def run_cuda(args, rank, world, log):
     assert xkv.get_device_status(stream) == 0
     clocks = clk.summary()
 
-    if world > 1:
-        t = torch.tensor([ms_total, e2e_ms], dtype=torch.float64, device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_total, e2e_ms = float(t[0]), float(t[1])
+    ms_total, e2e_ms = max_over_ranks([ms_total, e2e_ms], world, device)
     ms_step = ms_total / args.steps
-    tokens = w.batch * world
-    value = tokens / (ms_step / 1e3)
+    tokens, value = job_throughput(w.batch, world, ms_step)
     units_step = w.batch * L * w.n_kv_heads
     bytes_step = sr_bytes_per_unit(w) * units_step
     hbm_gbs_peak, bf16_peak, _, peak_kind = _peaks()
