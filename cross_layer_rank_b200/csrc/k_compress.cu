@@ -124,7 +124,7 @@ __global__ void emit_factors_kernel(const float* __restrict__ Vr, int n, int r, 
 // rows; the outer sum is an ordinary round-to-nearest fp32 chain.
 constexpr int kGramChunkStages = 4;  // 4 x 64 rows per TMEM chunk
 constexpr int kGramStages = 4;
-constexpr int kGramThreads = 192;
+constexpr int kGramThreads = 320;  // producer, MMA issuer, 8 epilogue warps (2 per TMEM lane quarter)
 
 inline size_t gram_tc_smem() { return 1024 + kGramStages * 2 * 16384 + (2 * kGramStages + 4) * 8 + 16; }
 
@@ -146,7 +146,7 @@ __global__ void __launch_bounds__(kGramThreads, 1)
   const int nchunks = (nk + kGramChunkStages - 1) / kGramChunkStages;
   if (tid == 0) {
     for (int i = 0; i < kGramStages; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
-    for (int i = 0; i < 2; ++i) { mbar_init(&accfull[i], 1); mbar_init(&accempty[i], 128); }
+    for (int i = 0; i < 2; ++i) { mbar_init(&accfull[i], 1); mbar_init(&accempty[i], 256); }
     fence_mbar_init();
   }
   if (warp == 1) tmem_alloc(tslot, 256);
@@ -190,37 +190,37 @@ __global__ void __launch_bounds__(kGramThreads, 1)
       }
     }
   } else {
-    const int lq = warp & 3;
+    // warp w reads TMEM lane quarter w % 4; warps 2-5 own columns 0-63 of the
+    // tile, warps 6-9 columns 64-127
+    const int lq = warp & 3, half = (warp - 2) >> 2;
     const int row = lq * 32 + lane;
-    const uint32_t tbase = tmem + (static_cast<uint32_t>(lq * 32) << 16);
-    float acc[128];
+    const uint32_t tbase = tmem + (static_cast<uint32_t>(lq * 32) << 16) + half * 64;
+    float acc[64];
 #pragma unroll
-    for (int i = 0; i < 128; ++i) acc[i] = 0.f;
+    for (int i = 0; i < 64; ++i) acc[i] = 0.f;
     bool ok = true;
     for (int c = 0; c < nchunks; ++c) {
       const int buf = c & 1;
       if (!mbar_wait(&accfull[buf], (c >> 1) & 1, status)) { ok = false; break; }
       tc_fence_after();
+      float v[64];
 #pragma unroll
-      for (int jb = 0; jb < 8; jb += 2) {
-        float v[32];
-        tmem_ld16(tbase + buf * 128 + jb * 16, v);
-        tmem_ld16(tbase + buf * 128 + jb * 16 + 16, v + 16);
-        tmem_ld_wait();
-#pragma unroll
-        for (int i = 0; i < 32; ++i) acc[jb * 16 + i] += v[i];
-      }
+      for (int jb = 0; jb < 4; ++jb) tmem_ld16(tbase + buf * 128 + jb * 16, v + jb * 16);
+      tmem_ld_wait();
       tc_fence_before();
       mbar_arrive(&accempty[buf]);
+#pragma unroll
+      for (int i = 0; i < 64; ++i) acc[i] += v[i];
     }
     if (ok) {
       // read-modify-write of C in batches whose loads are all issued before
       // any of their stores (C is read and written through one pointer, so a
       // plain += loop would wait for every load in turn)
       const int m = m0 + row;
-      float* crow = C + static_cast<int64_t>(m) * ldc + n0;
+      const int nb = n0 + half * 64;
+      float* crow = C + static_cast<int64_t>(m) * ldc + nb;
 #pragma unroll
-      for (int i0 = 0; i0 < 128; i0 += 32) {
+      for (int i0 = 0; i0 < 64; i0 += 32) {
         float4 cv[8];
 #pragma unroll
         for (int u = 0; u < 8; ++u) cv[u] = *reinterpret_cast<const float4*>(crow + i0 + 4 * u);
@@ -238,12 +238,12 @@ __global__ void __launch_bounds__(kGramThreads, 1)
         // the mirrored tile: lanes hold consecutive m, so each access is one
         // 128-byte row segment per warp
 #pragma unroll
-        for (int i0 = 0; i0 < 128; i0 += 16) {
-          float v[16];
+        for (int i0 = 0; i0 < 64; i0 += 16) {
+          float w[16];
 #pragma unroll
-          for (int u = 0; u < 16; ++u) v[u] = C[static_cast<int64_t>(n0 + i0 + u) * ldc + m];
+          for (int u = 0; u < 16; ++u) w[u] = C[static_cast<int64_t>(nb + i0 + u) * ldc + m];
 #pragma unroll
-          for (int u = 0; u < 16; ++u) C[static_cast<int64_t>(n0 + i0 + u) * ldc + m] = v[u] + acc[i0 + u];
+          for (int u = 0; u < 16; ++u) C[static_cast<int64_t>(nb + i0 + u) * ldc + m] = w[u] + acc[i0 + u];
         }
       }
     }

@@ -47,6 +47,13 @@ __device__ __forceinline__ void wait_prior_grid() { asm volatile("griddepcontrol
 // has started (its CTAs then wait in wait_prior_grid for this grid's end)
 __device__ __forceinline__ void allow_next_grid() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
+// 16-byte asynchronous global -> shared copies (L2 only)
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem)), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
 __host__ __device__ inline int tile_begin(int c, int n_tiles, int ctas) {
   return static_cast<int>((static_cast<int64_t>(c) * n_tiles) / ctas);
 }
@@ -605,6 +612,7 @@ constexpr int kCombineSplit = 4;
 constexpr int kCombineThreads = 256;
 constexpr int kMaxSlots = 64;
 constexpr int kCombineColsPerWarp = 4;
+constexpr int kCombineStageBytes = 64 * 1024;  // Bt_V rows staged for E, when they fit
 
 // Partials are read through L2 (__ldcg): they may have been written by other
 // CTAs of the same launch.  smf: (gq rV + 64 * 24 + 32 + gq (j1 - j0) + 2 + 128)
@@ -618,7 +626,7 @@ __device__ void merge_unit(const T* __restrict__ BtV, const float* __restrict__ 
   const int tpu = args.tiles_per_unit;
   const int rV = args.rV;
   // bf16 rows with 8-column groups: U stored as [g][e][v] for column 8v + e
-  const bool vec = sizeof(T) == 2 && rV % 8 == 0;
+  const bool vec = sizeof(T) == 2 && rV % 8 == 0 && args.sbv % 8 == 0;
   const int nv = rV / 8;
   float* Us = smf;                              // [gq][rV] (permuted when vec)
   float* ml = Us + gq * rV;                     // [slots][16] partial m, l
@@ -641,21 +649,18 @@ __device__ void merge_unit(const T* __restrict__ BtV, const float* __restrict__ 
   }
   __syncthreads();
   auto slot_ptr = [&](int c) -> const float* { return args.part + soff[c - fc]; };
-  // E's first Bt_V rows depend on nothing: their loads are issued first and
-  // land while the slot statistics are merged
-  const int jb0 = j0 + warp * kCombineColsPerWarp;
-  uint4 pre[2][kCombineColsPerWarp];
-  if (vec) {
-#pragma unroll
-    for (int t = 0; t < 2; ++t) {
-      const int v = 32 * t + lane;
-#pragma unroll
-      for (int cc = 0; cc < kCombineColsPerWarp; ++cc) {
-        const T* br = BtV + b * args.sbv + static_cast<int64_t>(h * hd + jb0 + cc) * rV;
-        pre[t][cc] = jb0 + cc < j1 && v < nv ? *reinterpret_cast<const uint4*>(br + 8 * v) : make_uint4(0, 0, 0, 0);
-      }
+  // E's Bt_V rows depend on nothing: cp.async stages them in shared memory
+  // while the partials are merged (when they fit; else E loads them itself)
+  const int ncols = j1 - j0;
+  uint4* Bs = reinterpret_cast<uint4*>((reinterpret_cast<uintptr_t>(soff + kMaxSlots) + 15) & ~uintptr_t(15));
+  const bool staged = vec && static_cast<int64_t>(ncols) * rV * 2 <= kCombineStageBytes;
+  if (staged) {
+    for (int i = tid; i < ncols * nv; i += blockDim.x) {
+      const int cc = i / nv, v = i - cc * nv;
+      cp_async16(Bs + i, BtV + b * args.sbv + static_cast<int64_t>(h * hd + j0 + cc) * rV + 8 * v);
     }
   }
+  cp_async_commit();
   wait_prior_grid();  // the partial slots (and, through the attend grid's own wait, the window partials)
   // ---- A
   for (int i = tid; i < nslots * 16; i += blockDim.x) ml[i] = __ldcg(slot_ptr(fc + i / 16) + i % 16);
@@ -717,6 +722,7 @@ __device__ void merge_unit(const T* __restrict__ BtV, const float* __restrict__ 
       }
     }
   }
+  cp_async_wait_all();
   __syncthreads();
   // ---- E
   for (int jb = j0 + warp * kCombineColsPerWarp; jb < j1; jb += nwarps * kCombineColsPerWarp) {
@@ -730,45 +736,32 @@ __device__ void merge_unit(const T* __restrict__ BtV, const float* __restrict__ 
       auto fold = [&](const uint4* w, int v) {
 #pragma unroll
         for (int e2 = 0; e2 < 4; ++e2) {
+          float2 f[kCombineColsPerWarp];
+#pragma unroll
+          for (int cc = 0; cc < kCombineColsPerWarp; ++cc)
+            f[cc] = bf2_to_f2(e2 == 0 ? w[cc].x : e2 == 1 ? w[cc].y : e2 == 2 ? w[cc].z : w[cc].w);
 #pragma unroll
           for (int g = 0; g < kMaxGQ; ++g) {
             if (g < gq) {
               const float u0 = Us[(g * 8 + 2 * e2) * nv + v], u1 = Us[(g * 8 + 2 * e2 + 1) * nv + v];
 #pragma unroll
-              for (int cc = 0; cc < kCombineColsPerWarp; ++cc) {
-                const uint32_t word = e2 == 0 ? w[cc].x : e2 == 1 ? w[cc].y : e2 == 2 ? w[cc].z : w[cc].w;
-                const float2 f = bf2_to_f2(word);
-                acc[cc][g] = fmaf(u0, f.x, fmaf(u1, f.y, acc[cc][g]));
-              }
+              for (int cc = 0; cc < kCombineColsPerWarp; ++cc) acc[cc][g] = fmaf(u0, f[cc].x, fmaf(u1, f[cc].y, acc[cc][g]));
             }
           }
         }
       };
-      auto load_w = [&](uint4* w, int v) {
-#pragma unroll
-        for (int cc = 0; cc < kCombineColsPerWarp; ++cc) {
-          const T* br = BtV + b * args.sbv + static_cast<int64_t>(h * hd + jb + cc) * rV;
-          w[cc] = cc < ncol && v < nv ? *reinterpret_cast<const uint4*>(br + 8 * v) : make_uint4(0, 0, 0, 0);
-        }
-      };
-      // rank-column groups v0 = 0 and 32 (all of rV <= 512): prefetched rows
-      // for the warp's first columns
-#pragma unroll
-      for (int t = 0; t < 2; ++t) {
-        const int v = 32 * t + lane;
-        uint4 w[kCombineColsPerWarp];
-        if (jb == jb0) {
-#pragma unroll
-          for (int cc = 0; cc < kCombineColsPerWarp; ++cc) w[cc] = pre[t][cc];
-        } else {
-          load_w(w, v);
-        }
-        if (v < nv) fold(w, v);
-      }
-      for (int v0 = 64; v0 < nv; v0 += 32) {
+      for (int v0 = 0; v0 < nv; v0 += 32) {
         const int v = v0 + lane;
         uint4 w[kCombineColsPerWarp];
-        load_w(w, v);
+#pragma unroll
+        for (int cc = 0; cc < kCombineColsPerWarp; ++cc) {
+          if (cc < ncol && v < nv)
+            w[cc] = staged ? Bs[(jb - j0 + cc) * nv + v]
+                           : *reinterpret_cast<const uint4*>(BtV + b * args.sbv +
+                                                             static_cast<int64_t>(h * hd + jb + cc) * rV + 8 * v);
+          else
+            w[cc] = make_uint4(0, 0, 0, 0);
+        }
         if (v < nv) fold(w, v);
       }
     } else {
@@ -786,18 +779,24 @@ __device__ void merge_unit(const T* __restrict__ BtV, const float* __restrict__ 
           }
       }
     }
+    // reduce-scatter of the 32 sums over the warp: lane l ends with the
+    // total of entry l = (column cc, head g) = (l / 8, l % 8)
+    static_assert(kCombineColsPerWarp * kMaxGQ == 32, "one entry per lane");
+    float* a = &acc[0][0];
 #pragma unroll
-    for (int cc = 0; cc < kCombineColsPerWarp; ++cc) {
+    for (int st = 16; st >= 1; st >>= 1) {
+      const bool up = (lane & st) != 0;
 #pragma unroll
-      for (int g = 0; g < kMaxGQ; ++g) {
-        if (g >= gq) break;
-        const float v = warp_sum(acc[cc][g]);
-        if (lane == 0 && cc < ncol) {
-          const int j = jb + cc;
-          out[(static_cast<int64_t>(b) * args.Hq + h * gq + g) * hd + j] =
-              fmaf(fw[g], wo[g * (j1 - j0) + j - j0], v) * Lg[g];
-        }
+      for (int i = 0; i < st; ++i) {
+        const float keep = up ? a[i + st] : a[i];
+        const float send = up ? a[i] : a[i + st];
+        a[i] = keep + __shfl_xor_sync(0xffffffffu, send, st);
       }
+    }
+    const int cc = lane / kMaxGQ, g = lane % kMaxGQ;
+    if (g < gq && cc < ncol) {
+      const int j = jb + cc;
+      out[(static_cast<int64_t>(b) * args.Hq + h * gq + g) * hd + j] = fmaf(fw[g], wo[g * (j1 - j0) + j - j0], a[0]) * Lg[g];
     }
   }
 }
@@ -1340,8 +1339,10 @@ __global__ void __launch_bounds__(256) sr_attend_simt_kernel(const T* __restrict
 
 size_t combine_smem(int gq, int rV, int hd) {
   const int cols = (hd + kCombineSplit - 1) / kCombineSplit;
+  const size_t stage = static_cast<size_t>(cols) * rV * 2;
   return (static_cast<size_t>(gq) * rV + kMaxSlots * 16 + kMaxSlots * kMaxGQ + 16 + 2 * kMaxGQ +
-          static_cast<size_t>(gq) * cols + 2 + 2 * kMaxSlots) * 4 + 16;
+          static_cast<size_t>(gq) * cols + 2 + 2 * kMaxSlots) * 4 + 16 + 16 +
+         (stage <= static_cast<size_t>(kCombineStageBytes) ? stage : 0);
 }
 
 size_t simt_smem(int gq, int rV, int hd) {
