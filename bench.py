@@ -331,6 +331,7 @@ def run_cuda(args, rank, world, log):
         e2e_ms = e2.elapsed_time(e3)
     assert xkv.get_device_status(stream) == 0
     clocks = clk.summary()
+    comparison = measure_full_reconstruction(xkv, w, model, device, stream, call_ms) if args.comparison else None
 
     ms_total, e2e_ms = max_over_ranks([ms_total, e2e_ms], world, device)
     ms_step = ms_total / args.steps
@@ -384,6 +385,8 @@ def run_cuda(args, rank, world, log):
         "clocks": clocks,
         "flops_per_step": sr_flops_per_unit(w) * units_step,
     }
+    if comparison is not None:
+        res["comparison"] = comparison
     if args.prefill:
         cm = prefill["compress_ms"]
         res["prefill"] = {"compress_group_ms_median": round(statistics.median(cm), 3), "groups_compressed": len(cm),
@@ -392,6 +395,43 @@ def run_cuda(args, rank, world, log):
                           "gram_tflops": round(gram_flops / (gram_ms / 1e3) / 1e12, 1),
                           "gram_frac_of_bf16_peak": round(gram_flops / (gram_ms / 1e3) / 1e12 / bf16_peak, 4)}
     return res, w
+
+
+def measure_full_reconstruction(xkv, w, model, device, stream, sr_call_ms):
+    """The comparison path of one layer for the whole batch: every K row
+    rebuilt (A_K Bt_K^T + RoPE) and every V row rebuilt (A_V Bt_V^T), then
+    dense decode attention over the T rebuilt rows; device time per layer,
+    median over eager runs with L2 flushed in between, beside the SR call."""
+    import torch
+    bf = torch.bfloat16
+    B, T, d = w.batch, w.T, w.d
+    K = torch.empty((B, T, d), dtype=bf, device=device)
+    V = torch.empty((B, T, d), dtype=bf, device=device)
+    out = torch.empty((B, w.n_q_heads, w.head_dim), dtype=torch.float32, device=device)
+    dp = xkv.dense_params(B, w.n_q_heads, w.n_kv_heads, w.head_dim, T, bf)
+    dws = xkv.workspace(xkv.xkv_dense_workspace_size(dp), device)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+    times = []
+    with torch.cuda.stream(stream):
+        for it in range(6):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for b in range(B):
+                xkv.xkv_full_reconstruct(model["A_K"][0][b], model["Bt_K"][0][b], w.n_kv_heads, w.head_dim, True,
+                                         w.rope_theta, K[b], stream)
+                xkv.xkv_full_reconstruct(model["A_V"][0][b], model["Bt_V"][0][b], w.n_kv_heads, w.head_dim, False,
+                                         w.rope_theta, V[b], stream)
+            xkv.xkv_dense_attention_decode(dp, model["q"][0], K, V, out, dws, stream)
+            e1.record(stream)
+            e1.synchronize()
+            if it > 0:
+                times.append(e0.elapsed_time(e1))
+    ms = statistics.median(times)
+    del K, V, flush
+    return {"path": "xkv_full_reconstruct (K with RoPE, V) for every row + xkv_dense_attention_decode",
+            "ms_per_layer": round(ms, 4), "sr_ms_per_layer": round(sr_call_ms, 4),
+            "sr_speedup": round(ms / sr_call_ms, 2)}
 
 
 def cpu_baseline(w, budget_s: float, log):
@@ -447,6 +487,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-prefill", dest="prefill", action="store_false")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--no-comparison", dest="comparison", action="store_false",
+                    help="skip timing the full-reconstruction comparison path")
     args = ap.parse_args()
     rank = int(os.environ.get("RANK", 0))
     world = int(os.environ.get("WORLD_SIZE", 1))

@@ -144,3 +144,17 @@ def test_sr_full_size_llama8b_64k_batch4_layer(xkv):
 
 def test_sr_full_size_qwen7b_128k_batch2_layer(xkv):
     _parity(xkv, synth.WORKLOADS["qwen7b_128k_b2"], layer=3)
+
+
+def test_stage_timing_reports_every_launch(xkv):
+    # xkv_sr_profile_enable / xkv_sr_profile_read: four non-negative stage
+    # durations of the last call; the attend stage did work
+    w = synth.Workload("sr_profile", 2, 4, 4, 2, 128, 8, 8 + 32 + 8 * 150, 96, 0.8, 128, 192, topk=37)
+    d_inp = sr_inputs_on_device(w, synth.compressed_cache(w, 0))
+    xkv.xkv_sr_profile_enable(True)
+    try:
+        run_sr(xkv, w, d_inp)
+        ms = xkv.xkv_sr_profile_read()
+    finally:
+        xkv.xkv_sr_profile_enable(False)
+    assert len(ms) == 4 and all(np.isfinite(ms)) and min(ms) >= 0.0 and ms[2] > 0.0
