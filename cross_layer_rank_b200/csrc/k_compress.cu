@@ -256,6 +256,172 @@ __global__ void __launch_bounds__(kGramThreads, 1)
   }
 }
 
+
+// Wide variant for n % 256 == 0: tiles of 128 rows x 256 columns (row block tm,
+// column block tn >= tm / 2, so every upper-triangular entry belongs to exactly
+// one tile), fp32 accumulators of 256 TMEM columns, double-buffered (all 512
+// columns).  Per 64-row step the MMA reads 12 KB of operands for twice the
+// work of a 128 x 128 tile, which leaves shared-memory bandwidth for the TMA
+// writes.  Entries left of the diagonal in a straddling tile are skipped; the
+// others are added to C and (off the diagonal) mirrored.
+constexpr int kGramWStages = 4;
+constexpr int kGramWStage = 16384 + 32768;  // A: 128 x 64, B: 256 x 64 bf16
+constexpr int kGramWThreads = 576;          // producer, MMA issuer, 16 epilogue warps
+
+inline size_t gram_tc256_smem() { return 1024 + kGramWStages * kGramWStage + (2 * kGramWStages + 4) * 8 + 16; }
+
+__global__ void __launch_bounds__(kGramWThreads, 1)
+    gram_tc256_kernel(const __grid_constant__ CUtensorMap xmap, int nk, int tiles_m, int tiles_w, float* __restrict__ C,
+                      int64_t ldc, int* status) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kGramWStages * kGramWStage);
+  uint64_t* empty = full + kGramWStages;
+  uint64_t* accfull = empty + kGramWStages;
+  uint64_t* accempty = accfull + 2;
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(accempty + 2);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  // tile list: row block tm holds column blocks tn = tm / 2 .. tiles_w - 1
+  int idx = blockIdx.x, tm = 0;
+  while (tm < tiles_m && idx >= tiles_w - tm / 2) { idx -= tiles_w - tm / 2; ++tm; }
+  const int tn = tm / 2 + idx;
+  const int m0 = tm * 128, n0 = tn * 256;
+  const int nchunks = (nk + kGramChunkStages - 1) / kGramChunkStages;
+  if (tid == 0) {
+    for (int i = 0; i < kGramWStages; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
+    for (int i = 0; i < 2; ++i) { mbar_init(&accfull[i], 1); mbar_init(&accempty[i], 512); }
+    fence_mbar_init();
+  }
+  if (warp == 1) tmem_alloc(tslot, 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tslot;
+  if (warp == 0) {
+    if (lane == 0) {
+      for (int a = 0; a < nk; ++a) {
+        const int slot = a % kGramWStages;
+        if (!mbar_wait(&empty[slot], ((a / kGramWStages) & 1) ^ 1, status)) break;
+        uint8_t* st = smem + slot * kGramWStage;
+        mbar_arrive_expect_tx(&full[slot], kGramWStage);
+        tma_load_2d(st, &xmap, &full[slot], a * 64, m0);
+        tma_load_2d(st + 16384, &xmap, &full[slot], a * 64, n0);
+        tma_load_2d(st + 32768, &xmap, &full[slot], a * 64, n0 + 128);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idesc = umma_idesc_bf16(128, 256);
+      int a = 0;
+      bool ok = true;
+      for (int c = 0; c < nchunks && ok; ++c) {
+        const int buf = c & 1;
+        if (!mbar_wait(&accempty[buf], ((c >> 1) & 1) ^ 1, status)) break;
+        tc_fence_after();
+        for (int s = 0; s < kGramChunkStages && a < nk; ++s, ++a) {
+          const int slot = a % kGramWStages;
+          if (!mbar_wait(&full[slot], (a / kGramWStages) & 1, status)) { ok = false; break; }
+          tc_fence_after();
+          uint8_t* st = smem + slot * kGramWStage;
+          const uint64_t ad = umma_desc_sw128(smem_u32(st));
+          const uint64_t bd = umma_desc_sw128(smem_u32(st + 16384));
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            umma_bf16(tmem + buf * 256, ad + 2 * kk, bd + 2 * kk, idesc, (s | kk) ? 1u : 0u);
+          umma_commit(&empty[slot]);
+        }
+        umma_commit(&accfull[buf]);
+      }
+    }
+  } else {
+    // warp w reads TMEM lane quarter w % 4; warps 2-5, 6-9, 10-13, 14-17 own
+    // columns 0-63, 64-127, 128-191, 192-255 of the tile
+    const int lq = warp & 3, quarter = (warp - 2) >> 2;
+    const int row = lq * 32 + lane;
+    const uint32_t tbase = tmem + (static_cast<uint32_t>(lq * 32) << 16) + quarter * 64;
+    float acc[64];
+#pragma unroll
+    for (int i = 0; i < 64; ++i) acc[i] = 0.f;
+    bool ok = true;
+    for (int c = 0; c < nchunks; ++c) {
+      const int buf = c & 1;
+      if (!mbar_wait(&accfull[buf], (c >> 1) & 1, status)) { ok = false; break; }
+      tc_fence_after();
+#pragma unroll
+      for (int jb = 0; jb < 4; ++jb) {
+        float v[16];
+        tmem_ld16(tbase + buf * 256 + jb * 16, v);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) acc[jb * 16 + i] += v[i];
+      }
+      tc_fence_before();
+      mbar_arrive(&accempty[buf]);
+    }
+    if (ok) {
+      const int m = m0 + row;
+      const int nb = n0 + quarter * 64;
+      if (nb > m) {
+        // whole column block right of the diagonal: batched read-modify-write
+        // (loads of a batch before its stores, C read and written through one
+        // pointer), then the mirrored entries
+        float* crow = C + static_cast<int64_t>(m) * ldc + nb;
+#pragma unroll
+        for (int i0 = 0; i0 < 64; i0 += 16) {
+          float4 cv[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) cv[u] = *reinterpret_cast<const float4*>(crow + i0 + 4 * u);
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int i = i0 + 4 * u;
+            cv[u].x += acc[i];
+            cv[u].y += acc[i + 1];
+            cv[u].z += acc[i + 2];
+            cv[u].w += acc[i + 3];
+            *reinterpret_cast<float4*>(crow + i) = cv[u];
+          }
+        }
+#pragma unroll
+        for (int i0 = 0; i0 < 64; i0 += 8) {
+          float w[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) w[u] = C[static_cast<int64_t>(nb + i0 + u) * ldc + m];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) C[static_cast<int64_t>(nb + i0 + u) * ldc + m] = w[u] + acc[i0 + u];
+        }
+      } else if (nb + 63 >= m) {
+        // the block meets the diagonal: entries j >= m, mirrored when j > m
+        // (predicated batches, loads before stores)
+        float* crow = C + static_cast<int64_t>(m) * ldc + nb;
+#pragma unroll
+        for (int i0 = 0; i0 < 64; i0 += 8) {
+          float w[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) w[u] = nb + i0 + u >= m ? crow[i0 + u] : 0.f;
+#pragma unroll
+          for (int u = 0; u < 8; ++u)
+            if (nb + i0 + u >= m) crow[i0 + u] = w[u] + acc[i0 + u];
+        }
+#pragma unroll
+        for (int i0 = 0; i0 < 64; i0 += 8) {
+          float w[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) w[u] = nb + i0 + u > m ? C[static_cast<int64_t>(nb + i0 + u) * ldc + m] : 0.f;
+#pragma unroll
+          for (int u = 0; u < 8; ++u)
+            if (nb + i0 + u > m) C[static_cast<int64_t>(nb + i0 + u) * ldc + m] = w[u] + acc[i0 + u];
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
 bool gram_tc_ok(int G, int d, xkv_dtype dt) { return dt == XKV_BF16 && (G * d) % 128 == 0 && !force_simt(); }
 
 }  // namespace
@@ -285,10 +451,19 @@ xkv_status gram_launch(const void* const* X, int G, int64_t rows, int d, int64_t
       return XKV_ERR_CUDA;
     const int tiles_n = n / 128;
     const int nk = static_cast<int>((rows + 63) / 64);
-    const size_t smem = gram_tc_smem();
-    cudaFuncSetAttribute(gram_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-    gram_tc_kernel<<<tiles_n * (tiles_n + 1) / 2, kGramThreads, smem, st>>>(xm, nk, tiles_n, C, n,
-                                                                             device_status_ptr());
+    if (n % 256 == 0) {
+      const int tiles_w = n / 256;
+      int tiles = 0;
+      for (int tm = 0; tm < tiles_n; ++tm) tiles += tiles_w - tm / 2;
+      const size_t smem = gram_tc256_smem();
+      cudaFuncSetAttribute(gram_tc256_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+      gram_tc256_kernel<<<tiles, kGramWThreads, smem, st>>>(xm, nk, tiles_n, tiles_w, C, n, device_status_ptr());
+    } else {
+      const size_t smem = gram_tc_smem();
+      cudaFuncSetAttribute(gram_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+      gram_tc_kernel<<<tiles_n * (tiles_n + 1) / 2, kGramThreads, smem, st>>>(xm, nk, tiles_n, C, n,
+                                                                               device_status_ptr());
+    }
   } else {
     for (int li = 0; li < G; ++li)
       for (int lj = 0; lj < G; ++lj) {
