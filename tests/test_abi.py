@@ -55,6 +55,15 @@ def test_sr_rejects_bad_shapes(xkv, bad):
         xkv.XKV_ERR_INVALID_ARG
 
 
+def test_sr_reports_unsupported_beyond_the_chunk_limit(xkv):
+    # n_mid = 24577: one middle chunk more than the top-k's shared memory holds
+    p = _sr(xkv, T=8 + 32 + 8 * 24577)
+    n = C.c_size_t(0)
+    assert xkv.lib.xkv_sr_workspace_size(C.byref(p), C.byref(n)) == xkv.XKV_ERR_UNSUPPORTED
+    p = _sr(xkv, T=8 + 32 + 8 * 24576)
+    assert xkv.lib.xkv_sr_workspace_size(C.byref(p), C.byref(n)) == xkv.XKV_OK
+
+
 def test_sr_rejects_null_and_misaligned_pointers_and_small_workspace(xkv):
     p = _sr(xkv)
     n = C.c_size_t(0)

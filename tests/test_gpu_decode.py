@@ -13,6 +13,7 @@ Llama-3.1-8B shape (64K, batch 4, sampled units) and the Qwen2.5-7B shape
 """
 import numpy as np
 import pytest
+import torch
 
 import oracle
 import synth
@@ -158,3 +159,41 @@ def test_stage_timing_reports_every_launch(xkv):
     finally:
         xkv.xkv_sr_profile_enable(False)
     assert len(ms) == 4 and all(np.isfinite(ms)) and min(ms) >= 0.0 and ms[2] > 0.0
+
+
+def test_sr_without_sink_or_recent_window(xkv):
+    # degenerate window: no raw rows at all, attention over the kept chunks only
+    w = synth.Workload("sr_nowin", 2, 4, 4, 2, 128, 8, 8 * 150, 96, 0.8, 128, 128, topk=37, sink=0, recent=0)
+    _parity(xkv, w)
+
+
+def test_sr_single_chunk_kept(xkv):
+    w = synth.Workload("sr_k1", 2, 4, 4, 2, 128, 8, 8 + 32 + 8 * 90, 96, 0.8, 128, 128, topk=1)
+    _parity(xkv, w)
+
+
+def test_sr_factors_shared_by_the_batch(xkv):
+    # Bt_K and Bt_V given once for the whole batch (batch stride 0)
+    w = synth.Workload("sr_shared_bt", 3, 4, 4, 2, 128, 8, 8 + 32 + 8 * 120, 96, 0.8, 128, 192, topk=33)
+    inp = synth.compressed_cache(w, 0)
+    inp["Bt_K"], inp["Bt_V"] = inp["Bt_K"][0], inp["Bt_V"][0]
+    d_inp = sr_inputs_on_device(w, inp)
+    B = w.batch
+    p = xkv.sr_params(B, w.n_q_heads, w.n_kv_heads, w.head_dim, w.T, w.rank_k, w.rank_v, w.chunk, w.topk, w.sink,
+                      w.recent, w.rope_theta, torch.bfloat16, bt_k_batch_stride=0, bt_v_batch_stride=0)
+    out = torch.full((B, w.n_q_heads, w.head_dim), float("nan"), device="cuda", dtype=torch.float32)
+    sel = torch.full((B, w.n_kv_heads, w.topk), -1, device="cuda", dtype=torch.int32)
+    xkv.xkv_sr_attention_decode(p, d_inp["q"], d_inp["A_K"], d_inp["Bt_K"], d_inp["A_V"], d_inp["Bt_V"],
+                                d_inp["landmarks"], d_inp["sr_K"], d_inp["sr_V"], out, sel)
+    torch.cuda.synchronize()
+    sel = sel.cpu().numpy()
+    _, _, scores = oracle.sr_decode(w, **inp)
+    check_selection(sel, scores, w.topk)
+    ref, _, _ = oracle.sr_decode(w, sel_in=sel, **inp)
+    assert np.abs(host(out) - ref).max() <= 1e-2
+
+
+def test_sr_largest_supported_chunk_count(xkv):
+    # n_mid = 24576 middle chunks (the top-k shared-memory limit), one unit
+    w = synth.Workload("sr_max_chunks", 1, 4, 4, 1, 128, 4, 8 + 32 + 8 * 24576, 96, 0.8, 128, 128, topk=96)
+    _parity(xkv, w)
