@@ -41,7 +41,7 @@ EXPORTS = (
     "xkv_sr_profile_enable", "xkv_sr_profile_read",
     "xkv_full_reconstruct",
     "xkv_dense_workspace_size", "xkv_dense_attention_decode",
-    "xkv_ner_workspace_size", "xkv_ner",
+    "xkv_ner_workspace_size", "xkv_ner", "xkv_energy_rank",
 )
 
 
@@ -96,6 +96,7 @@ def _load():
         "xkv_dense_attention_decode": (C.c_int, [C.POINTER(DenseParams), vp, vp, vp, vp, vp, sz, vp]),
         "xkv_ner_workspace_size": (C.c_int, [C.c_int, C.c_int, C.POINTER(sz)]),
         "xkv_ner": (C.c_int, [vp, C.c_int, C.c_int, C.c_double, vp, vp, vp, vp, sz, vp]),
+        "xkv_energy_rank": (C.c_int, [vp, C.c_int, C.c_int, C.c_double, vp, vp, vp, sz, vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -296,3 +297,16 @@ def xkv_ner(gram: torch.Tensor, block: int, ner_out, erank_out=None, rank_out=No
     ws = ws if ws is not None else workspace(xkv_ner_workspace_size(n, block), gram.device)
     _check(lib.xkv_ner(_ptr(gram), n, block, rank_rel_tol, _ptr(ner_out), _ptr(erank_out), _ptr(rank_out), _ptr(ws),
                        ws.numel(), _stream(stream)), "xkv_ner")
+
+
+def xkv_energy_rank(gram, block: int, energy: float = 0.95, rank_out=None, lambda_out=None, ws=None, stream=None):
+    """Per diagonal block: the rank keeping `energy` of the block's eigenvalue
+    total, and optionally its eigenvalues in descending order."""
+    n = gram.shape[0]
+    count = n // block
+    rank_out = rank_out if rank_out is not None else torch.empty(count, dtype=torch.int32, device=gram.device)
+    ws = ws if ws is not None else workspace(xkv_ner_workspace_size(n, block), gram.device)
+    _check(lib.xkv_energy_rank(_ptr(gram), n, block, float(energy), _ptr(rank_out), _ptr(lambda_out), _ptr(ws),
+                               ws.numel(), _stream(stream)), "xkv_energy_rank")
+    return rank_out
+

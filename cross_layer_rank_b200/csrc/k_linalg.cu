@@ -529,6 +529,65 @@ __global__ void __launch_bounds__(256) ner_kernel(const double* __restrict__ lam
   }
 }
 
+// ---------------------------------------------------------- energy rank
+// One CTA per block (xKV explainer, Fig. 2(c)): the block's eigenvalues
+// (negative ones count as 0) placed in descending order by their rank (ties:
+// lower index first), a block-wide prefix sum, and the smallest k whose k
+// largest eigenvalues reach `energy` of the total (0 for a zero block).
+__global__ void __launch_bounds__(256) energy_rank_kernel(const double* __restrict__ lam, int n, double energy,
+                                                          int32_t* __restrict__ rank_out, float* __restrict__ lam_out) {
+  extern __shared__ double srt[];  // [n] descending
+  __shared__ double wsum[8];
+  __shared__ double s_total;
+  __shared__ int s_rank;
+  const double* l = lam + static_cast<int64_t>(blockIdx.x) * n;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  for (int i = tid; i < n; i += blockDim.x) {
+    const double x = fmax(l[i], 0.0);
+    int pos = 0;
+    for (int j = 0; j < n; ++j) {
+      const double y = fmax(l[j], 0.0);
+      pos += (y > x) || (y == x && j < i);
+    }
+    srt[pos] = x;
+  }
+  if (tid == 0) s_rank = n;
+  __syncthreads();
+  // thread t sums its contiguous run [t c, (t+1) c) of the sorted values
+  const int c = (n + blockDim.x - 1) / blockDim.x, i0 = min(n, tid * c), i1 = min(n, i0 + c);
+  double run = 0.0;
+  for (int i = i0; i < i1; ++i) run += srt[i];
+  double incl = run;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const double y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) wsum[warp] = incl;
+  __syncthreads();
+  double before = 0.0;
+  for (int w = 0; w < warp; ++w) before += wsum[w];
+  if (tid == 0) {
+    double t = 0.0;
+    for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) t += wsum[w];
+    s_total = t;
+  }
+  __syncthreads();
+  const double total = s_total, target = energy * total;
+  double cum = before + incl - run;  // sum of the values ahead of this run
+  for (int i = i0; i < i1; ++i) {
+    cum += srt[i];
+    if (total > 0.0 && cum >= target) {
+      atomicMin(&s_rank, i + 1);
+      break;
+    }
+  }
+  __syncthreads();
+  if (tid == 0) rank_out[blockIdx.x] = total > 0.0 ? s_rank : 0;
+  if (lam_out)
+    for (int i = tid; i < n; i += blockDim.x) lam_out[static_cast<int64_t>(blockIdx.x) * n + i] = static_cast<float>(srt[i]);
+}
+
 // diagonal blocks of an n x n fp32 Gram -> count x (block x block) fp64
 __global__ void extract_blocks_kernel(const float* __restrict__ C, int n, int block, double* __restrict__ out) {
   const int b = blockIdx.y;
@@ -558,6 +617,22 @@ xkv_status ner_launch(const float* gram, int n, int block, double tol, float* ne
   xkv_status s = jacobi_launch(Wb, nullptr, lam, block, count, jws, st);
   if (s != XKV_OK) return s;
   ner_kernel<<<count, 256, 0, st>>>(lam, block, tol, ner, erank, rank);
+  return cudaPeekAtLastError() == cudaSuccess ? XKV_OK : XKV_ERR_CUDA;
+}
+
+xkv_status energy_rank_launch(const float* gram, int n, int block, double energy, int32_t* rank, float* lam_out,
+                               void* ws, cudaStream_t st) {
+  const int count = n / block;
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  double* Wb = reinterpret_cast<double*>(w);
+  double* lam = reinterpret_cast<double*>(w + align_up(static_cast<size_t>(count) * block * block * 8));
+  void* jws = w + align_up(static_cast<size_t>(count) * block * block * 8) + align_up(static_cast<size_t>(count) * block * 8);
+  extract_blocks_kernel<<<dim3(128, count), 256, 0, st>>>(gram, n, block, Wb);
+  xkv_status s = jacobi_launch(Wb, nullptr, lam, block, count, jws, st);
+  if (s != XKV_OK) return s;
+  const size_t smem = static_cast<size_t>(block) * 8;
+  cudaFuncSetAttribute(energy_rank_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  energy_rank_kernel<<<count, 256, smem, st>>>(lam, block, energy, rank, lam_out);
   return cudaPeekAtLastError() == cudaSuccess ? XKV_OK : XKV_ERR_CUDA;
 }
 

@@ -359,4 +359,14 @@ xkv_status xkv_ner(const float* gram, int n, int block, double rank_rel_tol, flo
                     static_cast<cudaStream_t>(stream));
 }
 
+xkv_status xkv_energy_rank(const float* gram, int n, int block, double energy, int32_t* rank_out, float* lambda_out,
+                           void* workspace, size_t ws_bytes, void* stream) {
+  if (!gram || !rank_out || !aligned16(gram) || n < 2 || block < 2 || block % 2 != 0 || n % block != 0)
+    return XKV_ERR_INVALID_ARG;
+  if (!(energy > 0.0) || !(energy <= 1.0)) return XKV_ERR_INVALID_ARG;
+  if (block > 8192) return XKV_ERR_UNSUPPORTED;
+  if (!workspace || ws_bytes < ner_workspace(n, block) || !aligned256(workspace)) return XKV_ERR_WORKSPACE;
+  return energy_rank_launch(gram, n, block, energy, rank_out, lambda_out, workspace, static_cast<cudaStream_t>(stream));
+}
+
 }  // extern "C"

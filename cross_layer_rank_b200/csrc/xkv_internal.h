@@ -72,6 +72,8 @@ xkv_status compress_launch(const CompressPlan& plan, const void* const* X, int G
 
 // ------------------------------------------------------------------ NER
 size_t ner_workspace(int n, int block);
+xkv_status energy_rank_launch(const float* gram, int n, int block, double energy, int32_t* rank, float* lam_out,
+                               void* ws, cudaStream_t st);
 xkv_status ner_launch(const float* gram, int n, int block, double tol, float* ner, float* erank, int32_t* rank,
                       void* ws, cudaStream_t st);
 

@@ -233,6 +233,17 @@ XKV_API xkv_status xkv_ner(const float* gram, int n, int block, double rank_rel_
                    float* erank_out, int32_t* rank_out, void* workspace, size_t ws_bytes,
                    void* stream);
 
+/* Energy rank per diagonal block ([xKV-blog] Fig. 2(c): the rank that keeps a
+ * given share of a layer's cache energy).  Eigenvalues lambda of C_ll, with
+ * values below zero (rounding only) counted as 0, sorted descending; rank =
+ * the smallest k with lambda_1 + ... + lambda_k >= energy * sum_i lambda_i, or
+ * 0 for a zero block.
+ *   rank_out [n/block] int32; lambda_out [n/block][block] f32 descending, or NULL.
+ *   energy in (0, 1]; n % block == 0, block even and <= 8192 (else
+ *   XKV_ERR_UNSUPPORTED).  Workspace: xkv_ner_workspace_size(n, block). */
+XKV_API xkv_status xkv_energy_rank(const float* gram, int n, int block, double energy, int32_t* rank_out,
+                                   float* lambda_out, void* workspace, size_t ws_bytes, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

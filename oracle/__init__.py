@@ -222,3 +222,21 @@ def ner(Cm: np.ndarray, block: int, rel_tol: float = 1e-9):
     if rc != 0:
         raise RuntimeError("oracle Jacobi did not converge")
     return nr, er, rk, ev
+
+
+def energy_rank(Cm: np.ndarray, block: int, energy: float = 0.95):
+    """[xKV-blog] Fig. 2(c): per diagonal block C_ll, the smallest k whose k
+    largest eigenvalues hold `energy` of the block's total (eigenvalues below
+    zero, which only rounding produces, count as 0; 0 for a zero block).
+    Eigenvalues from the oracle's Jacobi; returns (ranks, eigenvalues sorted
+    descending)."""
+    _, _, _, ev = ner(Cm, block)
+    lam = np.sort(np.maximum(ev, 0.0), axis=1)[:, ::-1]
+    ranks = np.zeros(lam.shape[0], dtype=np.int32)
+    for i, l in enumerate(lam):
+        total = l.sum()
+        if total > 0.0:
+            cum = np.cumsum(l)
+            ranks[i] = int(np.searchsorted(cum, energy * total, side="left")) + 1
+    return ranks, lam
+

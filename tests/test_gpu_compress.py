@@ -157,3 +157,30 @@ def test_compress_full_size_llama_group_16k_properties(xkv):
     assert np.abs(Bt.T @ Bt - np.eye(r)).max() <= 2e-2
     sto = np.linalg.norm(X - A @ Bt.T)
     assert sto <= best * 1.05
+
+
+@pytest.mark.parametrize("energy", [0.5, 0.9, 0.95, 0.99])
+def test_energy_rank_matches_oracle(xkv, energy):
+    # per-layer rank for a share of the cache energy, from the GPU's fp32 Gram;
+    # the GPU rank must reach the target on the oracle's spectrum and its
+    # predecessor must not (within 1e-5 of the total: the Gram is fp32)
+    w = synth.WORKLOADS["tiny_f32"].replace(name="energy", n_kv_heads=2, head_dim=64, group=3, n_layers=3)
+    layers = _layers(w, 1536)
+    n, d = 3 * 128, 128
+    X = [dev(l, torch.float32) for l in layers]
+    Cg = torch.zeros((n, n), dtype=torch.float32, device="cuda")
+    xkv.xkv_gram_accumulate(X, Cg)
+    lam_g = torch.empty((n // d, d), dtype=torch.float32, device="cuda")
+    rk = xkv.xkv_energy_rank(Cg, d, energy, lambda_out=lam_g)
+    torch.cuda.synchronize()
+    rk, lam_g = rk.cpu().numpy(), host(lam_g)
+    ranks_o, lam_o = oracle.energy_rank(oracle.gram(layers), d, energy)
+    for blk in range(n // d):
+        cum = np.cumsum(lam_o[blk])
+        total = cum[-1]
+        k = int(rk[blk])
+        assert 1 <= k <= d
+        assert cum[k - 1] >= energy * total - 1e-5 * total
+        assert k == 1 or cum[k - 2] < energy * total + 1e-5 * total
+        assert abs(k - ranks_o[blk]) <= 1
+        assert np.abs(lam_g[blk] - lam_o[blk]).max() <= 1e-4 * lam_o[blk][0]

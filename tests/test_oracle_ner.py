@@ -60,3 +60,43 @@ def test_per_block_reading_and_zero_block():
     ref, _, _, _ = oracle.ner(A.T @ A, 8)
     assert abs(ner[0] - ref[0]) < 1e-14
     assert ner[1] == 0.0 and rank[1] == 0 and erank[1] == 0.0
+
+
+# --------------------------------------------------------- energy rank
+def _diag_gram(blocks):
+    n = sum(len(b) for b in blocks)
+    C = np.zeros((n, n))
+    o = 0
+    for b in blocks:
+        C[o:o + len(b), o:o + len(b)] = np.diag(b)
+        o += len(b)
+    return C
+
+
+def test_energy_rank_closed_forms():
+    # flat: 16 equal eigenvalues need ceil(0.95 * 16) = 16; geometric 2^-i,
+    # i = 0..15: 2 - 2^(1-k) >= 0.95 (2 - 2^-15) first holds at k = 5; one
+    # dominant value: 1; a zero block: 0
+    flat = np.ones(64)
+    geo = 0.5 ** np.arange(16)
+    dom = np.concatenate([[1.0], np.full(15, 1e-9)])
+    zero = np.zeros(16)
+    C = _diag_gram([flat[:16], geo, dom, zero])
+    ranks, lam = oracle.energy_rank(C, 16, 0.95)
+    assert list(ranks) == [16, 5, 1, 0]
+    assert np.all(np.diff(lam, axis=1) <= 0)
+
+
+def test_energy_rank_rotation_invariant_and_matches_lapack():
+    # a rotated spectrum gives the same rank; eigenvalues agree with LAPACK
+    rng = np.random.default_rng(3)
+    d = 32
+    Q, _ = np.linalg.qr(rng.standard_normal((d, d)))
+    lam = np.sort(rng.uniform(0, 1, d) ** 4)[::-1]
+    M = Q @ np.diag(lam) @ Q.T
+    for e in (0.5, 0.9, 0.99):
+        r_rot, l_rot = oracle.energy_rank(M, d, e)
+        r_diag, _ = oracle.energy_rank(np.diag(lam), d, e)
+        assert r_rot[0] == r_diag[0] == int(np.searchsorted(np.cumsum(lam), e * lam.sum())) + 1
+        assert np.allclose(l_rot[0], np.sort(np.linalg.eigvalsh(M))[::-1], atol=1e-12)
+
