@@ -67,6 +67,36 @@ def attend_bytes_per_unit(w) -> int:
             + w.gq * w.head_dim * el)
 
 
+def stage_rooflines(w, stage_ms, peak_gbs):
+    """Achieved GB/s of each decode launch of one layer call (whole batch)
+    against the HBM peak, from its algorithmic bytes:
+      score   the landmarks and the queries;
+      top-k   the chunk scores (fp32) and, for the window blocks, the raw
+              sink/recent K and V rows (latency-bound: few bytes);
+      attend  the selected A rows, the Bt_K head slices and the queries;
+      combine the Bt_V head slices and the outputs (plus partials in L2)."""
+    el = 2 if w.dtype == "bf16" else 4
+    units = w.batch * w.n_kv_heads
+    byts = {
+        "score": units * (w.n_mid * w.head_dim * el + w.gq * w.head_dim * el),
+        "topk_window": units * (w.n_mid * 4 + (w.sink + w.recent) * w.head_dim * 2 * el),
+        "attend": units * attend_bytes_per_unit(w),
+        "combine": units * (w.rank_v * w.head_dim * el + w.gq * w.head_dim * 4),
+    }
+    out = {}
+    for (name, b), ms in zip(byts.items(), stage_ms):
+        gbs = b / (ms / 1e3) / 1e9 if ms > 0 else 0.0
+        out[name] = {"bytes": int(b), "achieved_gbs": round(gbs, 1), "frac": round(gbs / peak_gbs, 4)}
+    return out
+
+
+def landmark_bytes(w) -> int:
+    """xkv_build_landmarks for one layer and sequence: T rows of K read, the
+    middle chunks' landmarks written."""
+    el = 2 if w.dtype == "bf16" else 4
+    return w.T * w.d * el + w.n_kv_heads * w.n_mid * w.head_dim * el
+
+
 def sr_flops_per_unit(w) -> int:
     rows = w.topk * w.chunk
     return (2 * rows * w.rank_k * w.head_dim                 # K rebuild
@@ -377,6 +407,7 @@ def run_cuda(args, rank, world, log):
                      "launch_ms": round(stage_ms[2], 5)},
         "stages_ms": {"score": round(stage_ms[0], 5), "topk_window": round(stage_ms[1], 5),
                       "attend": round(stage_ms[2], 5), "combine": round(stage_ms[3], 5)},
+        "stage_rooflines": stage_rooflines(w, stage_ms, hbm_gbs_peak),
         "layer_call": {"ms": round(call_ms, 5), "bytes": bytes_call, "achieved_gbs": round(achieved_call, 1),
                        "frac": round(achieved_call / hbm_gbs_peak, 4)},
         "e2e": {"value": round(tokens / (e2e_ms / args.steps / 1e3), 2), "unit": "tokens/s",
@@ -391,6 +422,8 @@ def run_cuda(args, rank, world, log):
         cm = prefill["compress_ms"]
         res["prefill"] = {"compress_group_ms_median": round(statistics.median(cm), 3), "groups_compressed": len(cm),
                           "landmarks_ms_median": round(statistics.median(prefill["landmarks_ms"]), 4),
+                          "landmarks_frac_of_hbm": round(landmark_bytes(w) / (statistics.median(prefill["landmarks_ms"]) /
+                                                                               1e3) / 1e9 / hbm_gbs_peak, 4),
                           "gram_ms": round(gram_ms, 4),
                           "gram_tflops": round(gram_flops / (gram_ms / 1e3) / 1e12, 1),
                           "gram_frac_of_bf16_peak": round(gram_flops / (gram_ms / 1e3) / 1e12 / bf16_peak, 4)}
@@ -429,9 +462,14 @@ def measure_full_reconstruction(xkv, w, model, device, stream, sr_call_ms):
                 times.append(e0.elapsed_time(e1))
     ms = statistics.median(times)
     del K, V, flush
+    el = 2
+    # algorithmic bytes: A and Bt read, rebuilt K and V written, then read by the dense pass
+    byts = B * (T * (w.rank_k + w.rank_v) * el + d * (w.rank_k + w.rank_v) * el + 2 * 2 * T * d * el)
     return {"path": "xkv_full_reconstruct (K with RoPE, V) for every row + xkv_dense_attention_decode",
             "ms_per_layer": round(ms, 4), "sr_ms_per_layer": round(sr_call_ms, 4),
-            "sr_speedup": round(ms / sr_call_ms, 2)}
+            "sr_speedup": round(ms / sr_call_ms, 2), "bytes_per_layer": int(byts),
+            "achieved_gbs": round(byts / (ms / 1e3) / 1e9, 1),
+            "note": "comparison kernels untuned: the ratio overstates SR's advantage"}
 
 
 def cpu_baseline(w, budget_s: float, log):
