@@ -104,3 +104,17 @@ def test_landmarks_recon_dense_ner_validation(xkv):
     assert xkv.lib.xkv_dense_workspace_size(C.byref(bad), C.byref(n)) == xkv.XKV_ERR_INVALID_ARG
     assert xkv.lib.xkv_ner_workspace_size(100, 30, C.byref(n)) == xkv.XKV_ERR_INVALID_ARG
     assert xkv.lib.xkv_ner(fake, 128, 64, 1e-9, fake, None, None, None, 0, None) == xkv.XKV_ERR_WORKSPACE
+
+
+def test_energy_rank_validation(xkv):
+    # argument checks run before any device work: fake, aligned pointers suffice
+    g, r, ws = C.c_void_p(0x10000), C.c_void_p(0x20000), C.c_void_p(0x30000)
+    n = C.c_size_t(0)
+    assert xkv.lib.xkv_ner_workspace_size(256, 128, C.byref(n)) == xkv.XKV_OK
+    f = xkv.lib.xkv_energy_rank
+    assert f(g, 256, 128, 0.0, r, None, ws, n.value, None) == xkv.XKV_ERR_INVALID_ARG     # energy <= 0
+    assert f(g, 256, 128, 1.5, r, None, ws, n.value, None) == xkv.XKV_ERR_INVALID_ARG     # energy > 1
+    assert f(g, 256, 100, 0.9, r, None, ws, n.value, None) == xkv.XKV_ERR_INVALID_ARG     # n % block
+    assert f(g, 256, 128, 0.9, None, None, ws, n.value, None) == xkv.XKV_ERR_INVALID_ARG  # no rank output
+    assert f(g, 256, 128, 0.9, r, None, ws, n.value - 1, None) == xkv.XKV_ERR_WORKSPACE
+    assert f(g, 2 * 16384, 16384, 0.9, r, None, ws, 1 << 40, None) == xkv.XKV_ERR_UNSUPPORTED  # block > 8192
