@@ -191,6 +191,21 @@ void dense_split(const xkv_dense_params* p, int* splits, int64_t* per) {
 }
 
 // --------------------------------------------------------------- landmarks
+__device__ __forceinline__ void load2(const __nv_bfloat16* p, float* x) {
+  const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(p));
+  x[0] = f.x;
+  x[1] = f.y;
+}
+__device__ __forceinline__ void load2(const float* p, float* x) {
+  const float2 f = *reinterpret_cast<const float2*>(p);
+  x[0] = f.x;
+  x[1] = f.y;
+}
+__device__ __forceinline__ void store2(__nv_bfloat16* p, float a, float b) {
+  *reinterpret_cast<__nv_bfloat162*>(p) = __floats2bfloat162_rn(a, b);
+}
+__device__ __forceinline__ void store2(float* p, float a, float b) { *reinterpret_cast<float2*>(p) = make_float2(a, b); }
+
 template <typename T>
 __global__ void __launch_bounds__(256) landmarks_kernel(const T* __restrict__ K, int64_t ldk, int hd, int chunk,
                                                         int sink, int64_t n_mid, float theta, int chunks_per_block,
@@ -219,6 +234,61 @@ __global__ void __launch_bounds__(256) landmarks_kernel(const T* __restrict__ K,
     T* o = out + (static_cast<int64_t>(h) * n_mid + c) * hd;
     store_f(o + j, a0 * inv);
     store_f(o + j + half, a1 * inv);
+  }
+}
+
+// Same landmarks, one warp per chunk: lane l owns the frequency pairs
+// (2l, 2l + 1) (+ 64 per further pass) and reads them as 2-element vectors;
+// the angle of token t0 + e is the chunk's base angle (one turn reduction per
+// chunk and frequency) rotated by the offset e from a shared table (angle
+// addition), so a chunk costs one sin/cos pair per frequency instead of one
+// per token.
+constexpr int kLmRotMax = 40 * 1024;  // rotation table bytes: chunk x half x (cos, sin), under the 48 KiB default
+
+template <typename T>
+__global__ void __launch_bounds__(256) landmarks_rot_kernel(const T* __restrict__ K, int64_t ldk, int hd, int chunk,
+                                                            int sink, int64_t n_mid, float theta,
+                                                            int chunks_per_block, T* __restrict__ out) {
+  extern __shared__ float2 rot[];  // [chunk][half] (cos, sin) of e f_j turns
+  __shared__ double ft[128];
+  const int h = blockIdx.y, half = hd / 2;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+  for (int j = threadIdx.x; j < half; j += blockDim.x) ft[j] = rope_turns(theta, j, hd);
+  __syncthreads();
+  for (int i = threadIdx.x; i < chunk * half; i += blockDim.x) {
+    float c, sn;
+    rope_cs(ft[i % half], static_cast<double>(i / half), &c, &sn);
+    rot[i] = make_float2(c, sn);
+  }
+  __syncthreads();
+  const int64_t c0 = static_cast<int64_t>(blockIdx.x) * chunks_per_block;
+  const int64_t c1 = min(n_mid, c0 + chunks_per_block);
+  const float inv = 1.0f / static_cast<float>(chunk);
+  for (int64_t c = c0 + warp; c < c1; c += nwarps) {
+    const int64_t t0 = sink + c * chunk;
+    T* o = out + (static_cast<int64_t>(h) * n_mid + c) * hd;
+    for (int jp = 2 * lane; jp < half; jp += 64) {
+      float bc[2], bs[2];
+      rope_cs(ft[jp], static_cast<double>(t0), &bc[0], &bs[0]);
+      rope_cs(ft[jp + 1], static_cast<double>(t0), &bc[1], &bs[1]);
+      float a0[2] = {0.f, 0.f}, a1[2] = {0.f, 0.f};
+      for (int e = 0; e < chunk; ++e) {
+        const T* kr = K + (t0 + e) * ldk + h * hd;
+        float x0[2], x1[2];
+        load2(kr + jp, x0);
+        load2(kr + jp + half, x1);
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+          const float2 r = rot[e * half + jp + q];
+          const float cs = bc[q] * r.x - bs[q] * r.y;
+          const float sn = bs[q] * r.x + bc[q] * r.y;
+          a0[q] = fmaf(x0[q], cs, fmaf(-x1[q], sn, a0[q]));
+          a1[q] = fmaf(x1[q], cs, fmaf(x0[q], sn, a1[q]));
+        }
+      }
+      store2(o + jp, a0[0] * inv, a0[1] * inv);
+      store2(o + jp + half, a1[0] * inv, a1[1] * inv);
+    }
   }
 }
 
@@ -317,6 +387,19 @@ xkv_status landmarks_launch(const void* K, int64_t T, int64_t ldk, int hkv, int 
                             int recent, float theta, void* out, cudaStream_t st) {
   const int64_t n_mid = (T - sink - recent) / chunk;
   if (n_mid <= 0) return XKV_OK;
+  const size_t rot_bytes = static_cast<size_t>(chunk) * (hd / 2) * sizeof(float2);
+  if (hd % 4 == 0 && ldk % 2 == 0 && rot_bytes <= static_cast<size_t>(kLmRotMax)) {
+    const int cpb = 64;
+    dim3 grid(static_cast<unsigned>((n_mid + cpb - 1) / cpb), hkv);
+    if (dt == XKV_BF16)
+      landmarks_rot_kernel<__nv_bfloat16><<<grid, 256, rot_bytes, st>>>(static_cast<const __nv_bfloat16*>(K), ldk, hd,
+                                                                       chunk, sink, n_mid, theta, cpb,
+                                                                       static_cast<__nv_bfloat16*>(out));
+    else
+      landmarks_rot_kernel<float><<<grid, 256, rot_bytes, st>>>(static_cast<const float*>(K), ldk, hd, chunk, sink,
+                                                               n_mid, theta, cpb, static_cast<float*>(out));
+    return cudaPeekAtLastError() == cudaSuccess ? XKV_OK : XKV_ERR_CUDA;
+  }
   const int cpb = 64;
   dim3 grid(static_cast<unsigned>((n_mid + cpb - 1) / cpb), hkv);
   if (dt == XKV_BF16)
