@@ -29,7 +29,13 @@ struct GemmArgs {
   int* status;
 };
 
-constexpr int kGemmStages = 4;
+// ring depth: the projection streams a long K (G d); the reconstruction's K is
+// the rank, so two stages suffice and several CTAs share an SM (one's
+// epilogue overlaps another's MMAs)
+template <int MODE>
+__host__ __device__ constexpr int gemm_stages() {
+  return MODE == kProj ? 4 : 2;
+}
 constexpr int kGemmThreads = 192;
 
 template <int MODE>
@@ -39,7 +45,7 @@ __host__ __device__ constexpr int gemm_stage_bytes() {
 
 template <int MODE>
 inline size_t gemm_smem_bytes() {
-  return 1024 + kGemmStages * gemm_stage_bytes<MODE>() + 64 * 8 + (2 * kGemmStages + 2) * 8 + 16;
+  return 1024 + gemm_stages<MODE>() * gemm_stage_bytes<MODE>() + 64 * 8 + (2 * gemm_stages<MODE>() + 2) * 8 + 16;
 }
 
 template <int MODE>
@@ -49,6 +55,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   constexpr int SB = gemm_stage_bytes<MODE>();
+  constexpr int kGemmStages = gemm_stages<MODE>();
   double* ft = reinterpret_cast<double*>(smem + kGemmStages * SB);
   uint64_t* full = reinterpret_cast<uint64_t*>(ft + 64);
   uint64_t* empty = full + kGemmStages;

@@ -57,6 +57,21 @@ __global__ void __launch_bounds__(256) recon_simt_kernel(const T* __restrict__ A
 // ------------------------------------------------------------ dense decode
 // CTA (split, unit): tokens [t0, t1) of one KV head; 256 rows per pass, one
 // thread scores one row; values are accumulated by (column pair, row group).
+__device__ __forceinline__ void load2(const __nv_bfloat16* p, float* x) {
+  const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(p));
+  x[0] = f.x;
+  x[1] = f.y;
+}
+__device__ __forceinline__ void load2(const float* p, float* x) {
+  const float2 f = *reinterpret_cast<const float2*>(p);
+  x[0] = f.x;
+  x[1] = f.y;
+}
+__device__ __forceinline__ void store2(__nv_bfloat16* p, float a, float b) {
+  *reinterpret_cast<__nv_bfloat162*>(p) = __floats2bfloat162_rn(a, b);
+}
+__device__ __forceinline__ void store2(float* p, float a, float b) { *reinterpret_cast<float2*>(p) = make_float2(a, b); }
+
 template <typename T>
 __global__ void __launch_bounds__(256) dense_partial_kernel(const T* __restrict__ q, const T* __restrict__ K,
                                                             const T* __restrict__ V, int64_t Tn, int Hq, int Hkv,
@@ -92,11 +107,35 @@ __global__ void __launch_bounds__(256) dense_partial_kernel(const T* __restrict_
       const T* kr = K + (static_cast<int64_t>(b) * Tn + tb + tid) * d + h * hd;
 #pragma unroll
       for (int g = 0; g < kMaxGQ; ++g) s[g] = 0.f;
-      for (int j = 0; j < hd; ++j) {
-        const float kv = to_f(kr[j]);
+      if (sizeof(T) == 2 && hd % 8 == 0 && d % 8 == 0) {
+        // the row in 16-byte vectors (8 values per load)
+        for (int j0 = 0; j0 < hd; j0 += 64) {
+          // eight vectors' loads in flight before their use
+          uint4 w[8];
 #pragma unroll
-        for (int g = 0; g < kMaxGQ; ++g)
-          if (g < gq) s[g] = fmaf(qs[g * hd + j], kv, s[g]);
+          for (int v = 0; v < 8; ++v)
+            w[v] = j0 + 8 * v < hd ? *reinterpret_cast<const uint4*>(kr + j0 + 8 * v) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+          for (int v = 0; v < 8; ++v) {
+            if (j0 + 8 * v >= hd) break;
+            const uint32_t ww[4] = {w[v].x, w[v].y, w[v].z, w[v].w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float2 kv = bf2_to_f2(ww[e]);
+              const int j = j0 + 8 * v + 2 * e;
+#pragma unroll
+              for (int g = 0; g < kMaxGQ; ++g)
+                if (g < gq) s[g] = fmaf(qs[g * hd + j], kv.x, fmaf(qs[g * hd + j + 1], kv.y, s[g]));
+            }
+          }
+        }
+      } else {
+        for (int j = 0; j < hd; ++j) {
+          const float kv = to_f(kr[j]);
+#pragma unroll
+          for (int g = 0; g < kMaxGQ; ++g)
+            if (g < gq) s[g] = fmaf(qs[g * hd + j], kv, s[g]);
+        }
       }
     }
 #pragma unroll
@@ -135,7 +174,9 @@ __global__ void __launch_bounds__(256) dense_partial_kernel(const T* __restrict_
     }
     for (int r = rg; r < nr; r += rgroups) {
       const T* vr = V + (static_cast<int64_t>(b) * Tn + tb + r) * d + h * hd + 2 * cp;
-      const float v0 = to_f(vr[0]), v1 = to_f(vr[1]);
+      float vv[2];
+      load2(vr, vv);
+      const float v0 = vv[0], v1 = vv[1];
 #pragma unroll
       for (int g = 0; g < kMaxGQ; ++g) {
         if (g >= gq) break;
@@ -191,20 +232,6 @@ void dense_split(const xkv_dense_params* p, int* splits, int64_t* per) {
 }
 
 // --------------------------------------------------------------- landmarks
-__device__ __forceinline__ void load2(const __nv_bfloat16* p, float* x) {
-  const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(p));
-  x[0] = f.x;
-  x[1] = f.y;
-}
-__device__ __forceinline__ void load2(const float* p, float* x) {
-  const float2 f = *reinterpret_cast<const float2*>(p);
-  x[0] = f.x;
-  x[1] = f.y;
-}
-__device__ __forceinline__ void store2(__nv_bfloat16* p, float a, float b) {
-  *reinterpret_cast<__nv_bfloat162*>(p) = __floats2bfloat162_rn(a, b);
-}
-__device__ __forceinline__ void store2(float* p, float a, float b) { *reinterpret_cast<float2*>(p) = make_float2(a, b); }
 
 template <typename T>
 __global__ void __launch_bounds__(256) landmarks_kernel(const T* __restrict__ K, int64_t ldk, int hd, int chunk,
