@@ -526,6 +526,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-prefill", dest="prefill", action="store_false")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--also", default="qwen7b_128k_b2",
+                    help="comma-separated further workloads measured on one GPU (empty string: none)")
     ap.add_argument("--no-comparison", dest="comparison", action="store_false",
                     help="skip timing the full-reconstruction comparison path")
     args = ap.parse_args()
@@ -544,6 +546,19 @@ def main():
         torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", 0)))
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600))
     res, w = run_cuda(args, rank, world, log)
+    if world == 1 and args.also:
+        # the other shapes the decode path is reported on (same step, same
+        # timing; no prefill, comparison or CPU legs)
+        import copy
+        import torch
+        for name in [x for x in args.also.split(",") if x and x != args.workload]:
+            torch.cuda.empty_cache()
+            a2 = copy.copy(args)
+            a2.workload, a2.prefill, a2.comparison, a2.batch, a2.groups = name, False, False, 0, 0
+            r2, _ = run_cuda(a2, rank, world, log)
+            res.setdefault("other_workloads", {})[name] = {
+                k: r2[k] for k in ("value", "unit", "ms_per_step", "steps", "roofline", "stage_rooflines", "e2e",
+                                   "config", "clocks")}
     if rank == 0 and not args.no_cpu_baseline and world == 1:
         res["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds, log)
     if world > 1:
