@@ -209,6 +209,35 @@ def sr_decode(w, q, A_K, Bt_K, A_V, Bt_V, landmarks, sr_K, sr_V, T: Optional[int
     return out, sel, scores
 
 
+def xk_sr_decode(w, q, A_K, Bt_K, V, landmarks, sr_K, sr_V, T: Optional[int] = None,
+                 sel_in=None, units: Optional[Sequence[int]] = None):
+    """One decode step of the xK-SR mode (fp64): keys as in sr_decode (landmark
+    top-k, rows rebuilt from A_K Bt_K^T with RoPE), values read uncompressed
+    from V [B][T][d] for the same rows.  Returns (out, sel, scores) like
+    sr_decode."""
+    T = T or w.T
+    q, A_K, Bt_K, V, lm, sr_K, sr_V = (_f32(a) for a in (q, A_K, Bt_K, V, landmarks, sr_K, sr_V))
+    B = q.shape[0]
+    if V.shape[-1] != w.d or V.shape[-2] != T:
+        raise ValueError("V must be [B][T][d]")
+    p = _SRParams(B, w.n_q_heads, w.n_kv_heads, w.head_dim, T, A_K.shape[-1], 0,
+                  w.chunk, w.topk, w.sink, w.recent, float(w.rope_theta))
+    n_mid = (T - w.sink - w.recent) // w.chunk
+    out = np.full((B, w.n_q_heads, w.head_dim), np.nan, dtype=np.float64)
+    sel = np.full((B, w.n_kv_heads, w.topk), -1, dtype=np.int32)
+    scores = np.full((B, w.n_kv_heads, n_mid), np.nan, dtype=np.float64)
+    si = None if sel_in is None else np.ascontiguousarray(sel_in, dtype=np.int32)
+    u = None if units is None else np.ascontiguousarray(units, dtype=np.int32)
+    sbk = Bt_K.shape[-2] * Bt_K.shape[-1] if Bt_K.ndim == 3 else 0
+    rc = lib().xo_sr_decode(C.byref(p), _p(q), _p(A_K), C.c_int64(T * A_K.shape[-1]), _p(Bt_K), C.c_int64(sbk),
+                            _p(V), C.c_int64(T * w.d), None, C.c_int64(0), _p(lm), _p(sr_K), _p(sr_V),
+                            None if si is None else _p(si), None if u is None else _p(u),
+                            C.c_int(0 if u is None else u.size), _p(out), _p(sel), _p(scores))
+    if rc != 0:
+        raise ValueError("invalid SR decode shape")
+    return out, sel, scores
+
+
 def ner(Cm: np.ndarray, block: int, rel_tol: float = 1e-9):
     """Per diagonal block: (NER, erank, rank, eigenvalues) of KV-CoRE."""
     Cm = _f64(Cm)

@@ -424,12 +424,16 @@ static int xo_cmp_i32(const void* a, const void* b) {
  *   2. keep the top-k chunks (exact sort; ties -> lower c), ascending by c,
  *      unless sel_in supplies the selection;
  *   3. rebuild rows t of the kept chunks: K_t = RoPE_t(A_K[t] B_K), V_t = A_V[t] B_V
- *      (B_K restricted to head h's hd columns; Bt stores B transposed);
+ *      (B_K restricted to head h's hd columns; Bt stores B transposed).  In the
+ *      xK-SR mode ([xKV-blog] "选择性重建": keys compressed, values kept whole)
+ *      Bt_V is NULL and A_V is the uncompressed value cache [B][T][d]: V_t is
+ *      read as is, head h's hd columns of row t;
  *   4. raw sink rows [0, sink) and recent rows [T - recent, T) (RoPE on K);
  *   5. o_g = softmax(q_g K^T / sqrt(hd)) V over sink, kept and recent rows.
  * Shapes: q [B][Hq][hd]; A_K [B][T][rK] (batch stride sak); Bt_K [B][d][rK]
  * (batch stride sbk; 0 = one Bt for the batch); A_V [B][T][rV] (sav); Bt_V
- * [B][d][rV] (sbv); lm [B][Hkv][n_mid][hd]; srK, srV
+ * [B][d][rV] (sbv), or NULL with A_V [B][T][d] (sav; rank_v unused); lm
+ * [B][Hkv][n_mid][hd]; srK, srV
  * [B][sink+recent][d]; out [B][Hq][hd]; sel_out [B][Hkv][k];
  * scores_out [B][Hkv][n_mid] (optional). */
 XO_EXPORT int xo_sr_decode(const xo_sr_params* p, const float* q, const float* A_K, int64_t sak,
@@ -488,13 +492,17 @@ XO_EXPORT int xo_sr_decode(const xo_sr_params* p, const float* q, const float* A
       for (int e = 0; e < C; ++e, ++row) {
         const int64_t t = p->sink + (int64_t)sel[i] * C + e;
         const float* ak = A_K + b * sak + t * rK;
-        const float* av = A_V + b * sav + t * rV;
         for (int j = 0; j < hd; ++j) {
           const float* bk = Bt_K + b * sbk + (int64_t)(h * hd + j) * rK;
-          const float* bv = Bt_V + b * sbv + (int64_t)(h * hd + j) * rV;
           double sk = 0.0, sv = 0.0;
           for (int a = 0; a < rK; ++a) sk += (double)ak[a] * (double)bk[a];
-          for (int a = 0; a < rV; ++a) sv += (double)av[a] * (double)bv[a];
+          if (Bt_V) {
+            const float* av = A_V + b * sav + t * rV;
+            const float* bv = Bt_V + b * sbv + (int64_t)(h * hd + j) * rV;
+            for (int a = 0; a < rV; ++a) sv += (double)av[a] * (double)bv[a];
+          } else {
+            sv = A_V[b * sav + t * d + h * hd + j];
+          }
           x[j] = sk;
           Vr[row * hd + j] = sv;
         }

@@ -318,6 +318,14 @@ def queries(w: Workload, layer: int) -> np.ndarray:
     return to_storage(q.reshape(w.batch, w.n_q_heads, w.head_dim), w.dtype)
 
 
+def raw_values(w: Workload, layer: int, T: Optional[int] = None) -> np.ndarray:
+    """An uncompressed value cache V ~ N(0,1), [B][T][d] float32 in storage
+    precision (the xK-SR mode keeps values whole)."""
+    T = T or w.T
+    v = normal_chunked(stream_key(w.name, "Vraw", layer, T), w.batch * T * w.d)
+    return to_storage(v.reshape(w.batch, T, w.d), w.dtype)
+
+
 def compressed_cache(w: Workload, layer: int, T: Optional[int] = None):
     """Stand-ins for a compressed layer, drawn directly (decode-only tests).
 

@@ -7,6 +7,11 @@
 * with full rank and every chunk kept, SR on the factors equals dense attention
   over the ORIGINAL cache (exact reconstruction, KQ-SVD page 3.3);
 * a chunk planted to match the query is selected and dominates the output.
+
+xK-SR mode (same explainer: keys compressed, values kept whole):
+* with values equal to the rebuilt A_V Bt_V^T rows it reduces to SR;
+* with every chunk kept it is dense attention over rebuilt keys and raw values;
+* values outside the selected chunks and the window are never read.
 """
 import numpy as np
 import pytest
@@ -130,3 +135,68 @@ def test_rejects_ragged_middle():
     w = W.replace(T=W.T + 3)
     with pytest.raises(ValueError):
         oracle.sr_decode(w, **_inputs(w))
+
+
+# ---------------------------------------------------------------- xK-SR mode
+# Keys compressed and selected as above; values read uncompressed ([B][T][d]).
+
+def _xk_inputs(w=W, layer=0):
+    inp = _inputs(w, layer)
+    V = synth.raw_values(w, layer)
+    rows = list(range(w.sink)) + list(range(w.T - w.recent, w.T))
+    # the raw window is the same cache's rows
+    inp["sr_V"] = np.ascontiguousarray(V[:, rows])
+    x = {k: inp[k] for k in ("q", "A_K", "Bt_K", "landmarks", "sr_K", "sr_V")}
+    x["V"] = V
+    return x, inp
+
+
+def test_xk_values_from_factors_reduce_to_sr():
+    # V = A_V Bt_V^T (one factorisation per sequence, so every head's columns
+    # differ): xK-SR must give SR's output on the same selection
+    inp = _inputs()
+    V = np.stack([oracle.full_reconstruct(inp["A_V"][b], inp["Bt_V"][b], W.n_kv_heads, W.head_dim, False,
+                                          W.rope_theta) for b in range(W.batch)]).astype(np.float32)
+    x = {k: inp[k] for k in ("q", "A_K", "Bt_K", "landmarks", "sr_K", "sr_V")}
+    out_x, sel_x, sc_x = oracle.xk_sr_decode(W, V=V, **x)
+    out_s, sel_s, sc_s = oracle.sr_decode(W, **inp)
+    assert np.array_equal(sel_x, sel_s) and np.array_equal(sc_x, sc_s)
+    # V went through float32 once: agreement to that rounding
+    assert np.abs(out_x - out_s).max() < 1e-6
+
+
+def test_xk_all_chunks_equals_dense_over_rebuilt_keys_and_raw_values():
+    w = W.replace(topk=W.n_mid)
+    x, inp = _xk_inputs(w)
+    out, sel, _ = oracle.xk_sr_decode(w, **x)
+    assert np.array_equal(sel[0, 0], np.arange(w.n_mid))
+    Km = np.stack([oracle.full_reconstruct(inp["A_K"][b], inp["Bt_K"][b], w.n_kv_heads, w.head_dim, True,
+                                           w.rope_theta) for b in range(w.batch)])
+    K, V = _dense_cache(w, inp, Km, x["V"].astype(np.float64))
+    ref = oracle.dense_decode(inp["q"], K, V, w.n_kv_heads)
+    assert np.abs(out - ref).max() < 1e-6
+
+
+def test_xk_reads_only_selected_rows_and_window():
+    x, _ = _xk_inputs()
+    out, sel, _ = oracle.xk_sr_decode(W, **x)
+    b, h = 0, 1
+    hd, C = W.head_dim, W.chunk
+    chosen = set(sel[b, h].tolist())
+    skipped = next(c for c in range(W.n_mid) if c not in chosen)
+    kept = sel[b, h, 0]
+    # a middle chunk that was not selected: its values are never read
+    V2 = x["V"].copy()
+    t0 = W.sink + skipped * C
+    V2[b, t0:t0 + C, h * hd:(h + 1) * hd] += 100.0
+    out2, _, _ = oracle.xk_sr_decode(W, **{**x, "V": V2})
+    assert np.array_equal(out2, out)
+    # one row of a selected chunk: the unit's outputs move, the others do not
+    V3 = x["V"].copy()
+    V3[b, W.sink + kept * C, h * hd:(h + 1) * hd] += 100.0
+    out3, _, _ = oracle.xk_sr_decode(W, **{**x, "V": V3})
+    rows = slice(h * W.gq, (h + 1) * W.gq)
+    assert np.abs(out3[b, rows] - out[b, rows]).max() > 1e-6
+    mask = np.ones(out.shape[:2], dtype=bool)
+    mask[b, rows] = False
+    assert np.array_equal(out3[mask], out[mask])
