@@ -38,6 +38,7 @@ EXPORTS = (
     "xkv_build_landmarks",
     "xkv_sr_workspace_size", "xkv_sr_attention_decode",
     "xkv_sr_attention_decode_noalloc",
+    "xkv_xk_sr_workspace_size", "xkv_xk_sr_attention_decode",
     "xkv_sr_profile_enable", "xkv_sr_profile_read",
     "xkv_full_reconstruct",
     "xkv_dense_workspace_size", "xkv_dense_attention_decode",
@@ -88,6 +89,9 @@ def _load():
                                               vp]),
         "xkv_sr_attention_decode_noalloc": (C.c_int, [C.POINTER(SRParams), vp, vp, vp, vp, vp, vp, vp, vp, vp, vp,
                                                       vp]),
+        "xkv_xk_sr_workspace_size": (C.c_int, [C.POINTER(SRParams), C.POINTER(sz)]),
+        "xkv_xk_sr_attention_decode": (C.c_int, [C.POINTER(SRParams), vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz,
+                                                 vp]),
         "xkv_sr_profile_enable": (C.c_int, [C.c_int]),
         "xkv_sr_profile_read": (C.c_int, [C.POINTER(C.c_float)]),
         "xkv_full_reconstruct": (C.c_int, [vp, vp, i64, C.c_int, C.c_int, C.c_int, C.c_int, C.c_int, C.c_float,
@@ -248,6 +252,32 @@ def xkv_sr_attention_decode_noalloc(p: SRParams, q, A_K, Bt_K, A_V, Bt_V, landma
     _check(lib.xkv_sr_attention_decode_noalloc(C.byref(p), _ptr(q), _ptr(A_K), _ptr(Bt_K), _ptr(A_V), _ptr(Bt_V),
                                                _ptr(landmarks), _ptr(sr_K), _ptr(sr_V), _ptr(out), _ptr(sel_out),
                                                _stream(stream)), "xkv_sr_attention_decode_noalloc")
+
+
+def xk_sr_params(batch, n_q_heads, n_kv_heads, head_dim, T, rank_k, chunk, topk, sink, recent, rope_theta,
+                 dtype: torch.dtype, a_k_batch_stride=None, v_batch_stride=None, bt_k_batch_stride=None) -> SRParams:
+    """Parameters of the xK-SR mode: keys as in sr_params, values an uncompressed
+    [B][T][d] cache (batch stride defaults to T d)."""
+    d = n_kv_heads * head_dim
+    return SRParams(batch, n_q_heads, n_kv_heads, head_dim, T, rank_k, head_dim, chunk, topk, sink, recent,
+                    float(rope_theta), dtype_code(dtype),
+                    T * rank_k if a_k_batch_stride is None else a_k_batch_stride,
+                    T * d if v_batch_stride is None else v_batch_stride,
+                    d * rank_k if bt_k_batch_stride is None else bt_k_batch_stride, 0)
+
+
+def xkv_xk_sr_workspace_size(p: SRParams) -> int:
+    return _wsize(lib.xkv_xk_sr_workspace_size, C.byref(p))
+
+
+def xkv_xk_sr_attention_decode(p: SRParams, q, A_K, Bt_K, V, landmarks, sr_K, sr_V, out, sel_out=None, ws=None,
+                               stream=None):
+    """One xK-SR decode step of one layer (values read from the uncompressed V
+    [B][T][d]); writes out [B][Hq][hd] f32 (and sel_out)."""
+    ws = ws if ws is not None else workspace(xkv_xk_sr_workspace_size(p), q.device)
+    _check(lib.xkv_xk_sr_attention_decode(C.byref(p), _ptr(q), _ptr(A_K), _ptr(Bt_K), _ptr(V), _ptr(landmarks),
+                                          _ptr(sr_K), _ptr(sr_V), _ptr(out), _ptr(sel_out), _ptr(ws), ws.numel(),
+                                          _stream(stream)), "xkv_xk_sr_attention_decode")
 
 
 def xkv_sr_profile_enable(enable: bool = True) -> None:

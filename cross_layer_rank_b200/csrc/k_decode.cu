@@ -542,6 +542,7 @@ struct AttendArgs {
   int64_t T;
   int64_t sbk, sbv;  // batch strides of Bt_K / Bt_V (elements, 0 = shared)
   int Hq, Hkv, k, sink, recent, rK, rV;
+  int v_raw;  // values uncompressed (xK-SR): the value operand is V [B][T][d], head h at column h hd, rV = hd
   int tiles_per_unit, n_tiles, ctas, max_units;
   int slot_floats;
   float theta;
@@ -626,7 +627,7 @@ __device__ void merge_unit(const T* __restrict__ BtV, const float* __restrict__ 
   const int tpu = args.tiles_per_unit;
   const int rV = args.rV;
   // bf16 rows with 8-column groups: U stored as [g][e][v] for column 8v + e
-  const bool vec = sizeof(T) == 2 && rV % 8 == 0 && args.sbv % 8 == 0;
+  const bool vec = !args.v_raw && sizeof(T) == 2 && rV % 8 == 0 && args.sbv % 8 == 0;
   const int nv = rV / 8;
   float* Us = smf;                              // [gq][rV] (permuted when vec)
   float* ml = Us + gq * rV;                     // [slots][16] partial m, l
@@ -711,7 +712,7 @@ __device__ void merge_unit(const T* __restrict__ BtV, const float* __restrict__ 
         }
       }
       if (vec) {
-        const int c = 4 * i4 - g * rV, vv = c >> 3, e = c & 7;
+        const int c = 4 * i4 - g * rV, vv = c >> 3, e = c & 7;  // rV % 8 == 0: no float4 spans two heads
         float* dst = Us + (g * 8 + e) * nv + vv;
         dst[0] = acc.x;
         dst[nv] = acc.y;
@@ -721,9 +722,24 @@ __device__ void merge_unit(const T* __restrict__ BtV, const float* __restrict__ 
         reinterpret_cast<float4*>(Us)[i4] = acc;
       }
     }
+    // the last gq rV mod 4 entries (never in the permuted layout: there rV % 8 == 0)
+    for (int i = 4 * n4 + tid; i < gq * rV; i += blockDim.x) {
+      const int g = i / rV;
+      float acc = 0.f;
+      for (int c = 0; c < nslots; ++c) acc = fmaf(__ldcg(slot_ptr(fc + c) + 16 + i), sc[c * kMaxGQ + g], acc);
+      Us[i] = acc;
+    }
   }
   cp_async_wait_all();
   __syncthreads();
+  if (args.v_raw) {
+    // values were not compressed: U_g is already the kept rows' value sum
+    for (int i = tid; i < gq * ncols; i += blockDim.x) {
+      const int g = i / ncols, j = j0 + i % ncols;
+      out[(static_cast<int64_t>(b) * args.Hq + h * gq + g) * hd + j] = fmaf(fw[g], wo[i], Us[g * rV + j]) * Lg[g];
+    }
+    return;
+  }
   // ---- E
   for (int jb = j0 + warp * kCombineColsPerWarp; jb < j1; jb += nwarps * kCombineColsPerWarp) {
     const int ncol = min(kCombineColsPerWarp, j1 - jb);
@@ -930,6 +946,8 @@ __global__ void __launch_bounds__(kAttendThreads, 1)
       for (int x = tb; x < te && !*abort_flag; ++x) {
         const int u = x / tpu, ti = x % tpu;
         const int b = u / args.Hkv;
+        // first 64-column atom of the value rows: head h's columns when values are uncompressed
+        const int vz = args.v_raw ? (u % args.Hkv) * NAV : 0;
         const int nch = min(kTileChunks, k - ti * kTileChunks);
         const int32_t* su = args.sel + static_cast<int64_t>(u) * k + ti * kTileChunks;
         int rows[kTileChunks];
@@ -941,7 +959,7 @@ __global__ void __launch_bounds__(kAttendThreads, 1)
           mbar_arrive_expect_tx(&vfull[slot], 2 * NAV * 1024);
           for (int c2 = 0; c2 < 2; ++c2) {
             const int ch = (2 * v + c2 < nch) ? 2 * v + c2 : 2 * v;
-            tma_load_4d(Vs + slot * 16384 + c2 * NAVp * 1024, &mapAV, &vfull[slot], 0, rows[ch], 0, b);
+            tma_load_4d(Vs + slot * 16384 + c2 * NAVp * 1024, &mapAV, &vfull[slot], 0, rows[ch], vz, b);
           }
         }
       }
@@ -1313,13 +1331,16 @@ __global__ void __launch_bounds__(256) sr_attend_simt_kernel(const T* __restrict
         ms[g] = mx;
       }
       __syncthreads();
+      // value rows: A_V [t][rV], or head h's columns of V [t][d] when uncompressed
+      const int64_t vld = args.v_raw ? d : args.rV;
+      const T* avb = AV + b * sav + (args.v_raw ? h * hd : 0);
       for (int i = tid; i < gq * args.rV; i += blockDim.x) {
         const int g = i / args.rV, c = i % args.rV;
         float acc = us[i] * al[g];
         for (int r = 0; r < nr; ++r) {
           const int rr = rb + r;
           const int64_t t = args.sink + static_cast<int64_t>(args.sel[static_cast<int64_t>(u) * k + ti * kTileChunks + rr / chunk]) * chunk + rr % chunk;
-          acc = fmaf(ps[r * gq + g], to_f(AV[b * sav + t * args.rV + c]), acc);
+          acc = fmaf(ps[r * gq + g], to_f(avb[t * vld + c]), acc);
         }
         us[i] = acc;
       }
@@ -1333,7 +1354,6 @@ __global__ void __launch_bounds__(256) sr_attend_simt_kernel(const T* __restrict
       if (tid < gq) { slot[tid] = ms[tid]; slot[8 + tid] = ls[tid]; }
     }
   }
-  (void)d;
 }
 
 
@@ -1374,7 +1394,8 @@ xkv_status sr_plan(const xkv_sr_params* p, SRPlan* plan) {
     if (te > tb) mx = std::max(mx, (te - 1) / plan->tiles_per_unit - tb / plan->tiles_per_unit + 1);
   }
   plan->max_units_per_cta = mx;
-  plan->slot_floats = 16 + static_cast<size_t>(std::max(gq, 1)) * p->rank_v;
+  // a multiple of 4 floats, so that every slot's float4 reads stay aligned
+  plan->slot_floats = (16 + static_cast<size_t>(std::max(gq, 1)) * p->rank_v + 3) & ~size_t(3);
   size_t off = 0;
   plan->off_scores = off;  // rows padded to a multiple of 4 floats
   off = align_up(off + static_cast<size_t>(plan->units) * ((n_mid + 3) & ~int64_t(3)) * 4);
@@ -1479,7 +1500,9 @@ static xkv_status sr_launch_t(const xkv_sr_params* p, const SRPlan& plan, const 
   a.status = device_status_ptr();
   a.T = p->T;
   a.sbk = p->bt_k_batch_stride;
-  a.sbv = p->bt_v_batch_stride;
+  // Bt_V absent: the xK-SR mode, A_V is the uncompressed V [B][T][d] and rank_v = hd
+  a.v_raw = Bt_V == nullptr ? 1 : 0;
+  a.sbv = a.v_raw ? 0 : p->bt_v_batch_stride;
   a.Hq = p->n_q_heads;
   a.Hkv = p->n_kv_heads;
   a.k = p->topk;
@@ -1518,10 +1541,12 @@ static xkv_status sr_launch_t(const xkv_sr_params* p, const SRPlan& plan, const 
         return XKV_ERR_CUDA;
     }
     {
-      // (64 columns, token rows, atoms, batch): one box = 8 rows x the full rank
-      const uint64_t dims[4] = {64, static_cast<uint64_t>(p->T), static_cast<uint64_t>(p->rank_v / 64),
+      // (64 columns, token rows, atoms, batch): one box = 8 rows x the full rank;
+      // uncompressed values: rows of d columns, one box = 8 rows x head h's hd columns
+      const int vcols = a.v_raw ? d : p->rank_v;
+      const uint64_t dims[4] = {64, static_cast<uint64_t>(p->T), static_cast<uint64_t>(vcols / 64),
                                 static_cast<uint64_t>(p->batch)};
-      const uint64_t str[3] = {static_cast<uint64_t>(p->rank_v) * 2, 128, static_cast<uint64_t>(p->a_v_batch_stride) * 2};
+      const uint64_t str[3] = {static_cast<uint64_t>(vcols) * 2, 128, static_cast<uint64_t>(p->a_v_batch_stride) * 2};
       const uint32_t box[4] = {64, 8, static_cast<uint32_t>(p->rank_v / 64), 1};
       if (!make_tmap(&mAV, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, A_V, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B))
         return XKV_ERR_CUDA;

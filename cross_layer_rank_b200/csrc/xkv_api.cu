@@ -301,6 +301,49 @@ xkv_status xkv_sr_attention_decode_noalloc(const xkv_sr_params* p, const void* q
                    static_cast<cudaStream_t>(stream));
 }
 
+// ------------------------------------------- xK-SR decode (values uncompressed)
+// The SR kernels with the uncompressed value cache as their value operand:
+// rank_v = head_dim, no Bt_V, A_V = V [B][T][d] (head h at columns h hd).
+static xkv_status xk_params(const xkv_sr_params* p, xkv_sr_params* pv) {
+  if (!p) return XKV_ERR_INVALID_ARG;
+  *pv = *p;
+  pv->rank_v = p->head_dim;
+  pv->bt_v_batch_stride = 0;
+  const xkv_status s = check_sr(pv);
+  if (s != XKV_OK) return s;
+  if (p->a_v_batch_stride < p->T * p->n_kv_heads * p->head_dim) return XKV_ERR_INVALID_ARG;
+  return XKV_OK;
+}
+
+xkv_status xkv_xk_sr_workspace_size(const xkv_sr_params* p, size_t* bytes) {
+  if (!bytes) return XKV_ERR_INVALID_ARG;
+  xkv_sr_params pv;
+  const xkv_status s = xk_params(p, &pv);
+  if (s != XKV_OK) return s;
+  SRPlan plan;
+  sr_plan(&pv, &plan);
+  *bytes = plan.bytes;
+  return XKV_OK;
+}
+
+xkv_status xkv_xk_sr_attention_decode(const xkv_sr_params* p, const void* q, const void* A_K, const void* Bt_K,
+                                      const void* V, const void* landmarks, const void* sr_K, const void* sr_V,
+                                      float* out, int32_t* sel_out, void* workspace, size_t ws_bytes, void* stream) {
+  xkv_sr_params pv;
+  const xkv_status s = xk_params(p, &pv);
+  if (s != XKV_OK) return s;
+  const void* ptrs[] = {q, A_K, Bt_K, V, landmarks, out};
+  for (const void* x : ptrs)
+    if (!x || !aligned16(x)) return XKV_ERR_INVALID_ARG;
+  if (p->sink + p->recent > 0 && (!sr_K || !sr_V || !aligned16(sr_K) || !aligned16(sr_V))) return XKV_ERR_INVALID_ARG;
+  if (sel_out && !aligned16(sel_out)) return XKV_ERR_INVALID_ARG;
+  SRPlan plan;
+  sr_plan(&pv, &plan);
+  if (!workspace || ws_bytes < plan.bytes || !aligned256(workspace)) return XKV_ERR_WORKSPACE;
+  return sr_launch(&pv, plan, q, A_K, Bt_K, V, nullptr, landmarks, sr_K, sr_V, out, sel_out, workspace,
+                   static_cast<cudaStream_t>(stream));
+}
+
 // --------------------------------------------------- full reconstruction
 xkv_status xkv_full_reconstruct(const void* A, const void* Bt, int64_t T, int rank, int d, int n_kv_heads,
                                 int head_dim, int apply_rope, float rope_theta, xkv_dtype dt, void* out, void* stream) {

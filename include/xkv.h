@@ -187,6 +187,22 @@ XKV_API xkv_status xkv_sr_attention_decode_noalloc(const xkv_sr_params* p, const
                                            const void* landmarks, const void* sr_K, const void* sr_V,
                                            float* out, int32_t* sel_out, void* stream);
 
+/* One decode step of the xK-SR mode ([xKV-blog] "选择性重建": only the keys are
+ * compressed; the values stay whole).  Chunk scores, the exact top-k and the
+ * key rows K_t = RoPE_t(A_K[b][t] Bt_K[h hd : (h+1) hd]^T) are those of
+ * xkv_sr_attention_decode; the value of a kept row t is read from the
+ * uncompressed cache, V_t = V[b][t][h hd : (h+1) hd].
+ *   V         : [B][T][d] in p->dtype, 16-byte aligned; p->a_v_batch_stride is its
+ *               batch stride in elements (>= T d).  p->rank_v and
+ *               p->bt_v_batch_stride are ignored.
+ *   workspace : at least xkv_xk_sr_workspace_size bytes, 256-byte aligned.
+ * Every other argument, layout and error is that of xkv_sr_attention_decode. */
+XKV_API xkv_status xkv_xk_sr_workspace_size(const xkv_sr_params* p, size_t* bytes);
+XKV_API xkv_status xkv_xk_sr_attention_decode(const xkv_sr_params* p, const void* q, const void* A_K,
+                                              const void* Bt_K, const void* V, const void* landmarks,
+                                              const void* sr_K, const void* sr_V, float* out, int32_t* sel_out,
+                                              void* workspace, size_t ws_bytes, void* stream);
+
 /* Stage timing (measurement aid; the method has no counterpart).  While
  * enabled, every xkv_sr_attention_decode call records CUDA events on its
  * stream around its four launches: chunk scores, top-k (+ raw window

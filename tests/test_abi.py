@@ -78,6 +78,33 @@ def test_sr_rejects_null_and_misaligned_pointers_and_small_workspace(xkv):
     assert xkv.lib.xkv_sr_attention_decode(C.byref(p), *args, None, fake, 16, None) == xkv.XKV_ERR_WORKSPACE
 
 
+def test_xk_sr_validation(xkv):
+    import torch
+    T, d = 1024, 2 * 64
+
+    def xk(**kw):
+        base = dict(batch=1, n_q_heads=8, n_kv_heads=2, head_dim=64, T=T, rank_k=64, chunk=8, topk=16, sink=8,
+                    recent=32, rope_theta=500000.0, dtype=torch.float32)
+        base.update(kw)
+        return xkv.xk_sr_params(**base)
+
+    n = C.c_size_t(0)
+    p = xk()
+    p.rank_v = 0  # ignored: the value rows are the uncompressed cache
+    assert xkv.lib.xkv_xk_sr_workspace_size(C.byref(p), C.byref(n)) == xkv.XKV_OK and n.value > 0
+    # a value batch stride below T d
+    assert xkv.lib.xkv_xk_sr_workspace_size(C.byref(xk(v_batch_stride=T * 64)), C.byref(n)) == \
+        xkv.XKV_ERR_INVALID_ARG
+    assert xkv.lib.xkv_xk_sr_workspace_size(C.byref(xk(topk=124)), C.byref(n)) == xkv.XKV_ERR_INVALID_ARG
+    fake = C.c_void_p(1 << 20)
+    f = xkv.lib.xkv_xk_sr_attention_decode
+    assert f(C.byref(p), fake, fake, fake, None, fake, fake, fake, fake, None, fake, 1 << 30, None) == \
+        xkv.XKV_ERR_INVALID_ARG  # no V
+    assert f(C.byref(p), fake, fake, fake, fake, fake, fake, fake, fake, None, fake, 16, None) == \
+        xkv.XKV_ERR_WORKSPACE
+    assert T * d == p.a_v_batch_stride
+
+
 def test_compress_and_gram_validation(xkv):
     n = C.c_size_t(0)
     assert xkv.lib.xkv_compress_workspace_size(4, 1024, 128, 64, 64, 8192, xkv.XKV_F32, C.byref(n)) == xkv.XKV_OK

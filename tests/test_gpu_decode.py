@@ -98,6 +98,13 @@ def test_sr_topk_tied_boundary_bucket(xkv, n_tied):
     assert np.abs(host(out_g) - ref).max() <= 1e-2
 
 
+def test_sr_bf16_odd_value_rank(xkv):
+    # value rank 51 with a GQA group of 3: partial slots of 16 + 153 floats are
+    # padded to a multiple of 4 and the merge folds the last entry on its own
+    w = synth.Workload("sr_bf16_odd_rank", 1, 4, 4, 2, 128, 6, 8 + 32 + 8 * 90, 96, 0.8, 64, 51, topk=19)
+    _parity(xkv, w)
+
+
 def test_sr_f32_general_shape(xkv):
     # f32, hd 64, chunk 4, odd ranks: the CUDA-core path
     w = synth.Workload("sr_f32_general", 2, 4, 4, 3, 64, 6, 5 + 7 + 4 * 90, 48, 0.8, 48, 80, chunk=4, topk=23,
