@@ -68,6 +68,15 @@ def attend_bytes_per_unit(w) -> int:
             + w.gq * w.head_dim * el)
 
 
+def xk_attend_bytes_per_unit(w) -> int:
+    """The attend stage's algorithmic bytes per unit in the xK-SR mode: the
+    selected A_K rows, the selected rows' hd value columns of the head, the
+    Bt_K head slice and the group's queries."""
+    el = 2 if w.dtype == "bf16" else 4
+    return (w.topk * w.chunk * (w.rank_k + w.head_dim) * el + w.rank_k * w.head_dim * el
+            + w.gq * w.head_dim * el)
+
+
 def stage_rooflines(w, stage_ms, peak_gbs):
     """Achieved GB/s of each decode launch of one layer call (whole batch)
     against the HBM peak, from its algorithmic bytes:
@@ -363,6 +372,11 @@ def run_cuda(args, rank, world, log):
     assert xkv.get_device_status(stream) == 0
     clocks = clk.summary()
     comparison = measure_full_reconstruction(xkv, w, model, device, stream, call_ms) if args.comparison else None
+    xk = None
+    if args.xk and world == 1:
+        del graph, g1
+        torch.cuda.empty_cache()
+        xk = measure_xk_sr(xkv, w, model, device, stream, L, args.steps, args.warmup, _peaks()[0])
 
     ms_total, e2e_ms = max_over_ranks([ms_total, e2e_ms], world, device)
     ms_step = ms_total / args.steps
@@ -419,6 +433,8 @@ def run_cuda(args, rank, world, log):
     }
     if comparison is not None:
         res["comparison"] = comparison
+    if xk is not None:
+        res["xk_sr"] = xk
     if args.prefill:
         cm = prefill["compress_ms"]
         res["prefill"] = {"compress_group_ms_median": round(statistics.median(cm), 3), "groups_compressed": len(cm),
@@ -429,6 +445,69 @@ def run_cuda(args, rank, world, log):
                           "gram_tflops": round(gram_flops / (gram_ms / 1e3) / 1e12, 1),
                           "gram_frac_of_bf16_peak": round(gram_flops / (gram_ms / 1e3) / 1e12 / bf16_peak, 4)}
     return res, w
+
+
+def measure_xk_sr(xkv, w, model, device, stream, L, steps, warmup, peak_gbs):
+    """The xK-SR mode on the same compressed keys, landmarks and queries: values
+    read from an uncompressed [B][T][d] cache per layer (seeded normals, bf16).
+    Device time of `steps` replays of one CUDA graph of L layer calls, and the
+    attend launch's achieved GB/s from the library's stage events."""
+    import torch
+    bf = torch.bfloat16
+    Vs = []
+    for l in range(L):
+        Vs.append(synth.normal_torch(synth.stream_key(w.name, "Vraw", l, w.T), w.batch * w.T * w.d, device,
+                                     bf).view(w.batch, w.T, w.d))
+        torch.cuda.empty_cache()
+    p = xkv.xk_sr_params(w.batch, w.n_q_heads, w.n_kv_heads, w.head_dim, w.T, w.rank_k, w.chunk, w.topk, w.sink,
+                         w.recent, w.rope_theta, bf)
+    ws = xkv.workspace(xkv.xkv_xk_sr_workspace_size(p), device)
+    outs = [torch.empty((w.batch, w.n_q_heads, w.head_dim), dtype=torch.float32, device=device) for _ in range(L)]
+
+    def call(l):
+        xkv.xkv_xk_sr_attention_decode(p, model["q"][l], model["A_K"][l], model["Bt_K"][l], Vs[l], model["lm"][l],
+                                       model["srK"][l], model["srV"][l], outs[l], None, ws, stream)
+
+    with torch.cuda.stream(stream):
+        for l in range(L):
+            call(l)
+    stream.synchronize()
+    assert xkv.get_device_status(stream) == 0
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        for l in range(L):
+            call(l)
+    with torch.cuda.stream(stream):
+        for _ in range(warmup):
+            graph.replay()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(steps):
+            graph.replay()
+        e1.record(stream)
+        e1.synchronize()
+    ms_step = e0.elapsed_time(e1) / steps
+    xkv.xkv_sr_profile_enable(True)
+    stages = []
+    with torch.cuda.stream(stream):
+        for i in range(2 * L):
+            call(i % L)
+            stages.append(xkv.xkv_sr_profile_read())
+    xkv.xkv_sr_profile_enable(False)
+    assert xkv.get_device_status(stream) == 0
+    st = [statistics.median(s_[j] for s_ in stages) for j in range(4)]
+    bytes_attend = xk_attend_bytes_per_unit(w) * w.batch * w.n_kv_heads
+    gbs = bytes_attend / (st[2] / 1e3) / 1e9
+    del graph, Vs
+    torch.cuda.empty_cache()
+    return {"path": "xkv_xk_sr_attention_decode (keys compressed, values uncompressed in HBM)",
+            "value": round(w.batch / (ms_step / 1e3), 2), "unit": "tokens/s", "ms_per_step": round(ms_step, 4),
+            "stages_ms": {"score": round(st[0], 5), "topk_window": round(st[1], 5), "attend": round(st[2], 5),
+                          "combine": round(st[3], 5)},
+            "attend_roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peak_gbs, "unit": "GB/s",
+                                "frac": round(gbs / peak_gbs, 4), "bytes_per_launch": bytes_attend},
+            "value_cache_gb": round(L * w.batch * w.T * w.d * 2 / 1e9, 2)}
 
 
 def measure_full_reconstruction(xkv, w, model, device, stream, sr_call_ms):
@@ -526,6 +605,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-prefill", dest="prefill", action="store_false")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--no-xk", dest="xk", action="store_false",
+                    help="skip the xK-SR measurement (values uncompressed; one GPU only)")
     ap.add_argument("--also", default="qwen7b_128k_b2",
                     help="comma-separated further workloads measured on one GPU (empty string: none)")
     ap.add_argument("--no-comparison", dest="comparison", action="store_false",
@@ -554,7 +635,7 @@ def main():
         for name in [x for x in args.also.split(",") if x and x != args.workload]:
             torch.cuda.empty_cache()
             a2 = copy.copy(args)
-            a2.workload, a2.prefill, a2.comparison, a2.batch, a2.groups = name, False, False, 0, 0
+            a2.workload, a2.prefill, a2.comparison, a2.xk, a2.batch, a2.groups = name, False, False, False, 0, 0
             r2, _ = run_cuda(a2, rank, world, log)
             res.setdefault("other_workloads", {})[name] = {
                 k: r2[k] for k in ("value", "unit", "ms_per_step", "steps", "roofline", "stage_rooflines", "e2e",
