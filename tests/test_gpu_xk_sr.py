@@ -6,8 +6,9 @@ The selection rule and the tolerances are those of the SR parity tests: the
 top-k set equals the exact one except near-ties (1e-3 relative of the k-th
 score); outputs within 1e-2 max-abs (bf16 storage) or 2e-4 (f32) of the oracle
 run on the GPU's own selection.  Shapes: a small bf16 case on the tensor-core
-path with a ragged last tile, the f32 CUDA-core path with odd sizes, and one
-layer of the Llama-3.1-8B group at 16K.
+path with a ragged last tile, the f32 CUDA-core path with odd sizes, no raw
+window, one layer of the Llama-3.1-8B group at 16K and one layer of the
+Qwen2.5-7B shape at 128K, batch 2 (sampled units).
 """
 import numpy as np
 import pytest
@@ -45,14 +46,18 @@ def _run_xk(xkv, w, x, V):
     return host(out), sel.cpu().numpy()
 
 
-def _xk_parity(xkv, w, tol=1e-2):
-    x, V = _xk_inputs(w)
+def _xk_parity(xkv, w, tol=1e-2, layer=0, units=None):
+    x, V = _xk_inputs(w, layer)
     out_g, sel_g = _run_xk(xkv, w, x, V)
-    _, _, scores = oracle.xk_sr_decode(w, V=V, **x)
-    check_selection(sel_g, scores, w.topk)
-    ref, _, _ = oracle.xk_sr_decode(w, V=V, sel_in=sel_g, **x)
-    assert np.isfinite(out_g).all()
-    err = np.abs(out_g - ref).max()
+    _, _, scores = oracle.xk_sr_decode(w, V=V, units=units, **x)
+    check_selection(sel_g, scores, w.topk, units=units)
+    ref, _, _ = oracle.xk_sr_decode(w, V=V, sel_in=sel_g, units=units, **x)
+    rows = np.zeros(out_g.shape[:2], dtype=bool)
+    for u in (units if units is not None else range(x["q"].shape[0] * w.n_kv_heads)):
+        b, h = divmod(u, w.n_kv_heads)
+        rows[b, h * w.gq:(h + 1) * w.gq] = True
+    assert np.isfinite(out_g[rows]).all()
+    err = np.abs(out_g[rows] - ref[rows]).max()
     assert err <= tol, err
     return err
 
@@ -71,3 +76,12 @@ def test_xk_sr_f32_general_shape(xkv):
 def test_xk_sr_full_size_llama_group_16k(xkv):
     _xk_parity(xkv, synth.WORKLOADS["llama_group_16k"])
 
+
+def test_xk_sr_without_sink_or_recent_window(xkv):
+    w = synth.Workload("xk_nowin", 2, 4, 4, 2, 128, 8, 8 * 150, 96, 0.8, 128, 128, topk=37, sink=0, recent=0)
+    _xk_parity(xkv, w)
+
+
+def test_xk_sr_full_size_qwen7b_128k_batch2_layer(xkv):
+    # values whole: 2 x 131072 x 512 bf16 (268 MB) for the layer
+    _xk_parity(xkv, synth.WORKLOADS["qwen7b_128k_b2"], layer=3, units=[0, 3, 5, 6])
