@@ -688,9 +688,10 @@ __device__ void merge_unit(const T* __restrict__ BtV, const float* __restrict__ 
     }
   }
   __syncthreads();
-  // ---- D (float4 over rank columns, 8 slots' loads in flight)
+  // ---- D (float4 over rank columns, 16 slots' loads in flight; a float4
+  // must not span two heads, whose slot factors differ: rV % 4 == 0)
   {
-    const int n4 = gq * rV / 4;
+    const int n4 = rV % 4 == 0 ? gq * rV / 4 : 0;
     for (int i4 = tid; i4 < n4; i4 += blockDim.x) {
       const int g = (4 * i4) / rV;
       float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -722,7 +723,7 @@ __device__ void merge_unit(const T* __restrict__ BtV, const float* __restrict__ 
         reinterpret_cast<float4*>(Us)[i4] = acc;
       }
     }
-    // the last gq rV mod 4 entries (never in the permuted layout: there rV % 8 == 0)
+    // other value ranks entry by entry (never the permuted layout: there rV % 8 == 0)
     for (int i = 4 * n4 + tid; i < gq * rV; i += blockDim.x) {
       const int g = i / rV;
       float acc = 0.f;
