@@ -249,7 +249,23 @@ def measure_gram(xkv, w, device):
     e1.synchronize()
     ms = e0.elapsed_time(e1) / reps
     flops = n * (n + 1) * w.T  # unique entries of the symmetric product, 2 T flops each
-    return ms, flops
+    # KV-CoRE's NER and the energy rank of every layer of the group, from this
+    # Gram (the diagonal d x d blocks; scale-invariant, so the repeated sums do)
+    ner = torch.empty(w.group, dtype=torch.float32, device=device)
+    wsn = xkv.workspace(xkv.xkv_ner_workspace_size(n, w.d), device)
+    spectra = {}
+    for name, fn in (("ner", lambda: xkv.xkv_ner(C, w.d, ner, ws=wsn)),
+                     ("energy_rank_95", lambda: xkv.xkv_energy_rank(C, w.d, 0.95, ws=wsn))):
+        fn()
+        torch.cuda.synchronize()
+        e0.record()
+        fn()
+        e1.record()
+        e1.synchronize()
+        spectra[name + "_ms"] = round(e0.elapsed_time(e1), 3)
+    assert xkv.get_device_status() == 0
+    spectra["blocks"] = f"{w.group} x {w.d} x {w.d}"
+    return ms, flops, spectra
 
 
 # --------------------------------------------------------- multi-rank
@@ -287,7 +303,7 @@ def run_cuda(args, rank, world, log):
     L = n_groups * w.group
     bf = torch.bfloat16
     model, prefill = build_model(xkv, w, device, n_groups, log)
-    gram_ms, gram_flops = measure_gram(xkv, w, device) if args.prefill else (None, None)
+    gram_ms, gram_flops, spectra = measure_gram(xkv, w, device) if args.prefill else (None, None, None)
 
     p = xkv.sr_params(w.batch, w.n_q_heads, w.n_kv_heads, w.head_dim, w.T, w.rank_k, w.rank_v, w.chunk, w.topk,
                       w.sink, w.recent, w.rope_theta, bf)
@@ -443,7 +459,8 @@ def run_cuda(args, rank, world, log):
                                                                                1e3) / 1e9 / hbm_gbs_peak, 4),
                           "gram_ms": round(gram_ms, 4),
                           "gram_tflops": round(gram_flops / (gram_ms / 1e3) / 1e12, 1),
-                          "gram_frac_of_bf16_peak": round(gram_flops / (gram_ms / 1e3) / 1e12 / bf16_peak, 4)}
+                          "gram_frac_of_bf16_peak": round(gram_flops / (gram_ms / 1e3) / 1e12 / bf16_peak, 4),
+                          "spectra": spectra}
     return res, w
 
 
