@@ -7,7 +7,9 @@
  *     normalised effective rank from the same Gram;
  *   - decode-time Selective Reconstruction (SR) attention: landmark-guided top-k
  *     chunk selection, reconstruction of only the selected rows, RoPE, and
- *     online-softmax GQA attention over them plus a raw sink/recent window.
+ *     online-softmax GQA attention over them plus a raw sink/recent window;
+ *     and its xK-SR mode, where only the keys are compressed and the selected
+ *     rows' values are read from the uncompressed cache.
  *
  * Sources (page title -- section):
  *   [xKV-blog] "xKV大模型压缩秘籍：跨层共享，小白也能轻松上手，收藏必备！" --

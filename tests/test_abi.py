@@ -4,6 +4,7 @@ CUDA call and nothing is launched)."""
 import ctypes as C
 import os
 import re
+import subprocess
 
 import pytest
 
@@ -145,3 +146,17 @@ def test_energy_rank_validation(xkv):
     assert f(g, 256, 128, 0.9, None, None, ws, n.value, None) == xkv.XKV_ERR_INVALID_ARG  # no rank output
     assert f(g, 256, 128, 0.9, r, None, ws, n.value - 1, None) == xkv.XKV_ERR_WORKSPACE
     assert f(g, 2 * 16384, 16384, 0.9, r, None, ws, 1 << 40, None) == xkv.XKV_ERR_UNSUPPORTED  # block > 8192
+
+
+def test_plain_c_host_program(xkv, tmp_path):
+    # the boundary is plain C: a C99 program that includes only xkv.h builds
+    # against libxkv.so and sees the same validation results
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    libdir = os.path.dirname(xkv.LIB_PATH)
+    exe = str(tmp_path / "abi_host_check")
+    subprocess.check_call(["gcc", "-std=c99", "-Wall", "-Wextra", "-Werror", "-I", os.path.join(root, "include"),
+                           os.path.join(root, "tests", "abi_host_check.c"), "-L", libdir, "-lxkv",
+                           "-Wl,-rpath," + libdir, "-o", exe])
+    out = subprocess.run([exe], capture_output=True, text=True, timeout=120)
+    assert out.returncode == 0, out.stderr
+    assert out.stdout.strip() == "ok"
