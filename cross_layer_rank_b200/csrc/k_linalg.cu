@@ -264,6 +264,7 @@ void cholqr_pass(const float* Y, float* Q, int n, int b, double shift_rel, doubl
 // once).  On convergence column i of W is lambda_i v_i, so |lambda_i| is its
 // norm and v_i is column i of V.
 constexpr int kJB = 16;
+constexpr int kJacobiInnerSweeps = 2;
 
 struct JacobiState {
   int active;      // rotations performed in the current sweep
@@ -334,8 +335,11 @@ __global__ void __launch_bounds__(256) jacobi_round_kernel(double* __restrict__ 
   __syncthreads();
   if (!s_need) return;
   // cyclic Jacobi on G (round-robin over 32 indices: 31 steps of 16 pairs);
-  // entries already below 1e-14 of the diagonal scale are left alone
-  for (int sweep = 0; sweep < 12; ++sweep) {
+  // entries already below 1e-14 of the diagonal scale are left alone.  At
+  // most kJacobiInnerSweeps sweeps: the pair need not be fully diagonalised,
+  // since it meets again in the next outer sweep, and the outer test above
+  // decides convergence
+  for (int sweep = 0; sweep < kJacobiInnerSweeps; ++sweep) {
     __shared__ int s_any;
     if (tid == 0) s_any = 0;
     __syncthreads();
