@@ -68,6 +68,21 @@ def attend_bytes_per_unit(w) -> int:
             + w.gq * w.head_dim * el)
 
 
+def cache_ratio(w, values_compressed: bool = True):
+    """Dense K+V cache bytes of a layer over the compressed cache's bytes per
+    layer: the group's shared A_K and A_V plus its per-layer Bt slices, alone
+    and with the landmarks.  Uncompressed values (the xK-SR mode) count T d
+    elements instead of A_V and Bt_V.  The raw sink/recent rows are left out."""
+    el = 2 if w.dtype == "bf16" else 4
+    dense = 2 * w.T * w.d * el
+    rv = w.rank_v if values_compressed else 0
+    ab = (w.T * (w.rank_k + rv) + w.group * w.d * (w.rank_k + rv)) * el / w.group
+    if not values_compressed:
+        ab += w.T * w.d * el
+    lm = w.n_kv_heads * w.n_mid * w.head_dim * el
+    return round(dense / ab, 3), round(dense / (ab + lm), 3)
+
+
 def xk_attend_bytes_per_unit(w) -> int:
     """The attend stage's algorithmic bytes per unit in the xK-SR mode: the
     selected A_K rows, the selected rows' hd value columns of the head, the
@@ -444,6 +459,7 @@ def run_cuda(args, rank, world, log):
         "e2e": {"value": round(tokens / (e2e_ms / args.steps / 1e3), 2), "unit": "tokens/s",
                 "h2d_bytes_per_step": q_bytes, "d2h_bytes_per_step": o_bytes},
         "gpu_launches": 4 * L * args.steps,
+        "cache_ratio": dict(zip(("a_b", "with_landmarks"), cache_ratio(w))),
         "clocks": clocks,
         "flops_per_step": sr_flops_per_unit(w) * units_step,
     }
@@ -524,7 +540,8 @@ def measure_xk_sr(xkv, w, model, device, stream, L, steps, warmup, peak_gbs):
                           "combine": round(st[3], 5)},
             "attend_roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peak_gbs, "unit": "GB/s",
                                 "frac": round(gbs / peak_gbs, 4), "bytes_per_launch": bytes_attend},
-            "value_cache_gb": round(L * w.batch * w.T * w.d * 2 / 1e9, 2)}
+            "value_cache_gb": round(L * w.batch * w.T * w.d * 2 / 1e9, 2),
+            "cache_ratio": dict(zip(("a_b", "with_landmarks"), cache_ratio(w, values_compressed=False)))}
 
 
 def measure_full_reconstruction(xkv, w, model, device, stream, sr_call_ms):
@@ -656,7 +673,7 @@ def main():
             r2, _ = run_cuda(a2, rank, world, log)
             res.setdefault("other_workloads", {})[name] = {
                 k: r2[k] for k in ("value", "unit", "ms_per_step", "steps", "roofline", "stage_rooflines", "e2e",
-                                   "config", "clocks")}
+                                   "config", "clocks", "cache_ratio")}
     if rank == 0 and not args.no_cpu_baseline and world == 1:
         res["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds, log)
     if world > 1:
