@@ -68,6 +68,47 @@ def attend_bytes_per_unit(w) -> int:
             + w.gq * w.head_dim * el)
 
 
+def code_digest(text: str) -> str:
+    """sha1 of C/C++/CUDA source with comments and blank lines removed and runs
+    of white space folded (string and character literals kept), so that the
+    digest changes with the code and not with its comments or layout."""
+    out, i, n = [], 0, len(text)
+    while i < n:
+        c = text[i]
+        if c in "\"'":
+            j = i + 1
+            while j < n and text[j] != c:
+                j += 2 if text[j] == "\\" else 1
+            out.append(text[i:j + 1])
+            i = j + 1
+        elif text.startswith("//", i):
+            j = text.find("\n", i)
+            i = n if j < 0 else j
+        elif text.startswith("/*", i):
+            j = text.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+        else:
+            out.append(c)
+            i += 1
+    lines = [" ".join(ln.split()) for ln in "".join(out).splitlines()]
+    return hashlib.sha1("\n".join(ln for ln in lines if ln).encode()).hexdigest()
+
+
+def profiled_traffic(workload: str):
+    """DRAM bytes per launch of the dominant kernel from the committed ncu
+    summary (profiles/traffic.json), or None unless the kernel source's code
+    (comments aside) is still the code that was profiled."""
+    tp = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        ent = json.load(open(tp)).get(workload)
+        src = open(os.path.join(ROOT, ent["source"]), encoding="utf-8").read()
+        if code_digest(src) == ent["source_code_sha1"]:
+            return ent["bytes_per_launch"]
+    except Exception:
+        pass
+    return None
+
+
 def cache_ratio(w, values_compressed: bool = True):
     """Dense K+V cache bytes of a layer over the compressed cache's bytes per
     layer: the group's shared A_K and A_V plus its per-layer Bt slices, alone
@@ -421,18 +462,7 @@ def run_cuda(args, rank, world, log):
     # dominant kernel: selective reconstruction + attention (sr_attend)
     bytes_attend = attend_bytes_per_unit(w) * w.batch * w.n_kv_heads
     achieved_attend = bytes_attend / (stage_ms[2] / 1e3) / 1e9
-    # DRAM traffic per launch from the committed ncu summary, valid only while
-    # the kernel source is the one that was profiled
-    traffic = None
-    tp = os.path.join(ROOT, "profiles", "traffic.json")
-    if os.path.exists(tp):
-        try:
-            ent = json.load(open(tp)).get(args.workload)
-            src = open(os.path.join(ROOT, ent["source"]), "rb").read()
-            if ent and hashlib.sha1(src).hexdigest() == ent["source_sha1"]:
-                traffic = ent["bytes_per_launch"]
-        except Exception:
-            traffic = None
+    traffic = profiled_traffic(args.workload)
     q_bytes = sum(t.numel() * t.element_size() for t in model["q"])
     o_bytes = sum(t.numel() * t.element_size() for t in outs)
     res = {

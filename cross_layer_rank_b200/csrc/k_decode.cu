@@ -3,20 +3,28 @@
 // reconstruction of only the selected rows of K and V from the shared basis A
 // and the layer's B_l, RoPE on the rebuilt keys, and online-softmax GQA
 // attention (KQ-SVD page, 3.2) over them plus the raw sink/recent window.
+// The same kernels serve the xK-SR mode of the explainer (keys compressed,
+// values read whole from a [B][T][d] cache): the value operand is then head
+// h's columns of V and the combine skips the Bt_V projection.
 //
-// Kernels (one decode step of one layer = 4 launches):
+// Kernels (one decode step of one layer = 4 launches, chained with
+// programmatic dependent launch):
 //   sr_score   : s_c = (sum_g q_g) . landmark_c            (HBM stream of landmarks)
-//   sr_topk    : exact radix select of the k best chunks, ascending output
+//   sr_topk    : exact top-k per unit in one CTA (bucket histogram, a refining
+//                histogram of the boundary bucket, then a rank count or radix
+//                passes over its candidates; ties to the lower chunk),
+//                ascending output; extra blocks of the same grid compute the
+//                raw sink/recent window's partial (m, l, o)
 //   sr_attend  : persistent CTAs over (unit, 128-row tile) ranges.  tcgen05
 //                path: TMA gathers the selected 8-row chunk slabs of A_K
 //                (8 x 64 bf16 = one 1 KiB swizzle atom each) and the head's
 //                Bt_K slice, tcgen05.mma rebuilds the 128 x 128 key tile in
-//                TMEM, the epilogue applies RoPE and the q . k products, and
-//                256 threads fold p into u_g = sum_t p_gt A_V[t] (the value
+//                TMEM, the epilogue applies RoPE and the q . k products, and a
+//                second MMA folds p into u_g = sum_t p_gt A_V[t] (the value
 //                path is re-associated: o_g = (u_g / l_g) Bt_V^T, exact up to
 //                rounding).  A SIMT path covers f32 and other shapes.
-//   sr_combine : merges the per-CTA (m, l, u) partials with the sink/recent
-//                rows and applies Bt_V.
+//   sr_combine : merges the per-CTA (m, l, u) partials with the window
+//                partial and applies Bt_V.
 #include <float.h>
 
 #include <algorithm>
@@ -607,8 +615,10 @@ constexpr int kVAccCol = 256;  // TMEM columns of the value accumulators (2 x 64
 //   D  U_g = sum over slots of u 2^(m - M_g), kept in shared memory in an
 //      order where lane-consecutive 8-column groups are word-consecutive;
 //   E  o_g[j] = (U_g . Bt_V[h hd + j] + 2^(m_w - M_g) o_w,g[j]) / L_g for the
-//      split's columns (warp per column, 16-byte loads of the Bt_V rows of
-//      all of the warp's columns issued first).
+//      split's columns (a warp per 4 columns, whose Bt_V rows were staged in
+//      shared memory by cp.async or are loaded 16 bytes a lane; the warp's 32
+//      sums are reduce-scattered so each lane stores one).  With uncompressed
+//      values (xK-SR) U_g is already o_g's value sum and E is a scaled copy.
 constexpr int kCombineSplit = 4;
 constexpr int kCombineThreads = 256;
 constexpr int kMaxSlots = 64;

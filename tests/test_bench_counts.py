@@ -35,3 +35,13 @@ def test_cache_ratio_with_uncompressed_values():
     T, d, G, r = w.T, w.d, w.group, w.rank_k
     assert abs(r_ab - 2 * T * d / (T * d + (T + G * d) * r / G)) < 1e-3
     assert 1.0 < r_ab < 2.0
+
+
+def test_code_digest_ignores_comments_only():
+    a = 'int f(int x) {  // add one\n  /* block\n comment */ return x + 1;\n}\nconst char* s = "a // b";\n'
+    b = 'int f(int x) {  // plus one\n\n  return x + 1;   \n}\nconst char* s = "a // b";\n'
+    c = 'int f(int x) {\n  return x + 2;\n}\nconst char* s = "a // b";\n'
+    d = 'int f(int x) {\n  return x + 1;\n}\nconst char* s = "a // c";\n'
+    assert bench.code_digest(a) == bench.code_digest(b)
+    assert bench.code_digest(a) != bench.code_digest(c)
+    assert bench.code_digest(a) != bench.code_digest(d)
