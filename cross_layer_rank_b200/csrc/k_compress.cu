@@ -3,13 +3,15 @@
 // of KV-CoRE (2.A):
 //   1. C = sum over token shards of X_s^T X_s, X = [X_1 | ... | X_G] read through
 //      the G layer pointers (never concatenated).  bf16: each shard is
-//      transposed to a K-major copy and multiplied on tcgen05 tensor cores,
-//      upper-triangular 128 x 128 tiles with a mirrored fp32 epilogue.
+//      transposed to a K-major copy and multiplied on tcgen05 tensor cores:
+//      upper-triangular 128 x 256 tiles when G d is a multiple of 256 (else
+//      128 x 128), 256-row chunks accumulated in TMEM and summed in fp32
+//      registers, and a mirrored fp32 epilogue.
 //   2. top-r subspace: block subspace iteration Y = C Q, Q = qr(Y) (shifted
-//      Cholesky QR, two passes, fp64 small factors), started from a Gaussian
-//      block (Philox4x32-10 + Box-Muller on the device);
-//      Rayleigh-Ritz: H = Q^T C Q, eigenpairs of H by one-sided block Jacobi,
-//      V_r = Q U[:, top r].
+//      Cholesky QR, two passes, fp64 small factors with a blocked Cholesky),
+//      started from a Gaussian block (Philox4x32-10 + Box-Muller on the
+//      device); Rayleigh-Ritz: H = Q^T C Q, eigenpairs of H by one-sided block
+//      Jacobi, V_r = Q U[:, top r].
 //   3. A = X V_r: tcgen05 GEMM over the layer tensor maps with V_r split into a
 //      bf16 hi/lo pair (two MMAs per step keep ~16 significant bits of V_r);
 //      Bt = V_r stored in the cache dtype (layer l owns rows l d .. l d + d - 1).
