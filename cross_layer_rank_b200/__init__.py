@@ -40,6 +40,7 @@ EXPORTS = (
     "xkv_sr_attention_decode_noalloc",
     "xkv_xk_sr_workspace_size", "xkv_xk_sr_attention_decode",
     "xkv_sr_profile_enable", "xkv_sr_profile_read",
+    "xkv_selftest_expired_wait",
     "xkv_full_reconstruct",
     "xkv_dense_workspace_size", "xkv_dense_attention_decode",
     "xkv_ner_workspace_size", "xkv_ner", "xkv_energy_rank",
@@ -92,6 +93,7 @@ def _load():
         "xkv_xk_sr_workspace_size": (C.c_int, [C.POINTER(SRParams), C.POINTER(sz)]),
         "xkv_xk_sr_attention_decode": (C.c_int, [C.POINTER(SRParams), vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz,
                                                  vp]),
+        "xkv_selftest_expired_wait": (C.c_int, [vp]),
         "xkv_sr_profile_enable": (C.c_int, [C.c_int]),
         "xkv_sr_profile_read": (C.c_int, [C.POINTER(C.c_float)]),
         "xkv_full_reconstruct": (C.c_int, [vp, vp, i64, C.c_int, C.c_int, C.c_int, C.c_int, C.c_int, C.c_float,
@@ -278,6 +280,12 @@ def xkv_xk_sr_attention_decode(p: SRParams, q, A_K, Bt_K, V, landmarks, sr_K, sr
     _check(lib.xkv_xk_sr_attention_decode(C.byref(p), _ptr(q), _ptr(A_K), _ptr(Bt_K), _ptr(V), _ptr(landmarks),
                                           _ptr(sr_K), _ptr(sr_V), _ptr(out), _ptr(sel_out), _ptr(ws), ws.numel(),
                                           _stream(stream)), "xkv_xk_sr_attention_decode")
+
+
+def xkv_selftest_expired_wait(stream=None) -> None:
+    """Launch the bounded-wait self-test (a wait that runs out after about one
+    second); read the outcome with get_device_status()."""
+    _check(lib.xkv_selftest_expired_wait(_stream(stream)), "xkv_selftest_expired_wait")
 
 
 def xkv_sr_profile_enable(enable: bool = True) -> None:

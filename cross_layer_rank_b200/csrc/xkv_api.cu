@@ -9,6 +9,7 @@
 #include <algorithm>
 #include <mutex>
 
+#include "xkv_common.cuh"
 #include "xkv_internal.h"
 
 namespace xkv {
@@ -143,6 +144,27 @@ xkv_status xkv_get_device_status(void* stream) {
     if (cudaMemcpy(p, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) return XKV_ERR_CUDA;
   }
   return static_cast<xkv_status>(v);
+}
+
+// ------------------------------------------------ bounded-wait self-test
+// One CTA waits on an mbarrier that nothing completes: mbar_wait gives up
+// after kWaitLimitNs, records kDevTimeout and the kernel returns.
+__global__ void selftest_expired_wait_kernel(int* status) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) (void)mbar_wait(&bar, 0, status);
+  __syncthreads();
+}
+
+xkv_status xkv_selftest_expired_wait(void* stream) {
+  int* status = device_status_ptr();
+  if (!status) return XKV_ERR_CUDA;
+  selftest_expired_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(status);
+  return cudaPeekAtLastError() == cudaSuccess ? XKV_OK : XKV_ERR_CUDA;
 }
 
 // ------------------------------------------------------------------- Gram

@@ -205,6 +205,14 @@ XKV_API xkv_status xkv_xk_sr_attention_decode(const xkv_sr_params* p, const void
                                               const void* sr_K, const void* sr_V, float* out, int32_t* sel_out,
                                               void* workspace, size_t ws_bytes, void* stream);
 
+/* Failure-detection self-test (the pages have no counterpart).  Launches one
+ * CTA whose mbarrier wait nothing ever completes, through the same bounded wait
+ * every kernel of the library uses: after its limit (about one second) the
+ * wait gives up, records XKV_ERR_DEVICE_TIMEOUT in the device status word and
+ * the kernel returns, leaving the context usable.  Returns the launch status;
+ * xkv_get_device_status(stream) then reports (and clears) the timeout. */
+XKV_API xkv_status xkv_selftest_expired_wait(void* stream);
+
 /* Stage timing (measurement aid; the method has no counterpart).  While
  * enabled, every xkv_sr_attention_decode call records CUDA events on its
  * stream around its four launches: chunk scores, top-k (+ raw window
