@@ -85,3 +85,25 @@ def test_shared_basis_beats_per_layer_at_equal_storage_on_aligned_layers():
     per = sum(oracle.compress_group([l], 3)["err_subspace"] ** 2 for l in layers)
     assert shared["err_subspace"] ** 2 < per
     assert shared["err_subspace"] ** 2 < 1e-2 * np.sum(X ** 2)
+
+
+def test_full_reconstruct_at_full_rank_returns_each_layer():
+    # full_reconstruct (the comparison path's rebuild) of layer l from the
+    # group's factors: at full rank A Bt_l^T is X_l itself, and with RoPE every
+    # head's row is X_l's row turned by its position (the rotation pinned in
+    # the RoPE tests)
+    n_kv, hd = 2, 8
+    layers = _group(T=40, d=n_kv * hd, G=2)
+    d = n_kv * hd
+    res = oracle.compress_group(layers, 2 * d)
+    A = res["A"].astype(np.float32)
+    for l, X in enumerate(layers):
+        Bt = res["Bt"][l * d:(l + 1) * d].astype(np.float32)
+        plain = oracle.full_reconstruct(A, Bt, n_kv, hd, False, 500000.0)
+        assert np.abs(plain - X).max() <= 1e-5 * np.abs(X).max()
+        rot = oracle.full_reconstruct(A, Bt, n_kv, hd, True, 500000.0)
+        for t in (0, 1, 17, 39):
+            for h in range(n_kv):
+                sl = slice(h * hd, (h + 1) * hd)
+                ref = oracle.rope(X[t, sl], t, 500000.0)
+                assert np.abs(rot[t, sl] - ref).max() <= 1e-5 * np.abs(X).max()
