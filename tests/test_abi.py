@@ -5,6 +5,7 @@ import ctypes as C
 import os
 import re
 import subprocess
+import sys
 
 import pytest
 
@@ -160,3 +161,26 @@ def test_plain_c_host_program(xkv, tmp_path):
     out = subprocess.run([exe], capture_output=True, text=True, timeout=120)
     assert out.returncode == 0, out.stderr
     assert out.stdout.strip() == "ok"
+
+
+def test_package_fails_loudly_without_the_library(tmp_path):
+    # a copy of the binding with no libxkv.so beside it must refuse to import:
+    # there is no CPU or PyTorch fallback
+    pkg = tmp_path / "cross_layer_rank_b200"
+    pkg.mkdir()
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    src = open(os.path.join(root, "cross_layer_rank_b200", "__init__.py")).read()
+    (pkg / "__init__.py").write_text(src)
+    code = "import sys; sys.path.insert(0, sys.argv[1]); import cross_layer_rank_b200"
+    out = subprocess.run([sys.executable, "-c", code, str(tmp_path)], capture_output=True, text=True, timeout=300)
+    assert out.returncode != 0
+    assert "ImportError" in out.stderr and "libxkv.so not built" in out.stderr
+
+
+def test_binding_rejects_host_and_strided_tensors(xkv):
+    import torch
+    with pytest.raises(ValueError):
+        xkv._ptr(torch.zeros(4))  # host memory
+    if torch.cuda.is_available():
+        with pytest.raises(ValueError):
+            xkv._ptr(torch.zeros((4, 4), device="cuda").t())  # not contiguous
