@@ -117,6 +117,14 @@ def test_compress_and_gram_validation(xkv):
     # bf16 needs rank % 64 == 0
     assert xkv.lib.xkv_compress_workspace_size(4, 1024, 128, 48, 64, 0, xkv.XKV_BF16, C.byref(n)) == \
         xkv.XKV_ERR_UNSUPPORTED
+    # block width b = min(rank + oversample, G d, T) up to 3584 (the compression
+    # sweep's largest case, G = 8 at rank 1024 with p = 256, is far inside)
+    f = xkv.lib.xkv_compress_workspace_size
+    assert f(8, 32768, 1024, 1024, 256, 8192, xkv.XKV_BF16, C.byref(n)) == xkv.XKV_OK
+    assert f(8, 32768, 1024, 3520, 64, 8192, xkv.XKV_F32, C.byref(n)) == xkv.XKV_OK
+    assert f(8, 32768, 1024, 3520, 65, 8192, xkv.XKV_F32, C.byref(n)) == xkv.XKV_ERR_UNSUPPORTED
+    assert f(8, 32768, 1024, 4096, 1024, 8192, xkv.XKV_BF16, C.byref(n)) == xkv.XKV_ERR_UNSUPPORTED
+    assert f(8, 3000, 1024, 2048, 4096, 0, xkv.XKV_BF16, C.byref(n)) == xkv.XKV_OK  # b capped by T
     ptrs = (C.c_void_p * 2)(None, None)
     assert xkv.lib.xkv_gram_accumulate(ptrs, 2, 100, 64, 64, xkv.XKV_F32, C.c_void_p(1 << 20), None, 0, None) == \
         xkv.XKV_ERR_INVALID_ARG
