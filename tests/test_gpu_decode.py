@@ -57,6 +57,15 @@ def test_sr_bf16_gqa7_single_tile(xkv):
     _parity(xkv, w)
 
 
+@pytest.mark.parametrize("n_q_heads", [2, 16])
+def test_sr_bf16_gqa_group_extremes(xkv, n_q_heads):
+    # 2 KV heads: one query head per KV head (plain multi-head attention) and
+    # the largest group the kernels take (8)
+    w = synth.Workload(f"sr_bf16_hq{n_q_heads}", 1, 4, 4, 2, 128, n_q_heads, 8 + 32 + 8 * 100, 96, 0.8, 128, 128,
+                       topk=21)
+    _parity(xkv, w)
+
+
 def test_sr_bf16_odd_key_atom_count(xkv):
     # key rank 192 = three 64-column atoms: the last key stage is half empty;
     # value rank 320 leaves the last 128-column value block half empty
