@@ -77,3 +77,17 @@ def test_kv_group_structure():
     assert not np.allclose(Ks[0], Ks[1])
     Vs = synth.kv_group(w, 0, 0, "V", T=256)
     assert not np.allclose(Ks[0], Vs[0])
+
+
+def test_group_spectrum_has_no_gap_at_the_rank_and_a_gap_at_the_latent_dimension():
+    # the recipe's spectra: eigenvalues of the group Gram decay like i^(-2 alpha)
+    # with no gap at the compression rank (so a subspace projector is not
+    # unique there) and a sharp drop after the latent dimension m, where only
+    # the 0.01 N noise remains
+    w = synth.WORKLOADS["tiny_f32"]
+    X = np.concatenate([k.astype(np.float64) for k in synth.kv_group(w, 0, 0, "K")], axis=1)
+    lam = np.linalg.eigvalsh(X.T @ X)[::-1]
+    r, m = w.rank_k, w.latent
+    assert lam[r - 1] / lam[r] < 1.1
+    assert lam[m - 1] / lam[m] > 20.0
+    assert np.all(lam[m:] < 1e-3 * lam[0])
