@@ -45,3 +45,15 @@ def test_code_digest_ignores_comments_only():
     assert bench.code_digest(a) == bench.code_digest(b)
     assert bench.code_digest(a) != bench.code_digest(c)
     assert bench.code_digest(a) != bench.code_digest(d)
+
+
+def test_attend_bytes_per_unit_llama():
+    # per (sequence, layer, KV head) at the Llama shape: the selected A rows are
+    # k C (r_K + r_V) 2 = 4 MiB, the head's Bt_K slice r_K hd 2 = 128 KiB, the
+    # group's queries Gq hd 2 = 1 KiB; xK-SR swaps r_V for hd
+    w = synth.WORKLOADS["llama8b_64k_b4"]
+    assert bench.attend_bytes_per_unit(w) == 4 * 2**20 + 128 * 2**10 + 2**10
+    assert bench.xk_attend_bytes_per_unit(w) == 256 * 8 * (512 + 128) * 2 + 128 * 2**10 + 2**10
+    # launch totals used by the roofline lines: 32 units
+    assert bench.attend_bytes_per_unit(w) * w.batch * w.n_kv_heads == 138444800
+    assert bench.xk_attend_bytes_per_unit(w) * w.batch * w.n_kv_heads == 88113152
