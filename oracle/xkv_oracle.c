@@ -23,9 +23,9 @@
  *               cache: h_T = softmax(q_T K^T / sqrt(d)) V) and 3.3 (truncated SVD
  *               is the Frobenius-optimal rank-R approximation, P = V V^T).
  *
- * Readings where the pages leave a step open (each also listed in the design
- * notes): the Gram is uncentred; factors are A = X V_r and B = V_r^T (stored
- * transposed, Bt = V_r); keys are factorised before RoPE and RoPE (rotate-half,
+ * Readings where the pages leave a step open: the Gram is uncentred; factors
+ * are A = X V_r and B = V_r^T (stored transposed, Bt = V_r); keys are
+ * factorised before RoPE and RoPE (rotate-half,
  * inv_freq_j = theta^(-2j/hd)) is applied to rebuilt keys at their absolute
  * position; a landmark is the mean of a chunk's post-RoPE keys; the chunk score
  * of a KV head is the sum over its GQA query heads of q_g . l_c; top-k breaks
@@ -81,21 +81,30 @@ XO_EXPORT void xo_round_bf16_array(const double* x, float* y, int64_t n) {
 XO_EXPORT void xo_gram_accumulate(const float* const* layers, int G, int64_t T, int d,
                                   int64_t ldx, int64_t t0, int64_t t1, double* C) {
   const int n = G * d;
+  const int64_t rows = t1 - t0;
   (void)T;
-#pragma omp parallel for schedule(dynamic, 8)
+  if (rows <= 0) return;
+  /* Column i of X copied out contiguously (a change of layout only: each entry
+   * below is still the ascending-t sum of x_t[i] x_t[j]). */
+  float* cols = (float*)malloc(sizeof(float) * (size_t)n * (size_t)rows);
+#pragma omp parallel for schedule(static)
   for (int i = 0; i < n; ++i) {
     const float* Li = layers[i / d];
     const int ci = i % d;
+    for (int64_t t = 0; t < rows; ++t) cols[(int64_t)i * rows + t] = Li[(t0 + t) * ldx + ci];
+  }
+#pragma omp parallel for schedule(dynamic, 8)
+  for (int i = 0; i < n; ++i) {
+    const float* xi = cols + (int64_t)i * rows;
     for (int j = i; j < n; ++j) {
-      const float* Lj = layers[j / d];
-      const int cj = j % d;
+      const float* xj = cols + (int64_t)j * rows;
       double s = 0.0;
-      for (int64_t t = t0; t < t1; ++t)
-        s += (double)Li[t * ldx + ci] * (double)Lj[t * ldx + cj];
+      for (int64_t t = 0; t < rows; ++t) s += (double)xi[t] * (double)xj[t];
       C[(int64_t)i * n + j] += s;
       if (j != i) C[(int64_t)j * n + i] += s;
     }
   }
+  free(cols);
 }
 
 /* --------------------------------------------------------------- Jacobi */
@@ -566,4 +575,43 @@ XO_EXPORT int xo_ner(const double* C, int n, int block, double rel_tol, double* 
     free(Ab); free(Vb); free(w);
   }
   return status;
+}
+
+/* ---------------------------------------------------- multi-step decode */
+/* [xKV-blog] (the editor's note after "仅仅压缩还不够，xKV 还做了“选择性重建”"):
+ * the factorisation covers the long prefill; tokens generated afterwards stay
+ * raw in the recent window until a whole chunk of them can join the
+ * compressed cache.  Two steps of that roll, restated plainly:
+ *
+ * Projection of `rows` token rows onto a stored group basis V ((G d) x r):
+ *   A[t][k] = sum_i x_t[i] V[i][k],  x_t = [K_1[t] | ... | K_G[t]]
+ * (the same A = X V_r as the prefill factorisation, "xKV 到底做了什么").
+ * layers[l] is rows x d with row stride ldx; A is rows x r. */
+XO_EXPORT void xo_project_rows(const float* const* layers, int G, int64_t rows, int d, int64_t ldx,
+                               const float* V, int r, double* A) {
+  const int n = G * d;
+  for (int64_t t = 0; t < rows; ++t)
+    for (int k = 0; k < r; ++k) {
+      double s = 0.0;
+      for (int i = 0; i < n; ++i) s += (double)layers[i / d][t * ldx + (i % d)] * (double)V[(int64_t)i * r + k];
+      A[t * r + k] = s;
+    }
+}
+
+/* Landmark of one chunk whose C rows sit at absolute positions t0 .. t0+C-1
+ * ([xKV-blog] "选择性重建"): for KV head h, the mean over i of
+ * RoPE_{t0+i}(K[i, h hd : (h+1) hd]).  K rows have stride ldk; out is
+ * [Hkv][hd]. */
+XO_EXPORT void xo_chunk_landmark(const float* K, int64_t ldk, int Hkv, int hd, int C, int64_t t0, double theta,
+                                 double* out) {
+  double x[512], y[512];
+  for (int h = 0; h < Hkv; ++h) {
+    for (int j = 0; j < hd; ++j) out[h * hd + j] = 0.0;
+    for (int i = 0; i < C; ++i) {
+      for (int j = 0; j < hd; ++j) x[j] = (double)K[i * ldk + h * hd + j];
+      xo_rope(x, y, hd, (double)(t0 + i), theta);
+      for (int j = 0; j < hd; ++j) out[h * hd + j] += y[j];
+    }
+    for (int j = 0; j < hd; ++j) out[h * hd + j] /= (double)C;
+  }
 }
