@@ -269,3 +269,73 @@ def energy_rank(Cm: np.ndarray, block: int, energy: float = 0.95):
             ranks[i] = int(np.searchsorted(cum, energy * total, side="left")) + 1
     return ranks, lam
 
+
+# ------------------------------------------------------------ multi-step decode
+def project_rows(layers: Sequence[np.ndarray], V: np.ndarray) -> np.ndarray:
+    """A = [layers...] V for a few token rows (fp64); V is (G d) x r."""
+    layers = [_f32(l) for l in layers]
+    G = len(layers)
+    rows, d = layers[0].shape
+    V = _f32(V)
+    r = V.shape[1]
+    A = np.empty((rows, r), dtype=np.float64)
+    lib().xo_project_rows(_layer_ptrs(layers), C.c_int(G), C.c_int64(rows), C.c_int(d), C.c_int64(d), _p(V),
+                          C.c_int(r), _p(A))
+    return A
+
+
+def chunk_landmark(K_rows: np.ndarray, n_kv_heads: int, head_dim: int, t0: int, theta: float) -> np.ndarray:
+    """[Hkv][hd] mean of RoPE_{t0+i}(K_rows[i]) over the chunk's rows (fp64)."""
+    K_rows = _f32(K_rows)
+    Cn = K_rows.shape[0]
+    out = np.empty((n_kv_heads, head_dim), dtype=np.float64)
+    lib().xo_chunk_landmark(_p(K_rows), C.c_int64(K_rows.shape[1]), C.c_int(n_kv_heads), C.c_int(head_dim),
+                            C.c_int(Cn), C.c_int64(t0), C.c_double(theta), _p(out))
+    return out
+
+
+class SRState:
+    """Host-side state of one layer group for multi-step decode (test
+    infrastructure): the compressed rows A_K / A_V [B][T_cap][r], the group
+    bases Bt_K / Bt_V [B][G d][r], per layer the landmarks [B][Hkv][cap][hd] and
+    the raw window K / V [B][sink + recent + chunk][d] (sink rows first, then the
+    current recent rows), the length T, the middle-chunk count n_mid and the
+    number of recent rows w_cur.  Stored values are bf16 numbers held in
+    float32, as the library stores them."""
+
+    def __init__(self, w, A_K, A_V, Bt_K, Bt_V, lms, win_K, win_V, T, n_mid, w_cur):
+        self.w, self.A_K, self.A_V, self.Bt_K, self.Bt_V = w, A_K, A_V, Bt_K, Bt_V
+        self.lms, self.win_K, self.win_V = lms, win_K, win_V
+        self.T, self.n_mid, self.w_cur = T, n_mid, w_cur
+
+    def append(self, k_new: Sequence[np.ndarray], v_new: Sequence[np.ndarray]):
+        """One generated token for every layer of the group: k_new[l], v_new[l]
+        are [B][d] (pre-RoPE keys).  The rows join the raw window; when the
+        window holds recent + chunk rows, its oldest chunk is rolled into the
+        compressed cache: A rows by projection onto the stored bases, one
+        landmark per layer and KV head, and the window moves down by a chunk."""
+        w = self.w
+        s, Cn, G = w.sink, w.chunk, w.group
+        row = s + self.w_cur
+        for l in range(G):
+            self.win_K[l][:, row] = k_new[l]
+            self.win_V[l][:, row] = v_new[l]
+        self.w_cur += 1
+        self.T += 1
+        if self.w_cur < w.recent + Cn:
+            return False
+        t0 = s + self.n_mid * Cn
+        for b in range(self.A_K.shape[0]):
+            for X, A, Bt in ((self.win_K, self.A_K, self.Bt_K), (self.win_V, self.A_V, self.Bt_V)):
+                rows = [X[l][b, s:s + Cn] for l in range(G)]
+                A[b, t0:t0 + Cn] = round_bf16(project_rows(rows, Bt[b]))
+            for l in range(G):
+                lm = chunk_landmark(self.win_K[l][b, s:s + Cn], w.n_kv_heads, w.head_dim, t0, w.rope_theta)
+                self.lms[l][b, :, self.n_mid] = round_bf16(lm)
+        for X in (self.win_K, self.win_V):
+            for l in range(G):
+                X[l][:, s:s + w.recent] = X[l][:, s + Cn:s + Cn + w.recent].copy()
+        self.n_mid += 1
+        self.w_cur = w.recent
+        return True
+
