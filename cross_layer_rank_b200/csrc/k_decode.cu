@@ -597,7 +597,7 @@ constexpr int kSmemFt = kSmemRot + 8 * kRopeStride * 4;
 constexpr int kSmemRed = kSmemFt + 64 * 8;
 constexpr int kSmemSpart = kSmemRed + 64 * 4;                         // [128][8] partial scores of half 1
 constexpr int kSmemBars = kSmemSpart + 128 * kMaxGQ * 4;
-constexpr int kNumBars = 2 * kKStages + 2 * kBStages + 2 * kVStages + 12;
+constexpr int kNumBars = 2 * kKStages + 2 * kBStages + 2 * kVStages + 14;
 constexpr int kSmemEnd = kSmemBars + kNumBars * 8 + 16;
 constexpr int kVAccCol = 256;  // TMEM columns of the value accumulators (2 x 64)
 
@@ -863,7 +863,8 @@ __global__ void __launch_bounds__(kAttendThreads, 1)
   uint64_t* pempty = pfull + 2;
   uint64_t* vaccfull = pempty + 2;
   uint64_t* vaccempty = vaccfull + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(vaccempty + 2);
+  uint64_t* drain = vaccempty + 2;  // [2] last commit of each MMA issuer
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -882,6 +883,7 @@ __global__ void __launch_bounds__(kAttendThreads, 1)
       mbar_init(&pempty[i], 129);
       mbar_init(&vaccfull[i], 1);
       mbar_init(&vaccempty[i], 128);
+      mbar_init(&drain[i], 1);
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -947,6 +949,12 @@ __global__ void __launch_bounds__(kAttendThreads, 1)
           }
         }
       }
+      // on abort, the copies already issued still land in Ka / Kb: wait for
+      // them before the CTA releases its shared memory
+      if (*abort_flag) {
+        drain_ring(kfull, kKStages, ks, args.status);
+        drain_ring(bfull, kBStages, bs, args.status);
+      }
     }
   } else if (warp == 13) {
     // ---------------------------------------------------- TMA producer (values)
@@ -974,6 +982,7 @@ __global__ void __launch_bounds__(kAttendThreads, 1)
           }
         }
       }
+      if (*abort_flag) drain_ring(vfull, kVStages, vsn, args.status);
     }
   } else if (warp == 14) {
     // -------------------------------------------------------- key MMA issuer
@@ -1009,6 +1018,9 @@ __global__ void __launch_bounds__(kAttendThreads, 1)
       int j = 0;
       for (int x = tb; x < te && ok && !*abort_flag; ++x, ++j) ok = issue_keys(j);
       if (!ok) *abort_flag = 1;
+      // every MMA issued by this thread has finished before TMEM is released
+      umma_commit(&drain[0]);
+      (void)mbar_wait(&drain[0], 0, args.status);
     }
   } else if (warp == 15) {
     // ------------------------------------------------------ value MMA issuer
@@ -1042,6 +1054,8 @@ __global__ void __launch_bounds__(kAttendThreads, 1)
       int j = 0;
       for (int x = tb; x < te && ok && !*abort_flag; ++x, ++j) ok = issue_values(j, x);
       if (!ok) *abort_flag = 1;
+      umma_commit(&drain[1]);
+      (void)mbar_wait(&drain[1], 0, args.status);
     }
   } else if (warp < 8) {
     // --------------------------------------- key epilogue: RoPE, q.k, softmax

@@ -7,6 +7,8 @@
 //     semi-definite matrices: the Rayleigh-Ritz step (eigenvalues + vectors)
 //     and KV-CoRE's spectra (eigenvalues only);
 //   - ordering of eigenvalues and the NER reduction (KV-CoRE page, 2.B).
+#include <stdlib.h>
+
 #include <algorithm>
 
 #include "xkv_common.cuh"
@@ -445,20 +447,43 @@ __global__ void column_norms_kernel(const double* __restrict__ W, double* __rest
   if (lane == 0) lam[static_cast<int64_t>(prob) * n + c] = sqrt(s);
 }
 
+// A problem still rotating after the last sweep has not converged: its
+// eigenvalues (and vectors) are not final, which is recorded as a numerical
+// fault rather than returned silently.
+__global__ void jacobi_check_kernel(const JacobiState* state, int count, int* status) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < count && !state[i].converged) record_status(status, kDevNumerical);
+}
+
 size_t jacobi_workspace(int, int count) { return align_up(static_cast<size_t>(count) * sizeof(JacobiState)); }
+
+// Sweep limit: 40, or XKV_JACOBI_MAX_SWEEPS (a diagnostic override, e.g. 1 to
+// see the non-convergence report).
+static int jacobi_max_sweeps() {
+  static int v = 0;
+  if (v == 0) {
+    const char* e = getenv("XKV_JACOBI_MAX_SWEEPS");
+    const int x = e ? atoi(e) : 0;
+    v = x > 0 ? x : 40;
+  }
+  return v;
+}
 
 xkv_status jacobi_launch(double* W, double* V, double* lam, int n, int count, void* ws, cudaStream_t st) {
   JacobiState* state = static_cast<JacobiState*>(ws);
+  int* status = device_status_ptr();
+  if (!status) return XKV_ERR_CUDA;
   int nblk = (n + kJB - 1) / kJB;
   if (nblk & 1) ++nblk;
   if (nblk < 2) nblk = 2;
   jacobi_init_kernel<<<256, 256, 0, st>>>(V, n, count, state);
-  const int max_sweeps = 30;
+  const int max_sweeps = jacobi_max_sweeps();
   for (int s = 0; s < max_sweeps; ++s) {
     for (int r = 0; r < nblk - 1; ++r)
       jacobi_round_kernel<<<dim3(nblk / 2, count), 256, 0, st>>>(W, V, n, nblk, r, state, 1e-11);
     jacobi_sweep_end_kernel<<<(count + 127) / 128, 128, 0, st>>>(state, count);
   }
+  jacobi_check_kernel<<<(count + 127) / 128, 128, 0, st>>>(state, count, status);
   column_norms_kernel<<<dim3((n + 7) / 8, count), 256, 0, st>>>(W, lam, n, count);
   return cudaPeekAtLastError() == cudaSuccess ? XKV_OK : XKV_ERR_CUDA;
 }

@@ -15,6 +15,8 @@
 namespace xkv {
 
 static __device__ int g_device_status;
+// Where xkv_get_device_status's exchange kernel leaves the value it took out.
+static __device__ int g_device_status_taken;
 
 // Scratch of xkv_sr_attention_decode_noalloc: a fixed device array that is part
 // of the loaded module, so that entry point never allocates.
@@ -22,7 +24,6 @@ static __device__ __align__(256) unsigned char g_sr_static_scratch[XKV_SR_STATIC
 
 namespace {
 constexpr int kMaxDevices = 64;
-int* g_status_ptr[kMaxDevices] = {nullptr};
 int g_sms[kMaxDevices] = {0};
 std::mutex g_mu;
 
@@ -30,37 +31,70 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 EncodeTiledFn g_encode = nullptr;
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+CtxGetCurrentFn g_ctx_current = nullptr;
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 inline bool aligned256(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 255u) == 0; }
+
+// Device addresses of the module's __device__ symbols, looked up with
+// cudaGetSymbolAddress once per (device, context) with that device current.
+// A context created after cudaDeviceReset holds a freshly loaded module, so
+// the addresses are looked up again for it.
+struct SymbolCache {
+  CUcontext ctx = nullptr;
+  bool valid = false;
+  int* status = nullptr;
+  int* status_taken = nullptr;
+  void* scratch = nullptr;
+};
+SymbolCache g_sym[kMaxDevices];
+
+const SymbolCache* symbols() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_ctx_current) {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || !fn)
+      return nullptr;
+    g_ctx_current = reinterpret_cast<CtxGetCurrentFn>(fn);
+  }
+  // no context is current before the runtime's first call on this thread
+  CUcontext ctx = nullptr;
+  if (g_ctx_current(&ctx) != CUDA_SUCCESS) return nullptr;
+  SymbolCache& c = g_sym[dev];
+  if (!ctx || !c.valid || c.ctx != ctx) {
+    void* a = nullptr;
+    void* b = nullptr;
+    void* sc = nullptr;
+    // (the first lookup also makes the device's primary context current)
+    if (cudaGetSymbolAddress(&a, g_device_status) != cudaSuccess ||
+        cudaGetSymbolAddress(&b, g_device_status_taken) != cudaSuccess ||
+        cudaGetSymbolAddress(&sc, g_sr_static_scratch) != cudaSuccess)
+      return nullptr;
+    if (g_ctx_current(&ctx) != CUDA_SUCCESS || !ctx) return nullptr;
+    c.status = static_cast<int*>(a);
+    c.status_taken = static_cast<int*>(b);
+    c.scratch = sc;
+    c.ctx = ctx;
+    c.valid = true;
+  }
+  return &c;
+}
 }  // namespace
 
 int* device_status_ptr() {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
-  std::lock_guard<std::mutex> lk(g_mu);
-  if (!g_status_ptr[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess) return nullptr;
-    g_status_ptr[dev] = static_cast<int*>(p);
-  }
-  return g_status_ptr[dev];
+  const SymbolCache* c = symbols();
+  return c ? c->status : nullptr;
 }
 
-void* g_scratch_ptr[kMaxDevices] = {nullptr};
-
-// Device address of g_sr_static_scratch on the current device, looked up once
-// per device (with that device current) and cached.
+// Device address of g_sr_static_scratch on the current device and context.
 void* static_scratch_ptr() {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
-  std::lock_guard<std::mutex> lk(g_mu);
-  if (!g_scratch_ptr[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_sr_static_scratch) != cudaSuccess) return nullptr;
-    g_scratch_ptr[dev] = p;
-  }
-  return g_scratch_ptr[dev];
+  const SymbolCache* c = symbols();
+  return c ? c->scratch : nullptr;
 }
 
 int num_sms() {
@@ -132,17 +166,22 @@ const char* xkv_status_string(xkv_status s) {
 
 int xkv_version(void) { return (1 << 16) | 0; }
 
+// Takes the status word out and leaves 0 in one atomic step, so that a code
+// recorded by a kernel on another stream is either returned now or kept for
+// the next call, never lost between a read and a clear.
+__global__ void take_status_kernel(int* status, int* taken) { *taken = atomicExch(status, 0); }
+
 xkv_status xkv_get_device_status(void* stream) {
-  int* p = device_status_ptr();
-  if (!p) return XKV_ERR_CUDA;
+  const SymbolCache* c = symbols();
+  if (!c) return XKV_ERR_CUDA;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  int v = 0;
   if (cudaStreamSynchronize(st) != cudaSuccess) return XKV_ERR_CUDA;
-  if (cudaMemcpy(&v, p, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return XKV_ERR_CUDA;
-  if (v != 0) {
-    const int zero = 0;
-    if (cudaMemcpy(p, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) return XKV_ERR_CUDA;
-  }
+  take_status_kernel<<<1, 1, 0, st>>>(c->status, c->status_taken);
+  if (cudaPeekAtLastError() != cudaSuccess) return XKV_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyAsync(&v, c->status_taken, sizeof(int), cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    return XKV_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return XKV_ERR_CUDA;
   return static_cast<xkv_status>(v);
 }
 
@@ -233,6 +272,66 @@ xkv_status xkv_compress_group(const void* const* X_layers, int G, int64_t T, int
   if (!workspace || ws_bytes < p.bytes || !aligned256(workspace)) return XKV_ERR_WORKSPACE;
   return compress_launch(p, X_layers, G, T, d, ldx, dt, iters, seed, A, Bt, eigvals, gram_out, workspace,
                          static_cast<cudaStream_t>(stream));
+}
+
+// ------------------------------------------------- factorisation pieces
+static xkv_status check_factor(int G, int d, int64_t rows, int rank, int iters, int oversample, xkv_dtype dt) {
+  if (G < 1 || G > 8 || d < 64 || d % 64 != 0 || rows < 1 || rank < 1 || rank % 16 != 0 || iters < 1 ||
+      oversample < 0)
+    return XKV_ERR_INVALID_ARG;
+  if (rank > G * d || rank > rows) return XKV_ERR_INVALID_ARG;
+  if (dt != XKV_F32 && dt != XKV_BF16) return XKV_ERR_INVALID_ARG;
+  const int64_t b = std::min<int64_t>(std::min<int64_t>(static_cast<int64_t>(rank) + oversample, int64_t(G) * d), rows);
+  if (b > 3584) return XKV_ERR_UNSUPPORTED;
+  return XKV_OK;
+}
+
+xkv_status xkv_factor_workspace_size(int G, int d, int64_t rows, int rank, int oversample, xkv_dtype dt,
+                                     size_t* bytes) {
+  if (!bytes) return XKV_ERR_INVALID_ARG;
+  const xkv_status s = check_factor(G, d, rows, rank, 1, oversample, dt);
+  if (s != XKV_OK) return s;
+  FactorPlan p;
+  factor_plan(G * d, rows, rank, oversample, &p);
+  *bytes = p.bytes;
+  return XKV_OK;
+}
+
+xkv_status xkv_factor_gram(const float* gram, int G, int d, int64_t rows, xkv_dtype dt, int rank, int iters,
+                           int oversample, uint64_t seed, void* Bt, float* Vr_out, float* eigvals, void* workspace,
+                           size_t ws_bytes, void* stream) {
+  const xkv_status s = check_factor(G, d, rows, rank, iters, oversample, dt);
+  if (s != XKV_OK) return s;
+  if (!gram || !Bt || !aligned16(gram) || !aligned16(Bt)) return XKV_ERR_INVALID_ARG;
+  if ((Vr_out && !aligned16(Vr_out)) || (eigvals && !aligned16(eigvals))) return XKV_ERR_INVALID_ARG;
+  FactorPlan p;
+  factor_plan(G * d, rows, rank, oversample, &p);
+  if (!workspace || ws_bytes < p.bytes || !aligned256(workspace)) return XKV_ERR_WORKSPACE;
+  return factor_launch(p, gram, dt, iters, seed, Bt, Vr_out, eigvals, workspace, static_cast<cudaStream_t>(stream));
+}
+
+xkv_status xkv_project_workspace_size(int G, int d, int rank, size_t* bytes) {
+  if (!bytes || G < 1 || G > 8 || d < 64 || d % 64 != 0 || rank < 1) return XKV_ERR_INVALID_ARG;
+  *bytes = project_workspace(G * d, rank);
+  return XKV_OK;
+}
+
+xkv_status xkv_project(const void* const* X_layers, int G, int64_t T, int d, int64_t ldx, xkv_dtype dt,
+                       const void* V, xkv_dtype v_dtype, int rank, void* A, int64_t lda, void* workspace,
+                       size_t ws_bytes, void* stream) {
+  xkv_status s = check_layers(X_layers, G, d, ldx, dt);
+  if (s != XKV_OK) return s;
+  if (!V || !A || !aligned16(V) || !aligned16(A) || T < 0 || rank < 1 || rank > G * d || lda < rank ||
+      (v_dtype != XKV_F32 && v_dtype != XKV_BF16))
+    return XKV_ERR_INVALID_ARG;
+  if (T > (int64_t(1) << 31) - 1) return XKV_ERR_UNSUPPORTED;
+  const bool tc = project_tc_ok(d, rank, dt);
+  if (!tc && !(dt == XKV_F32 && v_dtype == XKV_F32)) return XKV_ERR_UNSUPPORTED;
+  if (tc && lda % 8 != 0) return XKV_ERR_INVALID_ARG;
+  if (tc && (!workspace || ws_bytes < project_workspace(G * d, rank) || !aligned256(workspace)))
+    return XKV_ERR_WORKSPACE;
+  return project_launch(X_layers, G, T, d, ldx, dt, V, v_dtype, rank, A, lda, workspace,
+                        static_cast<cudaStream_t>(stream));
 }
 
 // -------------------------------------------------------------- landmarks

@@ -118,6 +118,17 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* s
   }
 }
 
+// After an abort: wait (bounded) for the last phases armed on a ring of
+// `nslots` full barriers, `armed` phases having been armed in all, so that
+// every asynchronous copy the producer issued has landed before the CTA gives
+// up its shared memory.  The phase of use i of slot i % nslots has parity
+// (i / nslots) & 1, and no later phase of a slot is armed.
+__device__ inline void drain_ring(uint64_t* full, int nslots, uint32_t armed, int* status) {
+  const uint32_t n = static_cast<uint32_t>(nslots);
+  for (uint32_t i = armed > n ? armed - n : 0u; i < armed; ++i)
+    (void)mbar_wait(&full[i % n], (i / n) & 1u, status);
+}
+
 // ----------------------------------------------------------------- TMA
 __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* map, uint64_t* bar, int x,
                                             int y) {

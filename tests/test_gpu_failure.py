@@ -1,7 +1,8 @@
 """Failure detection on the GPU without a fault: a device-side wait that
 nothing completes runs out after the library's limit, the kernel returns, the
 status word reports XKV_ERR_DEVICE_TIMEOUT (cleared on read), and the context
-keeps working (an SR decode afterwards matches the oracle)."""
+keeps working (an SR decode afterwards matches the oracle).  An eigen-solve
+stopped before convergence is reported as XKV_ERR_NUMERICAL."""
 import time
 
 import numpy as np
@@ -29,3 +30,42 @@ def test_expired_wait_is_reported_and_the_context_stays_usable(xkv):
     assert xkv.get_device_status() == xkv.XKV_OK
     ref, _, _ = oracle.sr_decode(w, sel_in=sel.cpu().numpy(), **inp)
     assert np.abs(host(out) - ref).max() <= 2e-4
+
+
+_JACOBI_SCRIPT = r"""
+import sys
+sys.path.insert(0, {root!r})
+import torch
+import cross_layer_rank_b200 as xkv
+import synth
+w = synth.WORKLOADS["tiny_f32"]
+X = [torch.from_numpy(l).cuda() for l in synth.kv_group(w, 0, 0, "K")]
+n = 4 * w.d
+C = torch.zeros((n, n), dtype=torch.float32, device="cuda")
+xkv.xkv_gram_accumulate(X, C)
+ner = torch.empty(4, dtype=torch.float32, device="cuda")
+xkv.xkv_ner(C, w.d, ner)
+print(xkv.get_device_status(), xkv.get_device_status())
+"""
+
+
+@pytest.mark.parametrize("cap, expect", [("1", 5), ("", 0)])
+def test_unconverged_eigensolver_is_reported(xkv, cap, expect):
+    # the eigen-solver's sweep limit cut to one sweep (a diagnostic override
+    # read once per process, hence the child process) leaves the NER spectra
+    # unconverged: the device status reports XKV_ERR_NUMERICAL once, then 0;
+    # with the default limit nothing is reported
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ)
+    env.pop("XKV_JACOBI_MAX_SWEEPS", None)
+    if cap:
+        env["XKV_JACOBI_MAX_SWEEPS"] = cap
+    r = subprocess.run([sys.executable, "-c", _JACOBI_SCRIPT.format(root=root)], env=env, capture_output=True,
+                       text=True, timeout=600)
+    assert r.returncode == 0, r.stderr
+    first, second = (int(x) for x in r.stdout.split())
+    assert (first, second) == (expect, 0)
+    assert expect in (0, xkv.XKV_ERR_NUMERICAL)
