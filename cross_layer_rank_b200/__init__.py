@@ -35,6 +35,7 @@ EXPORTS = (
     "xkv_status_string", "xkv_version", "xkv_get_device_status",
     "xkv_gram_workspace_size", "xkv_gram_accumulate",
     "xkv_compress_workspace_size", "xkv_compress_group",
+    "xkv_factor_workspace_size", "xkv_factor_gram", "xkv_project_workspace_size", "xkv_project",
     "xkv_build_landmarks",
     "xkv_sr_workspace_size", "xkv_sr_attention_decode",
     "xkv_sr_attention_decode_noalloc",
@@ -83,6 +84,12 @@ def _load():
                                                   C.POINTER(sz)]),
         "xkv_compress_group": (C.c_int, [vp, C.c_int, i64, C.c_int, i64, C.c_int, C.c_int, C.c_int, C.c_int, i64,
                                          C.c_uint64, vp, vp, vp, vp, vp, sz, vp]),
+        "xkv_factor_workspace_size": (C.c_int, [C.c_int, C.c_int, i64, C.c_int, C.c_int, C.c_int, C.POINTER(sz)]),
+        "xkv_factor_gram": (C.c_int, [vp, C.c_int, C.c_int, i64, C.c_int, C.c_int, C.c_int, C.c_int, C.c_uint64,
+                                      vp, vp, vp, vp, sz, vp]),
+        "xkv_project_workspace_size": (C.c_int, [C.c_int, C.c_int, C.c_int, C.POINTER(sz)]),
+        "xkv_project": (C.c_int, [vp, C.c_int, i64, C.c_int, i64, C.c_int, vp, C.c_int, C.c_int, vp, i64, vp, sz,
+                                  vp]),
         "xkv_build_landmarks": (C.c_int, [vp, i64, i64, C.c_int, C.c_int, C.c_int, C.c_int, C.c_int, C.c_int,
                                           C.c_float, vp, vp]),
         "xkv_sr_workspace_size": (C.c_int, [C.POINTER(SRParams), C.POINTER(sz)]),
@@ -204,6 +211,43 @@ def xkv_compress_group(layers: Sequence[torch.Tensor], rank: int, A: torch.Tenso
     _check(lib.xkv_compress_group(ptrs, G, T, d, ldx, dt, rank, iters, oversample, shard_rows, seed, _ptr(A),
                                   _ptr(Bt), _ptr(eigvals), _ptr(gram_out), _ptr(ws), ws.numel(), _stream(stream)),
            "xkv_compress_group")
+
+
+def xkv_factor_workspace_size(G, d, rows, rank, oversample, dtype: torch.dtype) -> int:
+    return _wsize(lib.xkv_factor_workspace_size, G, d, rows, rank, oversample, dtype_code(dtype))
+
+
+def xkv_factor_gram(gram: torch.Tensor, G: int, d: int, rows: int, rank: int, Bt: torch.Tensor,
+                    iters: int = 8, oversample: int = 64, seed: int = 0x784B56, Vr_out: Optional[torch.Tensor] = None,
+                    eigvals: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None, stream=None):
+    """Top-r basis of a given (G d)^2 f32 Gram: Bt (G d x rank, Bt's dtype), optional f32 V_r and Ritz values."""
+    nbytes = xkv_factor_workspace_size(G, d, rows, rank, oversample, Bt.dtype)
+    ws = ws if ws is not None else workspace(nbytes, gram.device)
+    _check(lib.xkv_factor_gram(_ptr(gram), G, d, rows, dtype_code(Bt.dtype), rank, iters, oversample, seed, _ptr(Bt),
+                               _ptr(Vr_out), _ptr(eigvals), _ptr(ws), ws.numel(), _stream(stream)), "xkv_factor_gram")
+
+
+def xkv_project_workspace_size(G, d, rank) -> int:
+    return _wsize(lib.xkv_project_workspace_size, G, d, rank)
+
+
+def xkv_project(layers: Sequence[torch.Tensor], V: torch.Tensor, A: torch.Tensor, ws: Optional[torch.Tensor] = None,
+                stream=None):
+    """A = [layers...] V; A may be a row-strided view (rows of rank elements)."""
+    G = len(layers)
+    T, d = layers[0].shape
+    ldx = layers[0].stride(0)
+    for t in layers:
+        if t.shape != layers[0].shape or t.stride(0) != ldx or t.stride(1) != 1:
+            raise ValueError("layers must share shape and row stride")
+    rank = V.shape[1]
+    if A.shape[-1] != rank or A.stride(-1) != 1 or not A.is_cuda:
+        raise ValueError("A must be T x rank with contiguous rows")
+    ws = ws if ws is not None else workspace(xkv_project_workspace_size(G, d, rank), layers[0].device)
+    ptrs = (C.c_void_p * G)(*[t.data_ptr() for t in layers])
+    _check(lib.xkv_project(ptrs, G, T, d, ldx, dtype_code(layers[0].dtype), _ptr(V), dtype_code(V.dtype), rank,
+                           C.c_void_p(A.data_ptr()), A.stride(0), _ptr(ws), ws.numel(), _stream(stream)),
+           "xkv_project")
 
 
 # -------------------------------------------------------------- landmarks

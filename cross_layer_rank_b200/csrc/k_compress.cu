@@ -483,22 +483,19 @@ xkv_status gram_launch(const void* const* X, int G, int64_t rows, int d, int64_t
   return cudaPeekAtLastError() == cudaSuccess ? XKV_OK : XKV_ERR_CUDA;
 }
 
-xkv_status compress_plan(int G, int64_t T, int d, int rank, int oversample, int64_t shard_rows, xkv_dtype dt,
-                         CompressPlan* p) {
-  const int n = G * d;
-  int64_t b = std::min<int64_t>(std::min<int64_t>(static_cast<int64_t>(rank) + std::max(oversample, 0), n), T);
+// ---------------------------------------------------------- factorisation
+// Block width of the subspace iteration: b = min(rank + oversample, G d, rows).
+xkv_status factor_plan(int n, int64_t rows, int rank, int oversample, FactorPlan* p) {
+  const int64_t b = std::min<int64_t>(std::min<int64_t>(static_cast<int64_t>(rank) + std::max(oversample, 0), n), rows);
   p->n = n;
   p->b = static_cast<int>(b);
   p->rank = rank;
-  p->shard = shard_rows > 0 ? std::min<int64_t>(shard_rows, T) : T;
   size_t off = 0;
   auto take = [&](size_t bytes) {
     const size_t o = off;
     off = align_up(off + bytes);
     return o;
   };
-  p->off_gram = take(static_cast<size_t>(n) * n * 4);
-  p->off_gramws = take(gram_workspace(G, p->shard, d, dt));
   p->off_Q = take(static_cast<size_t>(n) * b * 4);
   p->off_Y = take(static_cast<size_t>(n) * b * 4);
   p->off_W = take(static_cast<size_t>(b) * b * 8);
@@ -506,21 +503,20 @@ xkv_status compress_plan(int G, int64_t T, int d, int rank, int oversample, int6
   p->off_U = take(static_cast<size_t>(b) * b * 8);
   p->off_lam = take(static_cast<size_t>(b) * 8 + 64);
   p->off_ord = take(static_cast<size_t>(b) * 4);
-  p->off_V = take(static_cast<size_t>(b) * rank * 4);  // Ur
+  p->off_Ur = take(static_cast<size_t>(b) * rank * 4);
   p->off_Vr = take(static_cast<size_t>(n) * rank * 4);
-  p->off_Vt = take(static_cast<size_t>(2) * rank * n * 2);
   p->off_jac = take(jacobi_workspace(static_cast<int>(b), 1));
   p->bytes = off;
   return XKV_OK;
 }
 
-xkv_status compress_launch(const CompressPlan& P, const void* const* X, int G, int64_t T, int d, int64_t ldx,
-                           xkv_dtype dt, int iters, uint64_t seed, void* A, void* Bt, float* eigvals,
-                           float* gram_out, void* ws, cudaStream_t st) {
+// Steps 2 of the factorisation on a given Gram C (n x n f32): subspace
+// iteration, Rayleigh-Ritz, V_r (f32, left in the workspace and optionally
+// copied to Vr_out), the Ritz values, and Bt = V_r in the cache dtype.
+xkv_status factor_launch(const FactorPlan& P, const float* C, xkv_dtype dt, int iters, uint64_t seed, void* Bt,
+                         float* Vr_out, float* eigvals, void* ws, cudaStream_t st) {
   uint8_t* w = static_cast<uint8_t*>(ws);
   const int n = P.n, b = P.b, r = P.rank;
-  const size_t es = dt == XKV_BF16 ? 2 : 4;
-  float* C = gram_out ? gram_out : reinterpret_cast<float*>(w + P.off_gram);
   float* Q = reinterpret_cast<float*>(w + P.off_Q);
   float* Y = reinterpret_cast<float*>(w + P.off_Y);
   double* W = reinterpret_cast<double*>(w + P.off_W);
@@ -529,23 +525,10 @@ xkv_status compress_launch(const CompressPlan& P, const void* const* X, int G, i
   double* lam = reinterpret_cast<double*>(w + P.off_lam);
   double* scal = lam + b;
   int* order = reinterpret_cast<int*>(w + P.off_ord);
-  float* Ur = reinterpret_cast<float*>(w + P.off_V);
+  float* Ur = reinterpret_cast<float*>(w + P.off_Ur);
   float* Vr = reinterpret_cast<float*>(w + P.off_Vr);
-  __nv_bfloat16* vhi = reinterpret_cast<__nv_bfloat16*>(w + P.off_Vt);
-  __nv_bfloat16* vlo = vhi + static_cast<int64_t>(r) * n;
   int* status = device_status_ptr();
-  xkv_status s;
-
-  // 1. Gram over token shards
-  if (cudaMemsetAsync(C, 0, static_cast<size_t>(n) * n * 4, st) != cudaSuccess) return XKV_ERR_CUDA;
-  for (int64_t t0 = 0; t0 < T; t0 += P.shard) {
-    const int64_t rows = std::min<int64_t>(P.shard, T - t0);
-    const void* Xs[8];
-    for (int l = 0; l < G; ++l) Xs[l] = static_cast<const uint8_t*>(X[l]) + t0 * ldx * es;
-    s = gram_launch(Xs, G, rows, d, ldx, dt, C, w + P.off_gramws, st);
-    if (s != XKV_OK) return s;
-  }
-  // 2. block subspace iteration
+  if (!status) return XKV_ERR_CUDA;
   gaussian_kernel<<<256, 256, 0, st>>>(Y, static_cast<int64_t>(n) * b, seed);
   auto orthonormalise = [&](float* src) {
     // shifted pass (robust to a rank-deficient block), then a plain pass
@@ -561,19 +544,59 @@ xkv_status compress_launch(const CompressPlan& P, const void* const* X, int G, i
   // Rayleigh-Ritz
   gemm_simt<float, float, float, float>(C, n, 1, Q, b, 1, Y, b, n, b, n, 1.0, 0.0, st);
   gemm_simt<float, float, double, double>(Q, 1, b, Y, b, 1, H, b, b, b, n, 1.0, 0.0, st);
-  s = jacobi_launch(H, U, lam, b, 1, w + P.off_jac, st);
+  xkv_status s = jacobi_launch(H, U, lam, b, 1, w + P.off_jac, st);
   if (s != XKV_OK) return s;
   order_desc(lam, b, order, st);
   gather_ritz_kernel<<<64, 256, 0, st>>>(U, order, b, r, Ur, lam, eigvals);
   gemm_simt<float, float, float, float>(Q, b, 1, Ur, r, 1, Vr, r, n, r, b, 1.0, 0.0, st);
-  // 3. factors
-  const bool tc = dt == XKV_BF16 && r % 64 == 0 && d % 64 == 0 && !force_simt();
   if (dt == XKV_BF16)
-    emit_factors_kernel<__nv_bfloat16><<<256, 256, 0, st>>>(Vr, n, r, static_cast<__nv_bfloat16*>(Bt), tc ? vhi : nullptr,
-                                                            vlo);
+    emit_factors_kernel<__nv_bfloat16><<<256, 256, 0, st>>>(Vr, n, r, static_cast<__nv_bfloat16*>(Bt), nullptr,
+                                                            nullptr);
   else
     emit_factors_kernel<float><<<256, 256, 0, st>>>(Vr, n, r, static_cast<float*>(Bt), nullptr, nullptr);
-  if (tc) {
+  if (Vr_out && cudaMemcpyAsync(Vr_out, Vr, static_cast<size_t>(n) * r * 4, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+    return XKV_ERR_CUDA;
+  return cudaPeekAtLastError() == cudaSuccess ? XKV_OK : XKV_ERR_CUDA;
+}
+
+// ------------------------------------------------------------- projection
+bool project_tc_ok(int d, int rank, xkv_dtype dt) { return dt == XKV_BF16 && rank % 64 == 0 && d % 64 == 0 && !force_simt(); }
+
+size_t project_workspace(int n, int rank) { return align_up(static_cast<size_t>(2) * rank * n * 2); }
+
+// V (n x rank, f32 or bf16) -> Vt hi (and lo for f32) (rank x n bf16)
+template <typename TV>
+__global__ void split_basis_kernel(const TV* __restrict__ V, int n, int r, __nv_bfloat16* __restrict__ vhi,
+                                   __nv_bfloat16* __restrict__ vlo) {
+  const int64_t total = static_cast<int64_t>(n) * r;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const float v = to_f(V[i]);
+    const int k = static_cast<int>(i / r), c = static_cast<int>(i % r);
+    const __nv_bfloat16 h = __float2bfloat16_rn(v);
+    vhi[static_cast<int64_t>(c) * n + k] = h;
+    if (vlo) vlo[static_cast<int64_t>(c) * n + k] = __float2bfloat16_rn(v - __bfloat162float(h));
+  }
+}
+
+// A (T x rank, row stride lda) = X V, X = [X_1 | ... | X_G] through the layer
+// pointers.  bf16 caches: tcgen05 GEMM; an f32 basis is split into a bf16
+// hi/lo pair (two products per step keep ~16 significant bits), a bf16 basis
+// is used as is.  f32 caches: CUDA-core GEMM per layer (f32 basis only).
+xkv_status project_launch(const void* const* X, int G, int64_t T, int d, int64_t ldx, xkv_dtype dt, const void* V,
+                          xkv_dtype v_dt, int r, void* A, int64_t lda, void* ws, cudaStream_t st) {
+  const int n = G * d;
+  if (T <= 0) return XKV_OK;
+  int* status = device_status_ptr();
+  if (!status) return XKV_ERR_CUDA;
+  if (project_tc_ok(d, r, dt)) {
+    __nv_bfloat16* vhi = static_cast<__nv_bfloat16*>(ws);
+    __nv_bfloat16* vlo = vhi + static_cast<int64_t>(r) * n;
+    const bool two = v_dt == XKV_F32;
+    if (two)
+      split_basis_kernel<float><<<256, 256, 0, st>>>(static_cast<const float*>(V), n, r, vhi, vlo);
+    else
+      split_basis_kernel<__nv_bfloat16><<<256, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(V), n, r, vhi, nullptr);
     TmapSet am;
     CUtensorMap bh, bl;
     for (int l = 0; l < G; ++l) {
@@ -596,22 +619,68 @@ xkv_status compress_launch(const CompressPlan& P, const void* const* X, int G, i
     g.K = n;
     g.bn = bn;
     g.layer_cols = d;
+    g.two_b = two ? 1 : 0;
     g.out = A;
-    g.ldo = r;
+    g.ldo = lda;
     g.status = status;
     const size_t smem = gemm_smem_bytes<kProj>();
     cudaFuncSetAttribute(gemm_tc_kernel<kProj>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     dim3 grid(static_cast<unsigned>((T + 127) / 128), r / bn);
     gemm_tc_kernel<kProj><<<grid, kGemmThreads, smem, st>>>(am, bh, bl, g);
-  } else if (dt == XKV_F32) {
+  } else if (dt == XKV_F32 && v_dt == XKV_F32) {
+    const float* Vf = static_cast<const float*>(V);
     for (int l = 0; l < G; ++l)
-      gemm_simt<float, float, float, float>(static_cast<const float*>(X[l]), ldx, 1, Vr + static_cast<int64_t>(l) * d * r,
-                                            r, 1, static_cast<float*>(A), r, static_cast<int>(T), r, d, 1.0,
+      gemm_simt<float, float, float, float>(static_cast<const float*>(X[l]), ldx, 1, Vf + static_cast<int64_t>(l) * d * r,
+                                            r, 1, static_cast<float*>(A), lda, static_cast<int>(T), r, d, 1.0,
                                             l > 0 ? 1.0 : 0.0, st);
   } else {
     return XKV_ERR_UNSUPPORTED;
   }
   return cudaPeekAtLastError() == cudaSuccess ? XKV_OK : XKV_ERR_CUDA;
+}
+
+// ------------------------------------------------------------ whole group
+xkv_status compress_plan(int G, int64_t T, int d, int rank, int oversample, int64_t shard_rows, xkv_dtype dt,
+                         CompressPlan* p) {
+  const int n = G * d;
+  factor_plan(n, T, rank, oversample, &p->f);
+  p->shard = shard_rows > 0 ? std::min<int64_t>(shard_rows, T) : T;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = align_up(off + bytes);
+    return o;
+  };
+  p->off_gram = take(static_cast<size_t>(n) * n * 4);
+  p->off_gramws = take(gram_workspace(G, p->shard, d, dt));
+  p->off_factor = take(p->f.bytes);
+  p->off_proj = take(project_workspace(n, rank));
+  p->bytes = off;
+  return XKV_OK;
+}
+
+xkv_status compress_launch(const CompressPlan& P, const void* const* X, int G, int64_t T, int d, int64_t ldx,
+                           xkv_dtype dt, int iters, uint64_t seed, void* A, void* Bt, float* eigvals,
+                           float* gram_out, void* ws, cudaStream_t st) {
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  const int n = P.f.n, r = P.f.rank;
+  const size_t es = dt == XKV_BF16 ? 2 : 4;
+  float* C = gram_out ? gram_out : reinterpret_cast<float*>(w + P.off_gram);
+  // 1. Gram over token shards
+  if (cudaMemsetAsync(C, 0, static_cast<size_t>(n) * n * 4, st) != cudaSuccess) return XKV_ERR_CUDA;
+  for (int64_t t0 = 0; t0 < T; t0 += P.shard) {
+    const int64_t rows = std::min<int64_t>(P.shard, T - t0);
+    const void* Xs[8];
+    for (int l = 0; l < G; ++l) Xs[l] = static_cast<const uint8_t*>(X[l]) + t0 * ldx * es;
+    const xkv_status s = gram_launch(Xs, G, rows, d, ldx, dt, C, w + P.off_gramws, st);
+    if (s != XKV_OK) return s;
+  }
+  // 2. top-r subspace, Ritz values, Bt
+  xkv_status s = factor_launch(P.f, C, dt, iters, seed, Bt, nullptr, eigvals, w + P.off_factor, st);
+  if (s != XKV_OK) return s;
+  // 3. A = X V_r from the f32 basis left in the factor workspace
+  const float* Vr = reinterpret_cast<const float*>(w + P.off_factor + P.f.off_Vr);
+  return project_launch(X, G, T, d, ldx, dt, Vr, XKV_F32, r, A, r, w + P.off_proj, st);
 }
 
 }  // namespace xkv

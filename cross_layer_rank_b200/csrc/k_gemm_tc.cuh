@@ -4,8 +4,8 @@
 // issues tcgen05.mma, warps 2..5 drain TMEM through a mode-specific epilogue:
 //   kRecon : bf16 store of A Bt^T with optional RoPE per head (position = row)
 //   kProj  : A operand split over up to 8 layer tensor maps along K; B given
-//            as a bf16 hi/lo pair (two MMAs per step) for ~16-bit coefficients;
-//            bf16 store
+//            as a bf16 hi/lo pair (two MMAs per step) for ~16-bit coefficients,
+//            or as one bf16 operand; bf16 store with row stride ldo
 #pragma once
 
 #include "xkv_common.cuh"
@@ -22,6 +22,7 @@ struct GemmArgs {
   int M, N, K;          // K multiple of 64
   int bn;               // 64 or 128
   int layer_cols;       // kProj: columns per layer map (d)
+  int two_b;            // kProj: B given as a hi/lo pair (1) or a single bf16 operand (0)
   void* out;            // bf16 [M][ldo]
   int64_t ldo;
   int hd;               // kRecon RoPE head size (0 = no RoPE)
@@ -81,7 +82,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
   if (warp == 0) {
     if (lane == 0) {
-      const uint32_t bytes = 16384 + (MODE == kProj ? 2 : 1) * g.bn * 128;
+      const uint32_t bytes = 16384 + (MODE == kProj && g.two_b ? 2 : 1) * g.bn * 128;
       for (int a = 0; a < nk; ++a) {
         const int slot = a % kGemmStages;
         if (!mbar_wait(&empty[slot], ((a / kGemmStages) & 1) ^ 1, g.status)) break;
@@ -95,7 +96,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           tma_load_2d(st, &amaps.m[0], &full[slot], a * 64, m0);
         }
         tma_load_2d(st + 16384, &bmap, &full[slot], a * 64, n0);
-        if (MODE == kProj) tma_load_2d(st + 2 * 16384, &bmap_lo, &full[slot], a * 64, n0);
+        if (MODE == kProj && g.two_b) tma_load_2d(st + 2 * 16384, &bmap_lo, &full[slot], a * 64, n0);
       }
     }
   } else if (warp == 1) {
@@ -110,7 +111,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const uint64_t bd = umma_desc_sw128(smem_u32(st + 16384));
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) umma_bf16(tmem, ad + 2 * kk, bd + 2 * kk, idesc, (a | kk) ? 1u : 0u);
-        if (MODE == kProj) {
+        if (MODE == kProj && g.two_b) {
           const uint64_t bl = umma_desc_sw128(smem_u32(st + 2 * 16384));
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) umma_bf16(tmem, ad + 2 * kk, bl + 2 * kk, idesc, 1u);

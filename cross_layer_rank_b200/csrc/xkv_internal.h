@@ -58,11 +58,21 @@ xkv_status landmarks_launch(const void* K, int64_t T, int64_t ldk, int hkv, int 
 size_t gram_workspace(int G, int64_t rows, int d, xkv_dtype dt);
 xkv_status gram_launch(const void* const* X, int G, int64_t rows, int d, int64_t ldx, xkv_dtype dt, float* C,
                        void* ws, cudaStream_t st);
-struct CompressPlan {
+struct FactorPlan {
   int n, b, rank;
+  size_t off_Q, off_Y, off_W, off_H, off_U, off_lam, off_ord, off_Ur, off_Vr, off_jac, bytes;
+};
+xkv_status factor_plan(int n, int64_t rows, int rank, int oversample, FactorPlan* plan);
+xkv_status factor_launch(const FactorPlan& plan, const float* C, xkv_dtype dt, int iters, uint64_t seed, void* Bt,
+                         float* Vr_out, float* eigvals, void* ws, cudaStream_t st);
+bool project_tc_ok(int d, int rank, xkv_dtype dt);
+size_t project_workspace(int n, int rank);
+xkv_status project_launch(const void* const* X, int G, int64_t T, int d, int64_t ldx, xkv_dtype dt, const void* V,
+                          xkv_dtype v_dt, int rank, void* A, int64_t lda, void* ws, cudaStream_t st);
+struct CompressPlan {
+  FactorPlan f;
   int64_t shard;
-  size_t off_gram, off_gramws, off_Q, off_Y, off_W, off_H, off_U, off_V, off_lam, off_ord, off_Vr,
-      off_Vt, off_jac, bytes;
+  size_t off_gram, off_gramws, off_factor, off_proj, bytes;
 };
 xkv_status compress_plan(int G, int64_t T, int d, int rank, int oversample, int64_t shard_rows, xkv_dtype dt,
                          CompressPlan* plan);

@@ -79,7 +79,11 @@ XKV_API const char* xkv_status_string(xkv_status status);
 XKV_API int xkv_version(void);
 
 /* Synchronises `stream`, then returns and clears the calling device's deferred
- * status word (XKV_OK if no device-side error was recorded). */
+ * status word (XKV_OK if no device-side error was recorded).  The word is
+ * taken out and reset to zero in one atomic device operation, so a code that
+ * a kernel on another stream records meanwhile is kept for the next call.
+ * Concurrent calls from several host threads for the same device share one
+ * small device slot for the value taken out; serialise them. */
 XKV_API xkv_status xkv_get_device_status(void* stream);
 
 /* ------------------------------------------------------------------ Gram */
@@ -117,6 +121,38 @@ XKV_API xkv_status xkv_compress_group(const void* const* X_layers, int G, int64_
                               xkv_dtype dt, int rank, int iters, int oversample, int64_t shard_rows,
                               uint64_t seed, void* A, void* Bt, float* eigvals, float* gram_out,
                               void* workspace, size_t ws_bytes, void* stream);
+
+/* The two halves of xkv_compress_group, for callers that accumulate the Gram
+ * themselves (e.g. over token shards held by several GPUs, whose partial Grams
+ * are summed by an all-reduce, [KV-CoRE] 2.A) or that project rows onto an
+ * existing basis (e.g. a chunk of generated tokens leaving the raw window).
+ *
+ * xkv_factor_gram: steps 2 of xkv_compress_group on a given Gram.
+ *   gram    : (G d) x (G d) f32, the uncentred Gram of `rows` token rows
+ *             (rows only caps the block width: b = min(rank + oversample, G d,
+ *             rows)).
+ *   Bt      : (G d) x rank in `dt`, the stored basis V_r.
+ *   Vr_out  : (G d) x rank f32 copy of V_r (may be NULL).
+ *   eigvals : rank f32 Ritz values, descending (may be NULL).
+ *   Same seed and Gram give the same bits, so ranks that factor one summed
+ *   Gram obtain one basis.  Argument rules as for xkv_compress_group.
+ *
+ * xkv_project: A = X V for X = [X_1 | ... | X_G] (T x G d through the layer
+ *   pointers, as for xkv_gram_accumulate) and V ((G d) x rank) in v_dtype:
+ *   an f32 basis enters the bf16 tensor-core product as a bf16 hi/lo pair,
+ *   a bf16 basis (e.g. a stored Bt) as is.  A is T x rank in `dt` with row
+ *   stride lda (elements; a multiple of 8 for bf16).  bf16 caches need
+ *   rank % 64 == 0; f32 caches need an f32 basis (XKV_ERR_UNSUPPORTED
+ *   otherwise).  Workspace: xkv_project_workspace_size (bf16 caches only). */
+XKV_API xkv_status xkv_factor_workspace_size(int G, int d, int64_t rows, int rank, int oversample, xkv_dtype dt,
+                                     size_t* bytes);
+XKV_API xkv_status xkv_factor_gram(const float* gram, int G, int d, int64_t rows, xkv_dtype dt, int rank,
+                           int iters, int oversample, uint64_t seed, void* Bt, float* Vr_out,
+                           float* eigvals, void* workspace, size_t ws_bytes, void* stream);
+XKV_API xkv_status xkv_project_workspace_size(int G, int d, int rank, size_t* bytes);
+XKV_API xkv_status xkv_project(const void* const* X_layers, int G, int64_t T, int d, int64_t ldx, xkv_dtype dt,
+                       const void* V, xkv_dtype v_dtype, int rank, void* A, int64_t lda, void* workspace,
+                       size_t ws_bytes, void* stream);
 
 /* ------------------------------------------------------------ landmarks */
 /* Chunk landmarks for the top-k selector of [xKV-blog] "选择性重建": for KV head
@@ -176,9 +212,10 @@ XKV_API xkv_status xkv_sr_attention_decode(const xkv_sr_params* p, const void* q
  * its own, or a decode loop that must run under a fixed memory budget.
  *   - Requests whose scratch (xkv_sr_workspace_size) exceeds the array return
  *     XKV_ERR_UNSUPPORTED and launch nothing.
- *   - The array's device address is looked up once per device, on the first
- *     call made with that device current; make that first call before any
- *     stream capture that includes this entry point.
+ *   - The array's device address is looked up once per device and CUDA
+ *     context, on the first call made with that device current (after
+ *     cudaDeviceReset the new context's module is looked up afresh); make that
+ *     first call before any stream capture that includes this entry point.
  *   - Nothing in the scratch needs to start at zero: every word the kernels
  *     read is written earlier in the same call.
  *   - Every call on a device shares the one array: calls that overlap in time
