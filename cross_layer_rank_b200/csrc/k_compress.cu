@@ -204,6 +204,7 @@ __global__ void __launch_bounds__(kGramThreads, 1)
     for (int c = 0; c < nchunks; ++c) {
       const int buf = c & 1;
       if (!mbar_wait(&accfull[buf], (c >> 1) & 1, status)) { ok = false; break; }
+      __syncwarp();  // converged for the warp-wide tcgen05.ld
       tc_fence_after();
       float v[64];
 #pragma unroll
@@ -250,6 +251,10 @@ __global__ void __launch_bounds__(kGramThreads, 1)
       }
     }
   }
+  // lane 0 of the role warps may still be in its loop: reconverge every warp
+  // before the block-wide barrier, so that the barrier cannot complete (and
+  // TMEM be released) while a role thread is still issuing
+  __syncwarp();
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
@@ -348,6 +353,7 @@ __global__ void __launch_bounds__(kGramWThreads, 1)
     for (int c = 0; c < nchunks; ++c) {
       const int buf = c & 1;
       if (!mbar_wait(&accfull[buf], (c >> 1) & 1, status)) { ok = false; break; }
+      __syncwarp();  // converged for the warp-wide tcgen05.ld
       tc_fence_after();
 #pragma unroll
       for (int jb = 0; jb < 4; ++jb) {
@@ -416,6 +422,10 @@ __global__ void __launch_bounds__(kGramWThreads, 1)
       }
     }
   }
+  // lane 0 of the role warps may still be in its loop: reconverge every warp
+  // before the block-wide barrier, so that the barrier cannot complete (and
+  // TMEM be released) while a role thread is still issuing
+  __syncwarp();
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {

@@ -117,7 +117,7 @@ __device__ uint32_t block_exclusive_scan(uint32_t v, uint32_t* warp_tot, uint32_
 template <typename T>
 __global__ void __launch_bounds__(256) sr_score_kernel(const T* __restrict__ q, const T* __restrict__ lm,
                                                        float* __restrict__ scores, int Hq, int Hkv, int hd,
-                                                       int64_t n_mid, int chunks_per_block) {
+                                                       int64_t n_mid, int64_t lm_cap, int chunks_per_block) {
   allow_next_grid();
   __shared__ float qbar[256];
   const int unit = blockIdx.y;
@@ -131,7 +131,7 @@ __global__ void __launch_bounds__(256) sr_score_kernel(const T* __restrict__ q, 
   const int64_t c0 = static_cast<int64_t>(blockIdx.x) * chunks_per_block;
   const int64_t c1 = min(c0 + chunks_per_block, n_mid);
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const T* base = lm + static_cast<int64_t>(unit) * n_mid * hd;
+  const T* base = lm + static_cast<int64_t>(unit) * lm_cap * hd;
   float* out = scores + static_cast<int64_t>(unit) * ((n_mid + 3) & ~int64_t(3));
   if (sizeof(T) == 2 && hd == 128) {
     // 16 lanes x 16 B cover one 256-B landmark row; a warp scores 2 rows per
@@ -213,6 +213,7 @@ struct WinArgs {
   const void* srV;
   float* win;
   int64_t T;
+  int64_t wbs;  // elements between sequences of the raw window
   int Hq, Hkv, hd, sink, recent;
   double ft[128];  // RoPE frequency of pair j in turns per position
 };
@@ -244,7 +245,7 @@ __device__ void window_partial(const WinArgs& wa, int unit, uint8_t* smem) {
     const int vpr = hd / 8;
     for (int v = tid; v < 2 * nsr * vpr; v += nt) {
       const int mat = v / (nsr * vpr), r = (v / vpr) % nsr, c8 = v % vpr;
-      const T* src = (mat ? srV : srK) + (static_cast<int64_t>(b) * nsr + r) * d + h * hd + c8 * 8;
+      const T* src = (mat ? srV : srK) + static_cast<int64_t>(b) * wa.wbs + static_cast<int64_t>(r) * d + h * hd + c8 * 8;
       const uint4 w = *reinterpret_cast<const uint4*>(src);
       float* dst = mat ? wV + r * hd + c8 * 8 : wK + r * ks + c8 * 8;
       const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
@@ -258,7 +259,7 @@ __device__ void window_partial(const WinArgs& wa, int unit, uint8_t* smem) {
   } else {
     for (int i = tid; i < nsr * hd; i += nt) {
       const int r = i / hd, j = i % hd;
-      const int64_t off = (static_cast<int64_t>(b) * nsr + r) * d + h * hd + j;
+      const int64_t off = static_cast<int64_t>(b) * wa.wbs + static_cast<int64_t>(r) * d + h * hd + j;
       wK[r * ks + j] = ldf(srK + off);
       wV[r * hd + j] = ldf(srV + off);
     }
@@ -913,6 +914,17 @@ __global__ void __launch_bounds__(kAttendThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   allow_next_grid();
+  // The first stage's Bt_K atoms depend on the CTA's first unit only, not on
+  // the selection the previous kernel writes: issue them before waiting.
+  int b_pre = 0;
+  if (warp == 12 && lane == 0 && te > tb) {
+    const int u = tb / tpu, b = u / args.Hkv, h = u % args.Hkv;
+    b_pre = min(kKAtoms, NKA);
+    for (int a = 0; a < b_pre; ++a) {
+      mbar_arrive_expect_tx(&bfull[a], kAtomBytes);
+      tma_load_3d(Kb + a * kAtomBytes, &mapBK, &bfull[a], a * 64, h * 128, args.sbk ? b : 0);
+    }
+  }
   wait_prior_grid();  // the selection
 
   if (warp == 12) {
@@ -941,6 +953,7 @@ __global__ void __launch_bounds__(kAttendThreads, 1)
                         sk * kKAtoms, b);
           const int na = min(kKAtoms, NKA - sk * kKAtoms);
           for (int a = 0; a < na; ++a, ++bs) {
+            if (static_cast<int>(bs) < b_pre) continue;  // issued before the wait
             const int bslot = bs % kBStages;
             if (!mbar_wait(&bempty[bslot], ((bs / kBStages) & 1) ^ 1, args.status)) { *abort_flag = 1; ok = false; break; }
             mbar_arrive_expect_tx(&bfull[bslot], kAtomBytes);
@@ -953,7 +966,7 @@ __global__ void __launch_bounds__(kAttendThreads, 1)
       // them before the CTA releases its shared memory
       if (*abort_flag) {
         drain_ring(kfull, kKStages, ks, args.status);
-        drain_ring(bfull, kBStages, bs, args.status);
+        drain_ring(bfull, kBStages, max(bs, static_cast<uint32_t>(b_pre)), args.status);
       }
     }
   } else if (warp == 13) {
@@ -962,6 +975,10 @@ __global__ void __launch_bounds__(kAttendThreads, 1)
     // the first (finite data; its softmax weights are zero)
     if (lane == 0) {
       uint32_t vsn = 0;
+      // values are needed only once the first tile's softmax weights exist:
+      // start after the first key stage has landed, so that the key path's
+      // first loads are not queued behind the value ring's
+      if (te > tb && !mbar_wait(&kfull[0], 0, args.status)) *abort_flag = 1;
       for (int x = tb; x < te && !*abort_flag; ++x) {
         const int u = x / tpu, ti = x % tpu;
         const int b = u / args.Hkv;
@@ -1097,6 +1114,7 @@ __global__ void __launch_bounds__(kAttendThreads, 1)
       const float2* rte = reinterpret_cast<const float2*>(rot_s + e * kRopeStride);
       const int buf = j & 1;
       if (!mbar_wait(&accfull[buf], (j >> 1) & 1, args.status)) { *abort_flag = 1; break; }
+      __syncwarp();  // converged for the warp-wide tcgen05.ld
       tc_fence_after();
       const uint32_t taddr = tmem + (static_cast<uint32_t>(lq * 32) << 16) + buf * 128;
       float s0[GQ], s1[GQ];
@@ -1216,6 +1234,7 @@ __global__ void __launch_bounds__(kAttendThreads, 1)
       }
       const int pb = j & 1;
       if (!mbar_wait(&vaccfull[pb], (j >> 1) & 1, args.status)) { *abort_flag = 1; break; }
+      __syncwarp();  // converged for the warp-wide tcgen05.ld
       tc_fence_after();
       float al[GQ];
 #pragma unroll
@@ -1248,6 +1267,10 @@ __global__ void __launch_bounds__(kAttendThreads, 1)
       }
     }
   }
+  // lane 0 of the role warps may still be in its loop: reconverge every warp
+  // before the block-wide barrier, so that the barrier cannot complete (and
+  // TMEM be released) while a role thread is still issuing
+  __syncwarp();
   tc_fence_before();
   __syncthreads();
   if (warp == 14) {
@@ -1486,8 +1509,9 @@ static xkv_status sr_launch_t(const xkv_sr_params* p, const SRPlan& plan, const 
   {
     const int cpb = 512;
     dim3 grid(static_cast<unsigned>((n_mid + cpb - 1) / cpb), static_cast<unsigned>(plan.units));
+    const int64_t lm_cap = p->landmark_capacity > 0 ? p->landmark_capacity : n_mid;
     sr_score_kernel<T><<<grid, 256, 0, st>>>(static_cast<const T*>(q), static_cast<const T*>(lm), scores,
-                                             p->n_q_heads, p->n_kv_heads, p->head_dim, n_mid, cpb);
+                                             p->n_q_heads, p->n_kv_heads, p->head_dim, n_mid, lm_cap, cpb);
     if (cudaPeekAtLastError() != cudaSuccess) return XKV_ERR_CUDA;
   }
   prof_mark(1, st);
@@ -1499,6 +1523,8 @@ static xkv_status sr_launch_t(const xkv_sr_params* p, const SRPlan& plan, const 
     wa.srV = sr_V;
     wa.win = win;
     wa.T = p->T;
+    wa.wbs = p->window_batch_stride > 0 ? p->window_batch_stride
+                                        : static_cast<int64_t>(p->sink + p->recent) * p->n_kv_heads * p->head_dim;
     wa.Hq = p->n_q_heads;
     wa.Hkv = p->n_kv_heads;
     wa.hd = p->head_dim;

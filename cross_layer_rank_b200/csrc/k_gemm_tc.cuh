@@ -125,6 +125,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int row = lq * 32 + lane;
     const int m = m0 + row;
     const bool ok = mbar_wait(&accbar[0], 0, g.status);
+    __syncwarp();  // converged for the warp-wide tcgen05.ld
     tc_fence_after();
     const uint32_t taddr = tmem + (static_cast<uint32_t>(lq * 32) << 16);
     if (ok) {
@@ -173,6 +174,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       }
     }
   }
+  // lane 0 of the role warps may still be in its loop: reconverge every warp
+  // before the block-wide barrier, so that the barrier cannot complete (and
+  // TMEM be released) while a role thread is still issuing
+  __syncwarp();
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
