@@ -41,6 +41,7 @@ EXPORTS = (
     "xkv_sr_attention_decode_noalloc",
     "xkv_xk_sr_workspace_size", "xkv_xk_sr_attention_decode",
     "xkv_sr_profile_enable", "xkv_sr_profile_read",
+    "xkv_sr_append_workspace_size", "xkv_sr_append",
     "xkv_selftest_expired_wait",
     "xkv_full_reconstruct",
     "xkv_dense_workspace_size", "xkv_dense_attention_decode",
@@ -60,7 +61,18 @@ class SRParams(C.Structure):
                 ("T", C.c_int64), ("rank_k", C.c_int), ("rank_v", C.c_int), ("chunk", C.c_int),
                 ("topk", C.c_int), ("sink", C.c_int), ("recent", C.c_int), ("rope_theta", C.c_float),
                 ("dtype", C.c_int), ("a_k_batch_stride", C.c_int64), ("a_v_batch_stride", C.c_int64),
-                ("bt_k_batch_stride", C.c_int64), ("bt_v_batch_stride", C.c_int64)]
+                ("bt_k_batch_stride", C.c_int64), ("bt_v_batch_stride", C.c_int64),
+                ("window_batch_stride", C.c_int64), ("landmark_capacity", C.c_int64)]
+
+
+class AppendParams(C.Structure):
+    """Mirror of xkv_append_params."""
+    _fields_ = [("batch", C.c_int), ("group", C.c_int), ("n_kv_heads", C.c_int), ("head_dim", C.c_int),
+                ("chunk", C.c_int), ("sink", C.c_int), ("recent", C.c_int), ("rope_theta", C.c_float),
+                ("dtype", C.c_int), ("T", C.c_int64), ("rank_k", C.c_int), ("rank_v", C.c_int),
+                ("a_k_batch_stride", C.c_int64), ("a_v_batch_stride", C.c_int64),
+                ("bt_k_batch_stride", C.c_int64), ("bt_v_batch_stride", C.c_int64),
+                ("window_batch_stride", C.c_int64), ("landmark_capacity", C.c_int64)]
 
 
 class DenseParams(C.Structure):
@@ -101,6 +113,9 @@ def _load():
         "xkv_xk_sr_attention_decode": (C.c_int, [C.POINTER(SRParams), vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz,
                                                  vp]),
         "xkv_selftest_expired_wait": (C.c_int, [vp]),
+        "xkv_sr_append_workspace_size": (C.c_int, [C.POINTER(AppendParams), C.POINTER(sz)]),
+        "xkv_sr_append": (C.c_int, [C.POINTER(AppendParams), vp, vp, vp, vp, vp, vp, vp, vp, vp, C.POINTER(C.c_int),
+                                    vp, sz, vp]),
         "xkv_sr_profile_enable": (C.c_int, [C.c_int]),
         "xkv_sr_profile_read": (C.c_int, [C.POINTER(C.c_float)]),
         "xkv_full_reconstruct": (C.c_int, [vp, vp, i64, C.c_int, C.c_int, C.c_int, C.c_int, C.c_int, C.c_float,
@@ -264,28 +279,43 @@ def xkv_build_landmarks(K: torch.Tensor, n_kv_heads: int, head_dim: int, chunk: 
 # -------------------------------------------------------------- SR decode
 def sr_params(batch, n_q_heads, n_kv_heads, head_dim, T, rank_k, rank_v, chunk, topk, sink, recent, rope_theta,
               dtype: torch.dtype, a_k_batch_stride=None, a_v_batch_stride=None, bt_k_batch_stride=None,
-              bt_v_batch_stride=None) -> SRParams:
-    """Batch strides default to dense [B][T][r] A and per-batch dense [B][d][r] Bt."""
+              bt_v_batch_stride=None, window_batch_stride=0, landmark_capacity=0) -> SRParams:
+    """Batch strides default to dense [B][T][r] A and per-batch dense [B][d][r] Bt;
+    window and landmark strides default to the exact sizes (0)."""
     d = n_kv_heads * head_dim
     return SRParams(batch, n_q_heads, n_kv_heads, head_dim, T, rank_k, rank_v, chunk, topk, sink, recent,
                     float(rope_theta), dtype_code(dtype),
                     T * rank_k if a_k_batch_stride is None else a_k_batch_stride,
                     T * rank_v if a_v_batch_stride is None else a_v_batch_stride,
                     d * rank_k if bt_k_batch_stride is None else bt_k_batch_stride,
-                    d * rank_v if bt_v_batch_stride is None else bt_v_batch_stride)
+                    d * rank_v if bt_v_batch_stride is None else bt_v_batch_stride,
+                    window_batch_stride, landmark_capacity)
 
 
 def xkv_sr_workspace_size(p: SRParams) -> int:
     return _wsize(lib.xkv_sr_workspace_size, C.byref(p))
 
 
+def _addr(t: Optional[torch.Tensor]):
+    """Device address of a tensor whose layout the call's strides describe (a
+    view such as one layer's rows of a group basis is accepted)."""
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("expected a CUDA tensor")
+    if t.numel() > 0 and t.shape[-1] > 1 and t.stride(-1) != 1:
+        raise ValueError("expected contiguous rows")
+    return C.c_void_p(t.data_ptr())
+
+
 def xkv_sr_attention_decode(p: SRParams, q, A_K, Bt_K, A_V, Bt_V, landmarks, sr_K, sr_V, out,
                             sel_out=None, ws=None, stream=None):
-    """One SR decode step of one layer; writes out [B][Hq][hd] f32 (and sel_out)."""
+    """One SR decode step of one layer; writes out [B][Hq][hd] f32 (and sel_out).
+    A, Bt, landmarks and windows may be views: their strides come from p."""
     ws = ws if ws is not None else workspace(xkv_sr_workspace_size(p), q.device)
-    _check(lib.xkv_sr_attention_decode(C.byref(p), _ptr(q), _ptr(A_K), _ptr(Bt_K), _ptr(A_V), _ptr(Bt_V),
-                                       _ptr(landmarks), _ptr(sr_K), _ptr(sr_V), _ptr(out), _ptr(sel_out), _ptr(ws),
-                                       ws.numel(), _stream(stream)), "xkv_sr_attention_decode")
+    _check(lib.xkv_sr_attention_decode(C.byref(p), _ptr(q), _addr(A_K), _addr(Bt_K), _addr(A_V), _addr(Bt_V),
+                                       _addr(landmarks), _addr(sr_K), _addr(sr_V), _ptr(out), _ptr(sel_out),
+                                       _ptr(ws), ws.numel(), _stream(stream)), "xkv_sr_attention_decode")
 
 
 SR_STATIC_SCRATCH_BYTES = 8 << 20
@@ -309,7 +339,7 @@ def xk_sr_params(batch, n_q_heads, n_kv_heads, head_dim, T, rank_k, chunk, topk,
                     float(rope_theta), dtype_code(dtype),
                     T * rank_k if a_k_batch_stride is None else a_k_batch_stride,
                     T * d if v_batch_stride is None else v_batch_stride,
-                    d * rank_k if bt_k_batch_stride is None else bt_k_batch_stride, 0)
+                    d * rank_k if bt_k_batch_stride is None else bt_k_batch_stride, 0, 0, 0)
 
 
 def xkv_xk_sr_workspace_size(p: SRParams) -> int:
@@ -391,4 +421,35 @@ def xkv_energy_rank(gram, block: int, energy: float = 0.95, rank_out=None, lambd
     _check(lib.xkv_energy_rank(_ptr(gram), n, block, float(energy), _ptr(rank_out), _ptr(lambda_out), _ptr(ws),
                                ws.numel(), _stream(stream)), "xkv_energy_rank")
     return rank_out
+
+
+# ------------------------------------------------------- multi-step decode
+def decode_layout(T: int, sink: int, recent: int, chunk: int):
+    """(n_mid, window rows) of a cache of T tokens built by prefill plus appends:
+    n0 = T - sink - recent; n_mid = n0 // chunk; the window holds recent + n0 % chunk rows."""
+    n0 = T - sink - recent
+    return n0 // chunk, recent + n0 % chunk
+
+
+def append_params(batch, group, n_kv_heads, head_dim, chunk, sink, recent, rope_theta, dtype: torch.dtype, T,
+                  rank_k, rank_v, a_k_batch_stride, a_v_batch_stride, bt_k_batch_stride, bt_v_batch_stride,
+                  window_batch_stride, landmark_capacity) -> AppendParams:
+    return AppendParams(batch, group, n_kv_heads, head_dim, chunk, sink, recent, float(rope_theta), dtype_code(dtype),
+                        T, rank_k, rank_v, a_k_batch_stride, a_v_batch_stride, bt_k_batch_stride, bt_v_batch_stride,
+                        window_batch_stride, landmark_capacity)
+
+
+def xkv_sr_append(p: AppendParams, k_new, v_new, win_K, win_V, Bt_K, Bt_V, A_K, A_V, landmarks, ws=None,
+                  stream=None) -> bool:
+    """Append one token per layer (lists of G tensors); returns True when a chunk was rolled."""
+    G = p.group
+    arr = lambda ts: (C.c_void_p * G)(*[t.data_ptr() for t in ts])
+    n = C.c_size_t(0)
+    _check(lib.xkv_sr_append_workspace_size(C.byref(p), C.byref(n)), "xkv_sr_append_workspace_size")
+    ws = ws if ws is not None else workspace(n.value, A_K.device)
+    rolled = C.c_int(0)
+    _check(lib.xkv_sr_append(C.byref(p), arr(k_new), arr(v_new), arr(win_K), arr(win_V), _ptr(Bt_K), _ptr(Bt_V),
+                             _ptr(A_K), _ptr(A_V), arr(landmarks), C.byref(rolled), _ptr(ws), ws.numel(),
+                             _stream(stream)), "xkv_sr_append")
+    return bool(rolled.value)
 

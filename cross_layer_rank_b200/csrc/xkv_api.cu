@@ -366,6 +366,12 @@ static xkv_status check_sr(const xkv_sr_params* p) {
     return XKV_ERR_INVALID_ARG;
   if (p->dtype != XKV_F32 && p->dtype != XKV_BF16) return XKV_ERR_INVALID_ARG;
   if (!(p->rope_theta > 1.0f)) return XKV_ERR_INVALID_ARG;
+  if (p->window_batch_stride < 0 ||
+      (p->window_batch_stride != 0 && p->window_batch_stride < static_cast<int64_t>(p->sink + p->recent) * d) ||
+      p->window_batch_stride % 8 != 0)
+    return XKV_ERR_INVALID_ARG;
+  if (p->landmark_capacity < 0 || (p->landmark_capacity != 0 && p->landmark_capacity < n_mid))
+    return XKV_ERR_INVALID_ARG;
   const int gq = p->n_q_heads / p->n_kv_heads;
   if (gq > 8 || p->head_dim > 256 || p->sink + p->recent > 64 || n_mid > kMaxMidChunks || p->rank_v > 4096 ||
       p->topk > 1024)
@@ -467,6 +473,63 @@ xkv_status xkv_xk_sr_attention_decode(const xkv_sr_params* p, const void* q, con
   if (!workspace || ws_bytes < plan.bytes || !aligned256(workspace)) return XKV_ERR_WORKSPACE;
   return sr_launch(&pv, plan, q, A_K, Bt_K, V, nullptr, landmarks, sr_K, sr_V, out, sel_out, workspace,
                    static_cast<cudaStream_t>(stream));
+}
+
+// ------------------------------------------------------ multi-step decode
+static xkv_status check_append(const xkv_append_params* p) {
+  if (!p || p->batch < 1 || p->group < 1 || p->group > 8 || p->n_kv_heads < 1 || p->head_dim < 2 ||
+      p->head_dim % 2 != 0 || p->head_dim > 256 || p->chunk < 1 || p->sink < 0 || p->recent < 0 ||
+      p->T < p->sink + p->recent || p->rank_k < 1 || p->rank_v < 1 || !(p->rope_theta > 1.0f))
+    return XKV_ERR_INVALID_ARG;
+  if (p->dtype != XKV_F32 && p->dtype != XKV_BF16) return XKV_ERR_INVALID_ARG;
+  const int64_t d = static_cast<int64_t>(p->n_kv_heads) * p->head_dim;
+  const int64_t n = d * p->group;
+  if (p->rank_k > n || p->rank_v > n) return XKV_ERR_INVALID_ARG;
+  const int64_t n0 = p->T - p->sink - p->recent;
+  const int64_t n_mid = n0 / p->chunk;
+  const bool roll = n0 % p->chunk == p->chunk - 1;
+  const int64_t rows_needed = p->sink + (n_mid + (roll ? 1 : 0)) * p->chunk;
+  if (p->window_batch_stride < (p->sink + p->recent + p->chunk) * d || p->window_batch_stride % 8 != 0)
+    return XKV_ERR_INVALID_ARG;
+  if (p->landmark_capacity < n_mid + (roll ? 1 : 0)) return XKV_ERR_INVALID_ARG;
+  if (p->a_k_batch_stride < rows_needed * p->rank_k || p->a_v_batch_stride < rows_needed * p->rank_v)
+    return XKV_ERR_INVALID_ARG;
+  if ((p->bt_k_batch_stride != 0 && p->bt_k_batch_stride < n * p->rank_k) ||
+      (p->bt_v_batch_stride != 0 && p->bt_v_batch_stride < n * p->rank_v) || p->bt_k_batch_stride < 0 ||
+      p->bt_v_batch_stride < 0)
+    return XKV_ERR_INVALID_ARG;
+  if (p->dtype == XKV_BF16 && (!project_tc_ok(static_cast<int>(d), p->rank_k, XKV_BF16) ||
+                               !project_tc_ok(static_cast<int>(d), p->rank_v, XKV_BF16)))
+    return XKV_ERR_UNSUPPORTED;
+  if (p->recent > 56) return XKV_ERR_UNSUPPORTED;
+  return XKV_OK;
+}
+
+xkv_status xkv_sr_append_workspace_size(const xkv_append_params* p, size_t* bytes) {
+  if (!bytes) return XKV_ERR_INVALID_ARG;
+  const xkv_status s = check_append(p);
+  if (s != XKV_OK) return s;
+  *bytes = append_workspace(p);
+  return XKV_OK;
+}
+
+xkv_status xkv_sr_append(const xkv_append_params* p, const void* const* k_new, const void* const* v_new,
+                         void* const* win_K, void* const* win_V, const void* Bt_K, const void* Bt_V, void* A_K,
+                         void* A_V, void* const* landmarks, int* rolled, void* workspace, size_t ws_bytes,
+                         void* stream) {
+  const xkv_status s = check_append(p);
+  if (s != XKV_OK) return s;
+  if (!k_new || !v_new || !win_K || !win_V || !landmarks) return XKV_ERR_INVALID_ARG;
+  for (int l = 0; l < p->group; ++l)
+    if (!k_new[l] || !v_new[l] || !win_K[l] || !win_V[l] || !landmarks[l] || !aligned16(k_new[l]) ||
+        !aligned16(v_new[l]) || !aligned16(win_K[l]) || !aligned16(win_V[l]) || !aligned16(landmarks[l]))
+      return XKV_ERR_INVALID_ARG;
+  const void* ptrs[] = {Bt_K, Bt_V, A_K, A_V};
+  for (const void* x : ptrs)
+    if (!x || !aligned16(x)) return XKV_ERR_INVALID_ARG;
+  if (!workspace || ws_bytes < append_workspace(p) || !aligned256(workspace)) return XKV_ERR_WORKSPACE;
+  return append_launch(p, k_new, v_new, win_K, win_V, Bt_K, Bt_V, A_K, A_V, landmarks, rolled, workspace,
+                       static_cast<cudaStream_t>(stream));
 }
 
 // --------------------------------------------------- full reconstruction

@@ -80,6 +80,12 @@ xkv_status compress_launch(const CompressPlan& plan, const void* const* X, int G
                            int64_t ldx, xkv_dtype dt, int iters, uint64_t seed, void* A, void* Bt,
                            float* eigvals, float* gram_out, void* ws, cudaStream_t st);
 
+// ---------------------------------------------------- multi-step decode
+size_t append_workspace(const xkv_append_params* p);
+xkv_status append_launch(const xkv_append_params* p, const void* const* k_new, const void* const* v_new,
+                         void* const* win_K, void* const* win_V, const void* Bt_K, const void* Bt_V, void* A_K,
+                         void* A_V, void* const* landmarks, int* rolled, void* ws, cudaStream_t st);
+
 // ------------------------------------------------------------------ NER
 size_t ner_workspace(int n, int block);
 xkv_status energy_rank_launch(const float* gram, int n, int block, double energy, int32_t* rank, float* lam_out,

@@ -182,6 +182,10 @@ typedef struct xkv_sr_params {
   int64_t a_k_batch_stride, a_v_batch_stride;   /* elements between batches of A_K / A_V */
   int64_t bt_k_batch_stride, bt_v_batch_stride; /* elements between batches of Bt_K / Bt_V;
                                                    0 = one Bt shared by the batch */
+  int64_t window_batch_stride; /* elements between sequences of sr_K / sr_V; 0 = (sink + recent) d.
+                                  A window buffer with room for recent + chunk rows (multi-step
+                                  decode, xkv_sr_append) passes (sink + recent + chunk) d. */
+  int64_t landmark_capacity;   /* chunks allocated per (sequence, KV head) in landmarks; 0 = n_mid */
 } xkv_sr_params;
 
 /* One decode step of xKV-SR for one layer ([xKV-blog] "选择性重建", [xKV-abs];
@@ -194,8 +198,10 @@ typedef struct xkv_sr_params {
  *   A_K, A_V  : [B][T][rank] (batch strides in params).   Bt_K, Bt_V : [d][rank] per
  *               batch element (batch strides in params; each sequence has its own
  *               factorisation, or 0 to share one).
- *   landmarks : [B][Hkv][n_mid][hd].   sr_K, sr_V : [B][sink+recent][d]; row i < sink
- *               is token i, row sink + i is token T - recent + i; keys pre-RoPE.
+ *   landmarks : [B][Hkv][cap][hd], cap = landmark_capacity (or n_mid); chunk c < n_mid
+ *               of (b, h) at [b][h][c].   sr_K, sr_V : [B][rows][d] with batch stride
+ *               window_batch_stride; row i < sink is token i, row sink + i is token
+ *               T - recent + i; keys pre-RoPE.
  *   out       : [B][Hq][hd] f32.   sel_out : [B][Hkv][topk] int32, or NULL. */
 XKV_API xkv_status xkv_sr_workspace_size(const xkv_sr_params* p, size_t* bytes);
 XKV_API xkv_status xkv_sr_attention_decode(const xkv_sr_params* p, const void* q, const void* A_K,
@@ -264,6 +270,56 @@ XKV_API xkv_status xkv_selftest_expired_wait(void* stream);
  * XKV_ERR_INVALID_ARG (stage_ms NULL, or nothing recorded yet). */
 XKV_API xkv_status xkv_sr_profile_enable(int enable);
 XKV_API xkv_status xkv_sr_profile_read(float* stage_ms);
+
+/* ---------------------------------------------------- multi-step decode */
+/* Appends one generated token per layer of a group to the raw recent window
+ * and, when the window then holds recent + chunk rows, rolls its oldest chunk
+ * into the compressed cache.  [xKV-blog] (the editor's note after
+ * "仅仅压缩还不够，xKV 还做了“选择性重建”") compresses only the long prefill;
+ * here tokens generated afterwards stay raw until a chunk of them is complete,
+ * then join the compressed cache exactly as prefill tokens did:
+ *   - A_K / A_V rows of the chunk = x V on the group's stored bases Bt_K / Bt_V
+ *     (x = the chunk's rows of all G layers side by side, [xKV-blog]
+ *     "xKV 到底做了什么"), rounded to the cache dtype;
+ *   - landmark[l][b][h][n_mid] = mean over the chunk of RoPE_t(K_l[t, h]) at
+ *     the tokens' absolute positions ([xKV-blog] "选择性重建");
+ *   - the window moves down by one chunk.
+ * The state is a function of the length T before the call: with
+ * n0 = T - sink - recent, the window holds w = recent + n0 % chunk rows after
+ * the sink rows, n_mid = n0 / chunk chunks are compressed, and the new token
+ * goes to window row sink + w.  A decode at length T passes recent = w and
+ * the strides below in xkv_sr_params.
+ *   k_new, v_new : host arrays of G device pointers, each [B][d] (keys pre-RoPE).
+ *   win_K, win_V : host arrays of G device pointers, each [B][rows][d], rows >=
+ *                  sink + recent + chunk, batch stride window_batch_stride.
+ *   Bt_K, Bt_V   : group bases [B][G d][rank] (batch strides; 0 = shared), the
+ *                  Bt that xkv_compress_group returned; layer l owns rows l d...
+ *   A_K, A_V     : [B][capacity][rank] (batch strides >= (T + 1) rank).
+ *   landmarks    : host array of G device pointers, each [B][Hkv][cap][hd],
+ *                  cap = landmark_capacity >= n_mid + 1.
+ *   rolled       : host int, set to 1 when a chunk was rolled (may be NULL).
+ * bf16 caches need d % 64 == 0 and ranks % 64 == 0; f32 caches use CUDA cores.
+ * Workspace: xkv_sr_append_workspace_size.  Calls are stream-ordered; a decode
+ * of any layer of the group after the call sees the new state. */
+typedef struct xkv_append_params {
+  int batch;                   /* B */
+  int group;                   /* G <= 8 */
+  int n_kv_heads, head_dim;    /* d = n_kv_heads head_dim */
+  int chunk, sink, recent;
+  float rope_theta;
+  xkv_dtype dtype;
+  int64_t T;                   /* tokens cached before this append, >= sink + recent */
+  int rank_k, rank_v;
+  int64_t a_k_batch_stride, a_v_batch_stride;
+  int64_t bt_k_batch_stride, bt_v_batch_stride;
+  int64_t window_batch_stride; /* elements, >= (sink + recent + chunk) d, multiple of 8 */
+  int64_t landmark_capacity;   /* chunks per (sequence, KV head) */
+} xkv_append_params;
+XKV_API xkv_status xkv_sr_append_workspace_size(const xkv_append_params* p, size_t* bytes);
+XKV_API xkv_status xkv_sr_append(const xkv_append_params* p, const void* const* k_new, const void* const* v_new,
+                         void* const* win_K, void* const* win_V, const void* Bt_K, const void* Bt_V,
+                         void* A_K, void* A_V, void* const* landmarks, int* rolled, void* workspace,
+                         size_t ws_bytes, void* stream);
 
 /* -------------------------------------------------- full reconstruction */
 /* The comparison path of [xKV-blog] Fig. 6: rebuild every row,
