@@ -321,7 +321,78 @@ def measure_gram(xkv, w, device):
         spectra[name + "_ms"] = round(e0.elapsed_time(e1), 3)
     assert xkv.get_device_status() == 0
     spectra["blocks"] = f"{w.group} x {w.d} x {w.d}"
-    return ms, flops, spectra
+    proj_ms, proj_flops = measure_projection(xkv, X, w.rank_k, device)
+    return ms, flops, spectra, proj_ms, proj_flops
+
+
+def _time_ms(fn, reps=3):
+    """Mean device time of fn() over reps calls (after one untimed call)."""
+    import torch
+    fn()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        fn()
+    e1.record()
+    e1.synchronize()
+    return e0.elapsed_time(e1) / reps
+
+
+def measure_projection(xkv, X, rank, device):
+    """Device time of A = X V_r (xkv_project, f32 basis as a bf16 hi/lo pair)
+    for X = the given layers; algorithmic flops 2 T (G d) r (the hi/lo pair's
+    second product is not counted)."""
+    import torch
+    G = len(X)
+    T, d = X[0].shape
+    n = G * d
+    V = torch.randn((n, rank), dtype=torch.float32, device=device) / math.sqrt(n)
+    A = torch.empty((T, rank), dtype=torch.bfloat16, device=device)
+    ws = xkv.workspace(xkv.xkv_project_workspace_size(G, d, rank), device)
+    ms = _time_ms(lambda: xkv.xkv_project(X, V, A, ws))
+    flops = 2.0 * T * n * rank
+    return ms, flops
+
+
+def measure_compress_sweep(xkv, device, bf16_peak, log):
+    """The prefill compression sweep: d = 1024 (8 x 128), T = 32768 in four
+    8192-row shards, G = 1, 2, 4, 8 layers, r = 128 G.  Per G: the Gram over the
+    shards, the projection, and the whole xkv_compress_group call."""
+    import torch
+    out = {}
+    for G in (1, 2, 4, 8):
+        w = synth.compression_sweep(G)
+        X = synth.kv_group_torch(w, 0, 0, "K", device)
+        n, r, T = G * w.d, w.rank_k, w.T
+        C = torch.zeros((n, n), dtype=torch.float32, device=device)
+        wsg = xkv.workspace(xkv.xkv_gram_workspace_size(G, 8192, w.d, torch.bfloat16), device)
+
+        def gram():
+            for s0 in range(0, T, 8192):
+                xkv.xkv_gram_accumulate([x[s0:s0 + 8192] for x in X], C, wsg)
+        g_ms = _time_ms(gram)
+        g_fl = n * (n + 1) * T
+        p_ms, p_fl = measure_projection(xkv, X, r, device)
+        A = torch.empty((T, r), dtype=torch.bfloat16, device=device)
+        Bt = torch.empty((n, r), dtype=torch.bfloat16, device=device)
+        p = synth.oversample(r)
+        wsc = xkv.workspace(xkv.xkv_compress_workspace_size(G, T, w.d, r, p, 8192, torch.bfloat16), device)
+        c_ms = _time_ms(lambda: xkv.xkv_compress_group(X, r, A, Bt, iters=8, oversample=p, shard_rows=8192, ws=wsc),
+                        reps=1)
+        assert xkv.get_device_status() == 0
+        out[f"G{G}"] = {"n": n, "rank": r, "gram_ms": round(g_ms, 4),
+                        "gram_tflops": round(g_fl / (g_ms / 1e3) / 1e12, 1),
+                        "gram_frac_of_bf16_peak": round(g_fl / (g_ms / 1e3) / 1e12 / bf16_peak, 4),
+                        "projection_ms": round(p_ms, 4),
+                        "projection_tflops": round(p_fl / (p_ms / 1e3) / 1e12, 1),
+                        "projection_frac_of_bf16_peak": round(p_fl / (p_ms / 1e3) / 1e12 / bf16_peak, 4),
+                        "compress_group_ms": round(c_ms, 3)}
+        log(f"compression sweep G={G}: {out[f'G{G}']}")
+        del X, C, A, Bt, wsc, wsg
+        torch.cuda.empty_cache()
+    out["shape"] = "d = 1024, T = 32768 (4 shards of 8192), r = 128 G; flops: Gram n (n+1) T, projection 2 T n r"
+    return out
 
 
 # --------------------------------------------------------- multi-rank
@@ -359,7 +430,8 @@ def run_cuda(args, rank, world, log):
     L = n_groups * w.group
     bf = torch.bfloat16
     model, prefill = build_model(xkv, w, device, n_groups, log)
-    gram_ms, gram_flops, spectra = measure_gram(xkv, w, device) if args.prefill else (None, None, None)
+    gram_ms, gram_flops, spectra, proj_ms, proj_flops = (measure_gram(xkv, w, device) if args.prefill
+                                                         else (None,) * 5)
 
     p = xkv.sr_params(w.batch, w.n_q_heads, w.n_kv_heads, w.head_dim, w.T, w.rank_k, w.rank_v, w.chunk, w.topk,
                       w.sink, w.recent, w.rope_theta, bf)
@@ -514,7 +586,11 @@ def run_cuda(args, rank, world, log):
                           "gram_ms": round(gram_ms, 4),
                           "gram_tflops": round(gram_flops / (gram_ms / 1e3) / 1e12, 1),
                           "gram_frac_of_bf16_peak": round(gram_flops / (gram_ms / 1e3) / 1e12 / bf16_peak, 4),
-                          "spectra": spectra}
+                          "projection_ms": round(proj_ms, 4),
+                          "projection_tflops": round(proj_flops / (proj_ms / 1e3) / 1e12, 1),
+                          "projection_frac_of_bf16_peak": round(proj_flops / (proj_ms / 1e3) / 1e12 / bf16_peak, 4),
+                          "spectra": spectra,
+                          "sweep": measure_compress_sweep(xkv, device, bf16_peak, log)}
     return res, w
 
 
@@ -639,7 +715,7 @@ def cpu_baseline(w, budget_s: float, log):
     units_step = w.batch * w.n_layers * w.n_kv_heads
     step_s = dt / done * units_step
     return {"value": round(w.batch / step_s, 4), "unit": "tokens/s", "cores": oracle.num_threads(),
-            "kind": "oracle",
+            "kind": "oracle", "wall_s": round(dt, 3),
             "sample": f"{done} (layer, KV-head) units of one decode step (batch 1, T={w.T}), oracle SR decode in "
                       f"fp64, scaled to the full {w.n_layers}-layer batch-{w.batch} step ({units_step} units)"}
 
@@ -658,7 +734,11 @@ def run_reference(args, log):
     cb = dict(vals[0])
     cb["value"] = v
     return {"impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": 1, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": round(w.batch / v * 1e3, 3), "higher_is_better": True,
+            "warmup": args.warmup, "ms_per_step": round(w.batch / v * 1e3, 3),
+            "sampled": True, "sample_wall_s_per_step": round(statistics.median(x["wall_s"] for x in vals), 3),
+            "note": "each step runs the oracle on a bounded sample of (layer, KV head) units and scales its time "
+                    "to the whole step; ms_per_step is that scaled time, not the wall time of the sample",
+            "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": args.workload, "global_batch": w.batch, "seq_len": w.T, "layers": w.n_layers},
             "cpu_baseline": cb, "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0,

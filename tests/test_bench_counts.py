@@ -1,6 +1,7 @@
-"""The bench's algorithmic counts against the scope table's figures for the
-three decode shapes (Llama-3.1-8B group at 16K, the 32-layer Llama-3.1-8B at
-64K batch 4, the 28-layer Qwen2.5-7B at 128K batch 2): bytes per decode step
+"""The bench's algorithmic counts against figures worked out by hand from the
+per-unit byte formula, for the three decode shapes (Llama-3.1-8B group at 16K,
+the 32-layer Llama-3.1-8B at 64K batch 4, the 28-layer Qwen2.5-7B at 128K
+batch 2): bytes per decode step
 (landmarks + selected A rows + Bt slices + raw window + queries/outputs) and
 the cache compression ratios (A+B alone, and with the landmarks)."""
 import os
