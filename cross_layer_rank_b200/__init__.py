@@ -40,8 +40,11 @@ EXPORTS = (
     "xkv_sr_workspace_size", "xkv_sr_attention_decode",
     "xkv_sr_attention_decode_noalloc",
     "xkv_xk_sr_workspace_size", "xkv_xk_sr_attention_decode",
+    "xkv_xk_sr_host_workspace_size", "xkv_xk_sr_attention_decode_host_values",
     "xkv_sr_profile_enable", "xkv_sr_profile_read",
     "xkv_sr_append_workspace_size", "xkv_sr_append",
+    "xkv_sr_scores", "xkv_sr_topk", "xkv_sr_partial_workspace_size", "xkv_sr_attention_partial",
+    "xkv_merge_partials",
     "xkv_selftest_expired_wait",
     "xkv_full_reconstruct",
     "xkv_dense_workspace_size", "xkv_dense_attention_decode",
@@ -73,6 +76,11 @@ class AppendParams(C.Structure):
                 ("a_k_batch_stride", C.c_int64), ("a_v_batch_stride", C.c_int64),
                 ("bt_k_batch_stride", C.c_int64), ("bt_v_batch_stride", C.c_int64),
                 ("window_batch_stride", C.c_int64), ("landmark_capacity", C.c_int64)]
+
+
+class ShardParams(C.Structure):
+    """Mirror of xkv_sr_shard."""
+    _fields_ = [("position_offset", C.c_int64), ("chunk_begin", C.c_int64)]
 
 
 class DenseParams(C.Structure):
@@ -112,6 +120,15 @@ def _load():
         "xkv_xk_sr_workspace_size": (C.c_int, [C.POINTER(SRParams), C.POINTER(sz)]),
         "xkv_xk_sr_attention_decode": (C.c_int, [C.POINTER(SRParams), vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz,
                                                  vp]),
+        "xkv_xk_sr_host_workspace_size": (C.c_int, [C.POINTER(SRParams), C.POINTER(sz)]),
+        "xkv_xk_sr_attention_decode_host_values": (C.c_int, [C.POINTER(SRParams), vp, vp, vp, vp, vp, vp, vp, vp, vp,
+                                                             vp, sz, vp]),
+        "xkv_sr_scores": (C.c_int, [C.POINTER(SRParams), vp, vp, vp, i64, vp]),
+        "xkv_sr_topk": (C.c_int, [vp, i64, C.c_int, i64, C.c_int, vp, vp]),
+        "xkv_sr_partial_workspace_size": (C.c_int, [C.POINTER(SRParams), C.POINTER(sz)]),
+        "xkv_sr_attention_partial": (C.c_int, [C.POINTER(SRParams), C.POINTER(ShardParams), vp, vp, vp, vp, vp, vp,
+                                               vp, vp, vp, vp, vp, sz, vp]),
+        "xkv_merge_partials": (C.c_int, [vp, vp, C.c_int, C.c_int, C.c_int, vp, vp]),
         "xkv_selftest_expired_wait": (C.c_int, [vp]),
         "xkv_sr_append_workspace_size": (C.c_int, [C.POINTER(AppendParams), C.POINTER(sz)]),
         "xkv_sr_append": (C.c_int, [C.POINTER(AppendParams), vp, vp, vp, vp, vp, vp, vp, vp, vp, C.POINTER(C.c_int),
@@ -342,6 +359,23 @@ def xk_sr_params(batch, n_q_heads, n_kv_heads, head_dim, T, rank_k, chunk, topk,
                     d * rank_k if bt_k_batch_stride is None else bt_k_batch_stride, 0, 0, 0)
 
 
+def xkv_xk_sr_host_workspace_size(p: SRParams) -> int:
+    return _wsize(lib.xkv_xk_sr_host_workspace_size, C.byref(p))
+
+
+def xkv_xk_sr_attention_decode_host_values(p: SRParams, q, A_K, Bt_K, V_host: torch.Tensor, landmarks, sr_K, sr_V,
+                                           out, sel_out=None, ws=None, stream=None):
+    """xK-SR step with V [B][T][d] in pinned host memory (V_host.is_pinned());
+    only the kept chunks' rows are read over the host link."""
+    if V_host.is_cuda or not V_host.is_pinned():
+        raise ValueError("V_host must be a pinned host tensor")
+    ws = ws if ws is not None else workspace(xkv_xk_sr_host_workspace_size(p), q.device)
+    _check(lib.xkv_xk_sr_attention_decode_host_values(C.byref(p), _ptr(q), _addr(A_K), _addr(Bt_K),
+                                                      C.c_void_p(V_host.data_ptr()), _addr(landmarks), _addr(sr_K),
+                                                      _addr(sr_V), _ptr(out), _ptr(sel_out), _ptr(ws), ws.numel(),
+                                                      _stream(stream)), "xkv_xk_sr_attention_decode_host_values")
+
+
 def xkv_xk_sr_workspace_size(p: SRParams) -> int:
     return _wsize(lib.xkv_xk_sr_workspace_size, C.byref(p))
 
@@ -452,4 +486,37 @@ def xkv_sr_append(p: AppendParams, k_new, v_new, win_K, win_V, Bt_K, Bt_V, A_K, 
                              _ptr(A_K), _ptr(A_V), arr(landmarks), C.byref(rolled), _ptr(ws), ws.numel(),
                              _stream(stream)), "xkv_sr_append")
     return bool(rolled.value)
+
+
+# ------------------------------------------------------- token sharding
+def xkv_sr_scores(p: SRParams, q, landmarks, scores, stream=None):
+    """scores [B][Hkv][ld] f32 (ld >= n_mid, a multiple of 4): the local chunk scores."""
+    _check(lib.xkv_sr_scores(C.byref(p), _ptr(q), _addr(landmarks), _addr(scores), scores.stride(-2),
+                             _stream(stream)), "xkv_sr_scores")
+
+
+def xkv_sr_topk(scores, n: int, k: int, sel_out, stream=None):
+    """Exact top-k of each row of scores [..., ld] over its first n entries."""
+    rows = scores.numel() // scores.shape[-1]
+    _check(lib.xkv_sr_topk(_addr(scores), scores.stride(-2), rows, n, k, _ptr(sel_out), _stream(stream)),
+           "xkv_sr_topk")
+
+
+def xkv_sr_attention_partial(p: SRParams, shard: ShardParams, sel, q, A_K, Bt_K, A_V, Bt_V, sr_K, sr_V, out, ml_out,
+                             ws=None, stream=None):
+    """Attention of this device's token slice for the global selection sel; out
+    normalised by its own sum, ml_out = (M, L) per (sequence, query head)."""
+    if ws is None:
+        n = C.c_size_t(0)
+        _check(lib.xkv_sr_partial_workspace_size(C.byref(p), C.byref(n)), "xkv_sr_partial_workspace_size")
+        ws = workspace(n.value, q.device)
+    _check(lib.xkv_sr_attention_partial(C.byref(p), C.byref(shard), _ptr(sel), _ptr(q), _addr(A_K), _addr(Bt_K),
+                                        _addr(A_V), _addr(Bt_V), _addr(sr_K), _addr(sr_V), _ptr(out), _ptr(ml_out),
+                                        _ptr(ws), ws.numel(), _stream(stream)), "xkv_sr_attention_partial")
+
+
+def xkv_merge_partials(o, ml, out, stream=None):
+    """o [R][rows][hd], ml [R][rows][2] -> out [rows][hd] (the exact softmax combination)."""
+    R, rows, hd = o.shape[0], o.numel() // (o.shape[0] * o.shape[-1]), o.shape[-1]
+    _check(lib.xkv_merge_partials(_ptr(o), _ptr(ml), R, rows, hd, _ptr(out), _stream(stream)), "xkv_merge_partials")
 

@@ -117,7 +117,8 @@ __device__ uint32_t block_exclusive_scan(uint32_t v, uint32_t* warp_tot, uint32_
 template <typename T>
 __global__ void __launch_bounds__(256) sr_score_kernel(const T* __restrict__ q, const T* __restrict__ lm,
                                                        float* __restrict__ scores, int Hq, int Hkv, int hd,
-                                                       int64_t n_mid, int64_t lm_cap, int chunks_per_block) {
+                                                       int64_t n_mid, int64_t lm_cap, int64_t ld,
+                                                       int chunks_per_block) {
   allow_next_grid();
   __shared__ float qbar[256];
   const int unit = blockIdx.y;
@@ -132,7 +133,7 @@ __global__ void __launch_bounds__(256) sr_score_kernel(const T* __restrict__ q, 
   const int64_t c1 = min(c0 + chunks_per_block, n_mid);
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const T* base = lm + static_cast<int64_t>(unit) * lm_cap * hd;
-  float* out = scores + static_cast<int64_t>(unit) * ((n_mid + 3) & ~int64_t(3));
+  float* out = scores + static_cast<int64_t>(unit) * ld;
   if (sizeof(T) == 2 && hd == 128) {
     // 16 lanes x 16 B cover one 256-B landmark row; a warp scores 2 rows per
     // load and keeps 8 rows (4 loads per lane) in flight.
@@ -214,6 +215,7 @@ struct WinArgs {
   float* win;
   int64_t T;
   int64_t wbs;  // elements between sequences of the raw window
+  int64_t pos_off;  // global position of local token row 0
   int Hq, Hkv, hd, sink, recent;
   double ft[128];  // RoPE frequency of pair j in turns per position
 };
@@ -268,7 +270,7 @@ __device__ void window_partial(const WinArgs& wa, int unit, uint8_t* smem) {
   // 2. RoPE of the window keys at their positions
   for (int i = tid; i < nsr * half; i += nt) {
     const int r = i / half, jj = i % half;
-    const int64_t t = r < wa.sink ? r : wa.T - wa.recent + (r - wa.sink);
+    const int64_t t = wa.pos_off + (r < wa.sink ? r : wa.T - wa.recent + (r - wa.sink));
     float c, sn;
     rope_cs(fts[jj], static_cast<double>(t), &c, &sn);
     float* kr = wK + r * ks;
@@ -551,12 +553,21 @@ struct AttendArgs {
   int64_t T;
   int64_t sbk, sbv;  // batch strides of Bt_K / Bt_V (elements, 0 = shared)
   int Hq, Hkv, k, sink, recent, rK, rV;
-  int v_raw;  // values uncompressed (xK-SR): the value operand is V [B][T][d], head h at column h hd, rV = hd
+  int v_raw;  // values uncompressed (xK-SR), rV = hd: 1 = the value operand is V [B][T][d], head h at
+              // column h hd; 2 = the kept rows gathered from host memory, [units][k][chunk][hd]
   int tiles_per_unit, n_tiles, ctas, max_units;
   int slot_floats;
   float theta;
+  // token sharding: local row 0 is global position pos_off; selection entries
+  // are global chunk indices, kept only in [c_lo, c_hi), whose rows sit at
+  // local row sink + (c - c_lo) chunk (the whole sequence: 0, 0, n_mid)
+  int64_t pos_off;
+  int c_lo, c_hi;
+  float* ml_out;  // (M, L) per (sequence, query head) when the caller merges partials, or null
   double ft[128];  // RoPE turns per position of each frequency pair (host-computed, fp64)
 };
+
+__device__ __forceinline__ bool kept_here(const AttendArgs& a, int c) { return c >= a.c_lo && c < a.c_hi; }
 
 __device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y,
                                             int z, int w) {
@@ -685,17 +696,27 @@ __device__ void merge_unit(const T* __restrict__ BtV, const float* __restrict__ 
     float M = lane == 0 ? wml[g] : -INFINITY;
     for (int i = lane; i < nslots; i += 32) M = fmaxf(M, ml[i * 16 + g]);
     M = warp_max(M);
+    // M = -inf: no kept row and no window row for this head (a token shard
+    // whose chunks were all selected elsewhere): every factor and the output
+    // are 0, and (M, L) = (-inf, 0) tells the caller's merge to skip it
+    const bool none = M == -INFINITY;
     float L = 0.f;
     for (int i = lane; i < nslots; i += 32) {
-      const float f = exp2f(ml[i * 16 + g] - M);
+      const float f = none ? 0.f : exp2f(ml[i * 16 + g] - M);
       sc[i * kMaxGQ + g] = f;
       L = fmaf(ml[i * 16 + 8 + g], f, L);
     }
     L = warp_sum(L);
     if (lane == 0) {
-      const float f = exp2f(wml[g] - M);
+      const float f = none ? 0.f : exp2f(wml[g] - M);
       fw[g] = f;
-      Lg[g] = 1.f / fmaf(wml[8 + g], f, L);
+      const float Lt = fmaf(wml[8 + g], f, L);
+      Lg[g] = Lt > 0.f ? 1.f / Lt : 0.f;
+      if (args.ml_out && j0 == 0) {
+        float* mo = args.ml_out + (static_cast<int64_t>(b) * args.Hq + h * gq + g) * 2;
+        mo[0] = M;
+        mo[1] = Lt;
+      }
     }
   }
   __syncthreads();
@@ -938,7 +959,8 @@ __global__ void __launch_bounds__(kAttendThreads, 1)
         const int32_t* su = args.sel + static_cast<int64_t>(u) * k + ti * kTileChunks;
         int rows[kTileChunks];
 #pragma unroll
-        for (int ch = 0; ch < kTileChunks; ++ch) rows[ch] = ch < nch ? args.sink + su[ch] * 8 : 0;
+        for (int ch = 0; ch < kTileChunks; ++ch)
+          rows[ch] = ch < nch && kept_here(args, su[ch]) ? args.sink + (su[ch] - args.c_lo) * 8 : 0;
         // one 4-D box per chunk covers kKAtoms atoms (8 rows x 128 columns);
         // the Bt_K atoms of the stage follow on their own ring (L2 hits)
         // (an odd atom count leaves the last box half out of range: TMA fills
@@ -981,14 +1003,21 @@ __global__ void __launch_bounds__(kAttendThreads, 1)
       if (te > tb && !mbar_wait(&kfull[0], 0, args.status)) *abort_flag = 1;
       for (int x = tb; x < te && !*abort_flag; ++x) {
         const int u = x / tpu, ti = x % tpu;
-        const int b = u / args.Hkv;
-        // first 64-column atom of the value rows: head h's columns when values are uncompressed
-        const int vz = args.v_raw ? (u % args.Hkv) * NAV : 0;
+        // batch coordinate, first 64-column atom and row of each chunk's value
+        // rows: the unit's rank columns; head h's columns of V when values are
+        // uncompressed; the staged rows of selection position c when they were
+        // gathered from host memory
+        const int b = args.v_raw == 2 ? u : u / args.Hkv;
+        const int vz = args.v_raw == 1 ? (u % args.Hkv) * NAV : 0;
         const int nch = min(kTileChunks, k - ti * kTileChunks);
         const int32_t* su = args.sel + static_cast<int64_t>(u) * k + ti * kTileChunks;
+        const int pos0 = ti * kTileChunks;
         int rows[kTileChunks];
 #pragma unroll
-        for (int ch = 0; ch < kTileChunks; ++ch) rows[ch] = ch < nch ? args.sink + su[ch] * 8 : 0;
+        for (int ch = 0; ch < kTileChunks; ++ch)
+          rows[ch] = ch < nch ? (args.v_raw == 2 ? (pos0 + ch) * 8
+                                                 : kept_here(args, su[ch]) ? args.sink + (su[ch] - args.c_lo) * 8 : 0)
+                              : 0;
         for (int v = 0; v < (nch + 1) / 2 && !*abort_flag; ++v, ++vsn) {
           const int slot = vsn % kVStages;
           if (!mbar_wait(&vempty[slot], ((vsn / kVStages) & 1) ^ 1, args.status)) { *abort_flag = 1; break; }
@@ -1103,13 +1132,15 @@ __global__ void __launch_bounds__(kAttendThreads, 1)
       for (int i = et; i < kTileChunks * 64; i += 256) {
         const int ch = i >> 6, jj = i & 63;
         float c = 1.f, sn = 0.f;
-        if (ch < nch) rope_cs(ft[jj], static_cast<double>(args.sink + static_cast<int64_t>(su[ch]) * 8), &c, &sn);
+        if (ch < nch && kept_here(args, su[ch]))
+          rope_cs(ft[jj], static_cast<double>(args.pos_off + args.sink + static_cast<int64_t>(su[ch] - args.c_lo) * 8),
+                  &c, &sn);
         base_s[ch * kRopeStride + 2 * jj] = c;
         base_s[ch * kRopeStride + 2 * jj + 1] = sn;
       }
       named_bar_sync(1, 256);
       const int ch = row >> 3, e = row & 7;
-      const bool valid = ch < nch;
+      const bool valid = ch < nch && kept_here(args, su[ch]);
       const float2* bse = reinterpret_cast<const float2*>(base_s + ch * kRopeStride);
       const float2* rte = reinterpret_cast<const float2*>(rot_s + e * kRopeStride);
       const int buf = j & 1;
@@ -1178,9 +1209,10 @@ __global__ void __launch_bounds__(kAttendThreads, 1)
 #pragma unroll
       for (int g = 0; g < GQ; ++g) {
         const float mn = fmaxf(m[g], tmax[g]);
-        alpha[g] = exp2f(m[g] - mn);
+        // (no kept row yet: mn = -inf, nothing to rescale)
+        alpha[g] = mn == -INFINITY ? 1.f : exp2f(m[g] - mn);
         // the weights enter the value MMA as bf16: the sum uses the same values
-        pbf[g] = __float2bfloat16_rn(valid ? exp2f(s[g] - mn) : 0.f);
+        pbf[g] = __float2bfloat16_rn(valid && mn != -INFINITY ? exp2f(s[g] - mn) : 0.f);
         m[g] = mn;
         const float w = warp_sum(__bfloat162float(pbf[g]));
         if (lane == 0) red[32 + lq * 8 + g] = w;
@@ -1341,7 +1373,9 @@ __global__ void __launch_bounds__(256) sr_attend_simt_kernel(const T* __restrict
       for (int i = tid; i < nr * half; i += blockDim.x) {
         const int r = i / half, jj = i % half;
         const int rr = rb + r;
-        const int64_t t = args.sink + static_cast<int64_t>(args.sel[static_cast<int64_t>(u) * k + ti * kTileChunks + rr / chunk]) * chunk + rr % chunk;
+        const int cc = args.sel[static_cast<int64_t>(u) * k + ti * kTileChunks + rr / chunk];
+        const bool kept = kept_here(args, cc);
+        const int64_t t = args.sink + static_cast<int64_t>(kept ? cc - args.c_lo : 0) * chunk + rr % chunk;
         const T* a = AK + b * sak + t * args.rK;
         const T* b0 = BtK + b * args.sbk + static_cast<int64_t>(h * hd + jj) * args.rK;
         const T* b1 = BtK + b * args.sbk + static_cast<int64_t>(h * hd + jj + half) * args.rK;
@@ -1352,26 +1386,28 @@ __global__ void __launch_bounds__(256) sr_attend_simt_kernel(const T* __restrict
           y1 = fmaf(av, to_f(b1[c]), y1);
         }
         float cs, sn;
-        rope_cs(ft[jj], static_cast<double>(t), &cs, &sn);
-        Ks[r * hd + jj] = y0 * cs - y1 * sn;
-        Ks[r * hd + jj + half] = y1 * cs + y0 * sn;
+        rope_cs(ft[jj], static_cast<double>(args.pos_off + t), &cs, &sn);
+        Ks[r * hd + jj] = kept ? y0 * cs - y1 * sn : 0.f;
+        Ks[r * hd + jj + half] = kept ? y1 * cs + y0 * sn : 0.f;
       }
       __syncthreads();
       for (int i = tid; i < nr * gq; i += blockDim.x) {
         const int r = i / gq, g = i % gq;
+        const int rr = rb + r;
         float s = 0.f;
         for (int jj = 0; jj < hd; ++jj) s = fmaf(qs[g * hd + jj], Ks[r * hd + jj], s);
-        ps[r * gq + g] = s;
+        const bool kept = kept_here(args, args.sel[static_cast<int64_t>(u) * k + ti * kTileChunks + rr / chunk]);
+        ps[r * gq + g] = kept ? s : -INFINITY;
       }
       __syncthreads();
       if (tid < gq) {
         const int g = tid;
         float mx = ms[g];
         for (int r = 0; r < nr; ++r) mx = fmaxf(mx, ps[r * gq + g]);
-        al[g] = exp2f(ms[g] - mx);
+        al[g] = mx == -INFINITY ? 1.f : exp2f(ms[g] - mx);
         float sum = 0.f;
         for (int r = 0; r < nr; ++r) {
-          const float pv = exp2f(ps[r * gq + g] - mx);
+          const float pv = mx == -INFINITY ? 0.f : exp2f(ps[r * gq + g] - mx);
           ps[r * gq + g] = pv;
           sum += pv;
         }
@@ -1379,15 +1415,23 @@ __global__ void __launch_bounds__(256) sr_attend_simt_kernel(const T* __restrict
         ms[g] = mx;
       }
       __syncthreads();
-      // value rows: A_V [t][rV], or head h's columns of V [t][d] when uncompressed
-      const int64_t vld = args.v_raw ? d : args.rV;
-      const T* avb = AV + b * sav + (args.v_raw ? h * hd : 0);
+      // value rows: A_V [t][rV]; head h's columns of V [t][d] when uncompressed;
+      // the unit's staged rows [k][chunk][hd] when gathered from host memory
+      const int64_t vld = args.v_raw == 1 ? d : args.rV;
+      const T* avb = args.v_raw == 2 ? AV + static_cast<int64_t>(u) * k * chunk * hd
+                                      : AV + b * sav + (args.v_raw ? h * hd : 0);
       for (int i = tid; i < gq * args.rV; i += blockDim.x) {
         const int g = i / args.rV, c = i % args.rV;
         float acc = us[i] * al[g];
         for (int r = 0; r < nr; ++r) {
           const int rr = rb + r;
-          const int64_t t = args.sink + static_cast<int64_t>(args.sel[static_cast<int64_t>(u) * k + ti * kTileChunks + rr / chunk]) * chunk + rr % chunk;
+          const int64_t t =
+              args.v_raw == 2
+                  ? static_cast<int64_t>(ti * kTileChunks + rr / chunk) * chunk + rr % chunk
+                  : args.sink +
+                        static_cast<int64_t>(kept_here(args, args.sel[static_cast<int64_t>(u) * k + ti * kTileChunks + rr / chunk])
+                                                 ? args.sel[static_cast<int64_t>(u) * k + ti * kTileChunks + rr / chunk] - args.c_lo
+                                                 : 0) * chunk + rr % chunk;
           acc = fmaf(ps[r * gq + g], to_f(avb[t * vld + c]), acc);
         }
         us[i] = acc;
@@ -1404,6 +1448,47 @@ __global__ void __launch_bounds__(256) sr_attend_simt_kernel(const T* __restrict
   }
 }
 
+
+// ------------------------------------------------ host-resident values
+// xK-SR with the uncompressed values off the GPU (the xKV explainer,
+// "选择性重建": the value cache stays in host memory and only the selected
+// tokens' rows are fetched): the kept chunks' rows of head h, read from
+// page-locked host memory over the host link with 16-byte loads, land in a
+// device staging buffer [units][k][chunk][hd] that the attend kernels read.
+template <typename T>
+__global__ void __launch_bounds__(256) gather_host_values_kernel(const T* __restrict__ V, int64_t vbs,
+                                                                 const int32_t* __restrict__ sel, int k, int Hkv,
+                                                                 int hd, int chunk, int sink, T* __restrict__ stage) {
+  allow_next_grid();
+  wait_prior_grid();  // the selection
+  constexpr int kVec = 16 / sizeof(T);
+  constexpr int kUnroll = 4;
+  const int u = blockIdx.y, b = u / Hkv, h = u % Hkv;
+  const int64_t d = static_cast<int64_t>(Hkv) * hd;
+  const int per_row = hd / kVec;
+  const int64_t total = static_cast<int64_t>(k) * chunk * per_row;  // 16-byte pieces of the unit
+  const int64_t step = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t i0 = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i0 < total; i0 += kUnroll * step) {
+    uint4 v[kUnroll];
+    int64_t dst[kUnroll];
+#pragma unroll
+    for (int r = 0; r < kUnroll; ++r) {
+      const int64_t i = i0 + r * step;
+      dst[r] = -1;
+      if (i < total) {
+        const int piece = static_cast<int>(i % per_row);
+        const int64_t rr = i / per_row;  // staged row of the unit
+        const int pos = static_cast<int>(rr / chunk), e = static_cast<int>(rr % chunk);
+        const int64_t t = sink + static_cast<int64_t>(sel[static_cast<int64_t>(u) * k + pos]) * chunk + e;
+        v[r] = *reinterpret_cast<const uint4*>(V + b * vbs + t * d + h * hd + piece * kVec);
+        dst[r] = ((static_cast<int64_t>(u) * k + pos) * chunk + e) * hd + piece * kVec;
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < kUnroll; ++r)
+      if (dst[r] >= 0) *reinterpret_cast<uint4*>(stage + dst[r]) = v[r];
+  }
+}
 
 size_t combine_smem(int gq, int rV, int hd) {
   const int cols = (hd + kCombineSplit - 1) / kCombineSplit;
@@ -1496,7 +1581,7 @@ template <typename T>
 static xkv_status sr_launch_t(const xkv_sr_params* p, const SRPlan& plan, const void* q, const void* A_K,
                               const void* Bt_K, const void* A_V, const void* Bt_V, const void* lm,
                               const void* sr_K, const void* sr_V, float* out, int32_t* sel_out, void* ws,
-                              cudaStream_t st) {
+                              const void* v_host, void* stage, const SRShard* shard, cudaStream_t st) {
   const int64_t n_mid = (p->T - p->sink - p->recent) / p->chunk;
   const int gq = p->n_q_heads / p->n_kv_heads;
   uint8_t* w = static_cast<uint8_t*>(ws);
@@ -1510,8 +1595,10 @@ static xkv_status sr_launch_t(const xkv_sr_params* p, const SRPlan& plan, const 
     const int cpb = 512;
     dim3 grid(static_cast<unsigned>((n_mid + cpb - 1) / cpb), static_cast<unsigned>(plan.units));
     const int64_t lm_cap = p->landmark_capacity > 0 ? p->landmark_capacity : n_mid;
-    sr_score_kernel<T><<<grid, 256, 0, st>>>(static_cast<const T*>(q), static_cast<const T*>(lm), scores,
-                                             p->n_q_heads, p->n_kv_heads, p->head_dim, n_mid, lm_cap, cpb);
+    if (!shard)
+      sr_score_kernel<T><<<grid, 256, 0, st>>>(static_cast<const T*>(q), static_cast<const T*>(lm), scores,
+                                               p->n_q_heads, p->n_kv_heads, p->head_dim, n_mid, lm_cap,
+                                               (n_mid + 3) & ~int64_t(3), cpb);
     if (cudaPeekAtLastError() != cudaSuccess) return XKV_ERR_CUDA;
   }
   prof_mark(1, st);
@@ -1530,6 +1617,7 @@ static xkv_status sr_launch_t(const xkv_sr_params* p, const SRPlan& plan, const 
     wa.hd = p->head_dim;
     wa.sink = p->sink;
     wa.recent = p->recent;
+    wa.pos_off = shard ? shard->pos_off : 0;
     for (int j = 0; j < 128; ++j) wa.ft[j] = j < p->head_dim / 2 ? rope_turns(p->rope_theta, j, p->head_dim) : 0.0;
     const int nsr = p->sink + p->recent;
     const int64_t per = (n_mid + kTopkThreads - 1) / kTopkThreads;
@@ -1538,21 +1626,39 @@ static xkv_status sr_launch_t(const xkv_sr_params* p, const SRPlan& plan, const 
     // the opt-in covers static + dynamic shared memory above 48 KiB
     cudaFuncSetAttribute(sr_topk_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     const int64_t ld = (n_mid + 3) & ~int64_t(3);
-    if (launch_after_prior(sr_topk_kernel<T>, dim3(2 * plan.units), dim3(kTopkThreads), smem, st,
+    // with a given selection only the window blocks run (top-k units = 0)
+    const int topk_units = shard ? 0 : static_cast<int>(plan.units);
+    if (launch_after_prior(sr_topk_kernel<T>, dim3(topk_units + plan.units), dim3(kTopkThreads), smem, st,
                            static_cast<const float*>(scores), ld, sel, sel_out, n_mid, static_cast<int>(p->topk),
-                           static_cast<int>(plan.units), wa) != cudaSuccess)
+                           topk_units, wa) != cudaSuccess)
       return XKV_ERR_CUDA;
   }
   prof_mark(2, st);
   AttendArgs a;
-  a.sel = sel;
+  a.sel = shard ? shard->sel : sel;
+  a.pos_off = shard ? shard->pos_off : 0;
+  a.c_lo = shard ? shard->c_lo : 0;
+  a.c_hi = shard ? shard->c_hi : static_cast<int>(n_mid);
+  a.ml_out = shard ? shard->ml_out : nullptr;
   a.q = q;
   a.part = part;
   a.status = device_status_ptr();
   a.T = p->T;
   a.sbk = p->bt_k_batch_stride;
-  // Bt_V absent: the xK-SR mode, A_V is the uncompressed V [B][T][d] and rank_v = hd
-  a.v_raw = Bt_V == nullptr ? 1 : 0;
+  // Bt_V absent: the xK-SR mode, A_V is the uncompressed V [B][T][d] and rank_v = hd;
+  // with v_host, that V is in page-locked host memory and the kept rows are
+  // first gathered into the staging buffer
+  a.v_raw = v_host ? 2 : (Bt_V == nullptr ? 1 : 0);
+  if (v_host) {
+    dim3 grid(static_cast<unsigned>(std::max(1, std::min(64, p->topk / 4))), static_cast<unsigned>(plan.units));
+    if (launch_after_prior(gather_host_values_kernel<T>, grid, dim3(256), 0, st, static_cast<const T*>(v_host),
+                           p->a_v_batch_stride, static_cast<const int32_t*>(sel), static_cast<int>(p->topk),
+                           static_cast<int>(p->n_kv_heads), static_cast<int>(p->head_dim),
+                           static_cast<int>(p->chunk), static_cast<int>(p->sink), static_cast<T*>(stage)) !=
+        cudaSuccess)
+      return XKV_ERR_CUDA;
+    A_V = stage;
+  }
   a.sbv = a.v_raw ? 0 : p->bt_v_batch_stride;
   a.Hq = p->n_q_heads;
   a.Hkv = p->n_kv_heads;
@@ -1593,11 +1699,16 @@ static xkv_status sr_launch_t(const xkv_sr_params* p, const SRPlan& plan, const 
     }
     {
       // (64 columns, token rows, atoms, batch): one box = 8 rows x the full rank;
-      // uncompressed values: rows of d columns, one box = 8 rows x head h's hd columns
-      const int vcols = a.v_raw ? d : p->rank_v;
-      const uint64_t dims[4] = {64, static_cast<uint64_t>(p->T), static_cast<uint64_t>(vcols / 64),
-                                static_cast<uint64_t>(p->batch)};
-      const uint64_t str[3] = {static_cast<uint64_t>(vcols) * 2, 128, static_cast<uint64_t>(p->a_v_batch_stride) * 2};
+      // uncompressed values: rows of d columns, one box = 8 rows x head h's hd columns;
+      // staged values: (64 columns, staged rows k chunk, atoms, units)
+      const int vcols = a.v_raw == 1 ? d : p->rank_v;
+      const bool staged = a.v_raw == 2;
+      const uint64_t dims[4] = {64, static_cast<uint64_t>(staged ? static_cast<int64_t>(p->topk) * 8 : p->T),
+                                static_cast<uint64_t>(vcols / 64),
+                                static_cast<uint64_t>(staged ? plan.units : p->batch)};
+      const uint64_t str[3] = {static_cast<uint64_t>(vcols) * 2, 128,
+                               static_cast<uint64_t>(staged ? static_cast<int64_t>(p->topk) * 8 * vcols
+                                                            : p->a_v_batch_stride) * 2};
       const uint32_t box[4] = {64, 8, static_cast<uint32_t>(p->rank_v / 64), 1};
       if (!make_tmap(&mAV, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, A_V, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B))
         return XKV_ERR_CUDA;
@@ -1643,6 +1754,68 @@ static xkv_status sr_launch_t(const xkv_sr_params* p, const SRPlan& plan, const 
   return cudaPeekAtLastError() == cudaSuccess ? XKV_OK : XKV_ERR_CUDA;
 }
 
+// ------------------------------------------------------- token sharding
+xkv_status sr_scores_launch(const xkv_sr_params* p, const void* q, const void* lm, float* scores, int64_t ld,
+                            cudaStream_t st) {
+  const int64_t n_mid = (p->T - p->sink - p->recent) / p->chunk;
+  const int units = p->batch * p->n_kv_heads;
+  const int cpb = 512;
+  const int64_t lm_cap = p->landmark_capacity > 0 ? p->landmark_capacity : n_mid;
+  dim3 grid(static_cast<unsigned>((n_mid + cpb - 1) / cpb), static_cast<unsigned>(units));
+  if (p->dtype == XKV_BF16)
+    sr_score_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(q),
+                                                          static_cast<const __nv_bfloat16*>(lm), scores, p->n_q_heads,
+                                                          p->n_kv_heads, p->head_dim, n_mid, lm_cap, ld, cpb);
+  else
+    sr_score_kernel<float><<<grid, 256, 0, st>>>(static_cast<const float*>(q), static_cast<const float*>(lm), scores,
+                                                  p->n_q_heads, p->n_kv_heads, p->head_dim, n_mid, lm_cap, ld, cpb);
+  return cudaPeekAtLastError() == cudaSuccess ? XKV_OK : XKV_ERR_CUDA;
+}
+
+xkv_status sr_topk_launch(const float* scores, int64_t ld, int units, int64_t n, int k, int32_t* sel,
+                          cudaStream_t st) {
+  const int64_t per = (n + kTopkThreads - 1) / kTopkThreads;
+  const size_t smem = static_cast<size_t>(per * kTopkThreads + n) * 4 + static_cast<size_t>(n) + 16;
+  cudaFuncSetAttribute(sr_topk_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  WinArgs wa{};
+  sr_topk_kernel<float><<<units, kTopkThreads, smem, st>>>(scores, ld, sel, nullptr, n, k, units, wa);
+  return cudaPeekAtLastError() == cudaSuccess ? XKV_OK : XKV_ERR_CUDA;
+}
+
+// Merge of per-shard decode partials: row i (sequence, query head) of shard r
+// holds the output o_r normalised by its own softmax sum L_r and the running
+// maximum M_r (log2 units); the whole-sequence output is
+//   sum_r 2^(M_r - M) L_r o_r / sum_r 2^(M_r - M) L_r,  M = max_r M_r,
+// shards with L_r = 0 (nothing of theirs kept) contributing nothing.
+__global__ void merge_partials_kernel(const float* __restrict__ o, const float* __restrict__ ml, int R, int rows,
+                                      int hd, float* __restrict__ out) {
+  const int i = blockIdx.x;
+  float M = -INFINITY;
+  for (int r = 0; r < R; ++r) {
+    const float* m = ml + (static_cast<int64_t>(r) * rows + i) * 2;
+    if (m[1] > 0.f) M = fmaxf(M, m[0]);
+  }
+  float den = 0.f;
+  for (int r = 0; r < R; ++r) {
+    const float* m = ml + (static_cast<int64_t>(r) * rows + i) * 2;
+    if (m[1] > 0.f) den += exp2f(m[0] - M) * m[1];
+  }
+  for (int j = threadIdx.x; j < hd; j += blockDim.x) {
+    float num = 0.f;
+    for (int r = 0; r < R; ++r) {
+      const float* m = ml + (static_cast<int64_t>(r) * rows + i) * 2;
+      if (m[1] > 0.f) num = fmaf(exp2f(m[0] - M) * m[1], o[(static_cast<int64_t>(r) * rows + i) * hd + j], num);
+    }
+    out[static_cast<int64_t>(i) * hd + j] = den > 0.f ? num / den : 0.f;
+  }
+}
+
+xkv_status merge_partials_launch(const float* o, const float* ml, int R, int rows, int hd, float* out,
+                                 cudaStream_t st) {
+  merge_partials_kernel<<<rows, 128, 0, st>>>(o, ml, R, rows, hd, out);
+  return cudaPeekAtLastError() == cudaSuccess ? XKV_OK : XKV_ERR_CUDA;
+}
+
 xkv_status sr_profile_enable(int enable) {
   if (!enable) {
     g_prof.on = false;
@@ -1674,10 +1847,13 @@ xkv_status sr_profile_read(float* stage_ms) {
 
 xkv_status sr_launch(const xkv_sr_params* p, const SRPlan& plan, const void* q, const void* A_K, const void* Bt_K,
                      const void* A_V, const void* Bt_V, const void* landmarks, const void* sr_K, const void* sr_V,
-                     float* out, int32_t* sel_out, void* ws, cudaStream_t st) {
+                     float* out, int32_t* sel_out, void* ws, cudaStream_t st, const void* v_host, void* stage,
+                     const SRShard* shard) {
   if (p->dtype == XKV_BF16)
-    return sr_launch_t<__nv_bfloat16>(p, plan, q, A_K, Bt_K, A_V, Bt_V, landmarks, sr_K, sr_V, out, sel_out, ws, st);
-  return sr_launch_t<float>(p, plan, q, A_K, Bt_K, A_V, Bt_V, landmarks, sr_K, sr_V, out, sel_out, ws, st);
+    return sr_launch_t<__nv_bfloat16>(p, plan, q, A_K, Bt_K, A_V, Bt_V, landmarks, sr_K, sr_V, out, sel_out, ws,
+                                      v_host, stage, shard, st);
+  return sr_launch_t<float>(p, plan, q, A_K, Bt_K, A_V, Bt_V, landmarks, sr_K, sr_V, out, sel_out, ws, v_host,
+                            stage, shard, st);
 }
 
 }  // namespace xkv

@@ -532,6 +532,137 @@ xkv_status xkv_sr_append(const xkv_append_params* p, const void* const* k_new, c
                        static_cast<cudaStream_t>(stream));
 }
 
+// ------------------------------------ xK-SR decode, values in host memory
+static size_t host_stage_bytes(const xkv_sr_params* pv) {
+  const size_t es = pv->dtype == XKV_BF16 ? 2 : 4;
+  return align_up(static_cast<size_t>(pv->batch) * pv->n_kv_heads * pv->topk * pv->chunk * pv->head_dim * es);
+}
+
+xkv_status xkv_xk_sr_host_workspace_size(const xkv_sr_params* p, size_t* bytes) {
+  if (!bytes) return XKV_ERR_INVALID_ARG;
+  xkv_sr_params pv;
+  const xkv_status s = xk_params(p, &pv);
+  if (s != XKV_OK) return s;
+  SRPlan plan;
+  sr_plan(&pv, &plan);
+  *bytes = align_up(plan.bytes) + host_stage_bytes(&pv);
+  return XKV_OK;
+}
+
+xkv_status xkv_xk_sr_attention_decode_host_values(const xkv_sr_params* p, const void* q, const void* A_K,
+                                                  const void* Bt_K, const void* V_host, const void* landmarks,
+                                                  const void* sr_K, const void* sr_V, float* out, int32_t* sel_out,
+                                                  void* workspace, size_t ws_bytes, void* stream) {
+  xkv_sr_params pv;
+  const xkv_status s = xk_params(p, &pv);
+  if (s != XKV_OK) return s;
+  const void* ptrs[] = {q, A_K, Bt_K, V_host, landmarks, out};
+  for (const void* x : ptrs)
+    if (!x || !aligned16(x)) return XKV_ERR_INVALID_ARG;
+  if (p->sink + p->recent > 0 && (!sr_K || !sr_V || !aligned16(sr_K) || !aligned16(sr_V))) return XKV_ERR_INVALID_ARG;
+  if (sel_out && !aligned16(sel_out)) return XKV_ERR_INVALID_ARG;
+  const size_t es = p->dtype == XKV_BF16 ? 2 : 4;
+  if ((p->head_dim * es) % 16 != 0 || (p->a_v_batch_stride * es) % 16 != 0) return XKV_ERR_UNSUPPORTED;
+  // the values must be page-locked host memory mapped for the device
+  cudaPointerAttributes attr;
+  if (cudaPointerGetAttributes(&attr, V_host) != cudaSuccess || attr.type != cudaMemoryTypeHost) {
+    cudaGetLastError();
+    return XKV_ERR_INVALID_ARG;
+  }
+  void* v_dev = nullptr;
+  if (cudaHostGetDevicePointer(&v_dev, const_cast<void*>(V_host), 0) != cudaSuccess || !v_dev) {
+    cudaGetLastError();
+    return XKV_ERR_INVALID_ARG;
+  }
+  SRPlan plan;
+  sr_plan(&pv, &plan);
+  const size_t need = align_up(plan.bytes) + host_stage_bytes(&pv);
+  if (!workspace || ws_bytes < need || !aligned256(workspace)) return XKV_ERR_WORKSPACE;
+  void* stage = static_cast<uint8_t*>(workspace) + align_up(plan.bytes);
+  return sr_launch(&pv, plan, q, A_K, Bt_K, stage, nullptr, landmarks, sr_K, sr_V, out, sel_out, workspace,
+                   static_cast<cudaStream_t>(stream), v_dev, stage);
+}
+
+// ------------------------------------------------------- token sharding
+// the local slice of a token-sharded decode: p's own checks, with the global
+// k (topk) allowed above the local chunk count
+static xkv_status check_partial(const xkv_sr_params* p, xkv_sr_params* loc);
+
+xkv_status xkv_sr_scores(const xkv_sr_params* p, const void* q, const void* landmarks, float* scores, int64_t ld,
+                         void* stream) {
+  xkv_sr_params loc;
+  xkv_status s = check_partial(p, &loc);
+  if (s != XKV_OK) return s;
+  const int64_t n_mid = (p->T - p->sink - p->recent) / p->chunk;
+  if (!q || !landmarks || !scores || !aligned16(q) || !aligned16(landmarks) || !aligned16(scores) || ld < n_mid ||
+      ld % 4 != 0)
+    return XKV_ERR_INVALID_ARG;
+  return sr_scores_launch(p, q, landmarks, scores, ld, static_cast<cudaStream_t>(stream));
+}
+
+xkv_status xkv_sr_topk(const float* scores, int64_t ld, int rows, int64_t n, int k, int32_t* sel_out, void* stream) {
+  if (!scores || !sel_out || !aligned16(scores) || !aligned16(sel_out) || rows < 1 || n < 1 || k < 1 || k > n ||
+      ld < n || ld % 4 != 0)
+    return XKV_ERR_INVALID_ARG;
+  if (n > kMaxMidChunks || k > 1024) return XKV_ERR_UNSUPPORTED;
+  return sr_topk_launch(scores, ld, rows, n, k, sel_out, static_cast<cudaStream_t>(stream));
+}
+
+static xkv_status check_partial(const xkv_sr_params* p, xkv_sr_params* loc) {
+  if (!p) return XKV_ERR_INVALID_ARG;
+  *loc = *p;
+  if (p->chunk < 1 || p->T < p->sink + p->recent + p->chunk) return XKV_ERR_INVALID_ARG;
+  const int64_t n_mid = (p->T - p->sink - p->recent) / p->chunk;
+  if (p->topk < 1 || p->topk > 1024) return p->topk < 1 ? XKV_ERR_INVALID_ARG : XKV_ERR_UNSUPPORTED;
+  loc->topk = static_cast<int>(std::min<int64_t>(p->topk, n_mid));
+  const xkv_status s = check_sr(loc);
+  *loc = *p;
+  return s;
+}
+
+xkv_status xkv_sr_partial_workspace_size(const xkv_sr_params* p, size_t* bytes) {
+  if (!bytes) return XKV_ERR_INVALID_ARG;
+  xkv_sr_params loc;
+  const xkv_status s = check_partial(p, &loc);
+  if (s != XKV_OK) return s;
+  SRPlan plan;
+  sr_plan(&loc, &plan);
+  *bytes = plan.bytes;
+  return XKV_OK;
+}
+
+xkv_status xkv_sr_attention_partial(const xkv_sr_params* p, const xkv_sr_shard* shard, const int32_t* sel,
+                                    const void* q, const void* A_K, const void* Bt_K, const void* A_V,
+                                    const void* Bt_V, const void* sr_K, const void* sr_V, float* out, float* ml_out,
+                                    void* workspace, size_t ws_bytes, void* stream) {
+  xkv_sr_params loc;
+  const xkv_status s = check_partial(p, &loc);
+  if (s != XKV_OK) return s;
+  if (!shard || shard->position_offset < 0 || shard->chunk_begin < 0 || shard->chunk_begin > (int64_t(1) << 30))
+    return XKV_ERR_INVALID_ARG;
+  const void* ptrs[] = {sel, q, A_K, Bt_K, A_V, Bt_V, out, ml_out};
+  for (const void* x : ptrs)
+    if (!x || !aligned16(x)) return XKV_ERR_INVALID_ARG;
+  if (p->sink + p->recent > 0 && (!sr_K || !sr_V || !aligned16(sr_K) || !aligned16(sr_V))) return XKV_ERR_INVALID_ARG;
+  SRPlan plan;
+  sr_plan(&loc, &plan);
+  if (!workspace || ws_bytes < plan.bytes || !aligned256(workspace)) return XKV_ERR_WORKSPACE;
+  const int64_t n_mid = (p->T - p->sink - p->recent) / p->chunk;
+  SRShard sh;
+  sh.sel = sel;
+  sh.pos_off = shard->position_offset;
+  sh.c_lo = static_cast<int>(shard->chunk_begin);
+  sh.c_hi = static_cast<int>(shard->chunk_begin + n_mid);
+  sh.ml_out = ml_out;
+  return sr_launch(&loc, plan, q, A_K, Bt_K, A_V, Bt_V, nullptr, sr_K, sr_V, out, nullptr, workspace,
+                   static_cast<cudaStream_t>(stream), nullptr, nullptr, &sh);
+}
+
+xkv_status xkv_merge_partials(const float* o, const float* ml, int R, int rows, int hd, float* out, void* stream) {
+  if (!o || !ml || !out || R < 1 || rows < 1 || hd < 1) return XKV_ERR_INVALID_ARG;
+  return merge_partials_launch(o, ml, R, rows, hd, out, static_cast<cudaStream_t>(stream));
+}
+
 // --------------------------------------------------- full reconstruction
 xkv_status xkv_full_reconstruct(const void* A, const void* Bt, int64_t T, int rank, int d, int n_kv_heads,
                                 int head_dim, int apply_rope, float rope_theta, xkv_dtype dt, void* out, void* stream) {

@@ -38,10 +38,28 @@ constexpr int64_t kMaxMidChunks = 24576;
 xkv_status sr_plan(const xkv_sr_params* p, SRPlan* plan);
 xkv_status sr_profile_enable(int enable);
 xkv_status sr_profile_read(float* stage_ms);
+// A token shard of the sequence: the selection is given (global chunk
+// indices), only chunks in [c_lo, c_hi) are kept here, local row 0 sits at
+// global position pos_off, and (M, L) per query head are written to ml_out.
+struct SRShard {
+  const int32_t* sel;
+  int64_t pos_off;
+  int c_lo, c_hi;
+  float* ml_out;
+};
+// v_host (optional): the xK-SR value cache in page-locked host memory (device
+// address); its kept rows are gathered into `stage` [units][k][chunk][hd].
 xkv_status sr_launch(const xkv_sr_params* p, const SRPlan& plan, const void* q, const void* A_K,
                      const void* Bt_K, const void* A_V, const void* Bt_V, const void* landmarks,
                      const void* sr_K, const void* sr_V, float* out, int32_t* sel_out, void* ws,
-                     cudaStream_t st);
+                     cudaStream_t st, const void* v_host = nullptr, void* stage = nullptr,
+                     const SRShard* shard = nullptr);
+xkv_status sr_scores_launch(const xkv_sr_params* p, const void* q, const void* lm, float* scores, int64_t ld,
+                            cudaStream_t st);
+xkv_status sr_topk_launch(const float* scores, int64_t ld, int units, int64_t n, int k, int32_t* sel,
+                          cudaStream_t st);
+xkv_status merge_partials_launch(const float* o, const float* ml, int R, int rows, int hd, float* out,
+                                 cudaStream_t st);
 
 // --------------------------------------------------------- dense / recon
 size_t dense_workspace(const xkv_dense_params* p);

@@ -321,6 +321,79 @@ XKV_API xkv_status xkv_sr_append(const xkv_append_params* p, const void* const* 
                          void* A_K, void* A_V, void* const* landmarks, int* rolled, void* workspace,
                          size_t ws_bytes, void* stream);
 
+/* The xK-SR step with the uncompressed values in host memory, where the
+ * explainer ([xKV-blog] "选择性重建") keeps them: scores, the exact top-k and
+ * the rebuilt keys are those of xkv_xk_sr_attention_decode; then, for every
+ * (sequence b, KV head h), the kept chunks' rows of head h's columns are read
+ * from V_host over the host link into a device staging buffer (only those
+ * k chunk rows cross, never the whole cache), and attention proceeds as in
+ * the HBM-resident mode.
+ *   V_host    : [B][T][d] in p->dtype, page-locked host memory mapped for the
+ *               device (e.g. cudaHostAlloc / cudaHostRegister), 16-byte
+ *               aligned, batch stride p->a_v_batch_stride; anything else
+ *               (device or pageable memory) returns XKV_ERR_INVALID_ARG.
+ *   workspace : xkv_xk_sr_host_workspace_size bytes (the SR scratch plus the
+ *               staging buffer, B Hkv k chunk hd elements).
+ * head_dim times the element size must be a multiple of 16 bytes.  Every other
+ * argument, layout and error is that of xkv_xk_sr_attention_decode. */
+XKV_API xkv_status xkv_xk_sr_host_workspace_size(const xkv_sr_params* p, size_t* bytes);
+XKV_API xkv_status xkv_xk_sr_attention_decode_host_values(const xkv_sr_params* p, const void* q, const void* A_K,
+                                                  const void* Bt_K, const void* V_host, const void* landmarks,
+                                                  const void* sr_K, const void* sr_V, float* out,
+                                                  int32_t* sel_out, void* workspace, size_t ws_bytes,
+                                                  void* stream);
+
+/* --------------------------------------------------- token sharding */
+/* The path split over devices by tokens.  Prefill: [KV-CoRE] 2.A accumulates
+ * the covariance over streamed token rows, so per-device Grams add up: each
+ * device runs xkv_gram_accumulate on its rows, an all-reduce sums the Grams,
+ * every device runs xkv_factor_gram on the sum (same Gram and seed, same
+ * basis) and xkv_project on its own rows.  Decode: each device holds a
+ * contiguous slice of the token sequence (the sink on the first, the recent
+ * window on the last, whole middle chunks in between); per step
+ *   1. xkv_sr_scores   : chunk scores of the local middle chunks;
+ *   2. (all-gather of the scores, laid out chunk-major per (b, h))
+ *      xkv_sr_topk     : the exact top-k over all chunks, the same on every
+ *                        device ([xKV-blog] "选择性重建");
+ *   3. xkv_sr_attention_partial : attention over the kept chunks that are held
+ *                        here plus the local window rows, as a partial
+ *                        (o normalised by its own softmax sum L, and M);
+ *   4. (all-gather of the partials) xkv_merge_partials : the exact softmax
+ *                        combination of the partials.
+ * One device with the whole sequence gives xkv_sr_attention_decode's result. */
+typedef struct xkv_sr_shard {
+  int64_t position_offset; /* global position of local token row 0 */
+  int64_t chunk_begin;     /* global index of the first middle chunk held here */
+} xkv_sr_shard;
+
+/* Chunk scores s_c = sum_{g in group(h)} q_g . landmark[b][h][c] of the local
+ * middle chunks (n_mid = (T - sink - recent) / chunk of p); scores is
+ * [B][Hkv] rows of n_mid f32 with row stride ld (>= n_mid, multiple of 4). */
+XKV_API xkv_status xkv_sr_scores(const xkv_sr_params* p, const void* q, const void* landmarks, float* scores,
+                         int64_t ld, void* stream);
+/* Exact top-k of each of `rows` score rows of n entries (row stride ld, a
+ * multiple of 4, >= n): the k largest, ties to the lower index, ascending.
+ * n <= 24576, 1 <= k <= min(n, 1024). */
+XKV_API xkv_status xkv_sr_topk(const float* scores, int64_t ld, int rows, int64_t n, int k, int32_t* sel_out,
+                       void* stream);
+/* Attention of one device's token slice for a given selection.  p describes
+ * the local slice (T local rows, its own sink / recent rows, topk = the global
+ * k); sel [B][Hkv][topk] holds global chunk indices, of which those in
+ * [chunk_begin, chunk_begin + n_mid) are attended here (row sink + (c -
+ * chunk_begin) chunk, RoPE at position_offset + row).  out [B][Hq][hd] is the
+ * partial normalised by its own sum L; ml_out [B][Hq][2] = (M, L), M the
+ * running maximum of the scores scaled by log2(e)/sqrt(hd), (-inf, 0) when
+ * nothing is held here.  Workspace: xkv_sr_partial_workspace_size. */
+XKV_API xkv_status xkv_sr_partial_workspace_size(const xkv_sr_params* p, size_t* bytes);
+XKV_API xkv_status xkv_sr_attention_partial(const xkv_sr_params* p, const xkv_sr_shard* shard, const int32_t* sel,
+                                    const void* q, const void* A_K, const void* Bt_K, const void* A_V,
+                                    const void* Bt_V, const void* sr_K, const void* sr_V, float* out,
+                                    float* ml_out, void* workspace, size_t ws_bytes, void* stream);
+/* out[i] = sum_r 2^(M_ri - M_i) L_ri o_ri / sum_r 2^(M_ri - M_i) L_ri over R
+ * partials (o [R][rows][hd], ml [R][rows][2]); rows = B Hq. */
+XKV_API xkv_status xkv_merge_partials(const float* o, const float* ml, int R, int rows, int hd, float* out,
+                              void* stream);
+
 /* -------------------------------------------------- full reconstruction */
 /* The comparison path of [xKV-blog] Fig. 6: rebuild every row,
  *   out[t][c] = sum_i A[t][i] Bt[c][i]   (T x d, `dt`),
