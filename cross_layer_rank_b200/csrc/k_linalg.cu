@@ -4,9 +4,9 @@
 //   - shifted Cholesky QR pieces (Gram of a tall block, Cholesky, triangular
 //     inverse) in fp64;
 //   - a one-sided block Jacobi eigen-solver (fp64) for symmetric positive
-//     semi-definite matrices: the Rayleigh-Ritz step (eigenvalues + vectors)
-//     and KV-CoRE's spectra (eigenvalues only);
-//   - ordering of eigenvalues and the NER reduction (KV-CoRE page, 2.B).
+//     semi-definite matrices: the Rayleigh-Ritz step (eigenvalues + vectors);
+//   - ordering of eigenvalues, and the NER and energy-rank reductions of
+//     KV-CoRE's spectra (2.B), whose eigenvalues come from k_spectrum.cu.
 #include <stdlib.h>
 
 #include <algorithm>
@@ -632,7 +632,7 @@ __global__ void extract_blocks_kernel(const float* __restrict__ C, int n, int bl
 size_t ner_workspace(int n, int block) {
   const int count = n / block;
   return align_up(static_cast<size_t>(count) * block * block * 8) + align_up(static_cast<size_t>(count) * block * 8) +
-         jacobi_workspace(block, count);
+         spectrum_workspace(block, count);
 }
 
 xkv_status ner_launch(const float* gram, int n, int block, double tol, float* ner, float* erank, int32_t* rank,
@@ -643,7 +643,7 @@ xkv_status ner_launch(const float* gram, int n, int block, double tol, float* ne
   double* lam = reinterpret_cast<double*>(w + align_up(static_cast<size_t>(count) * block * block * 8));
   void* jws = w + align_up(static_cast<size_t>(count) * block * block * 8) + align_up(static_cast<size_t>(count) * block * 8);
   extract_blocks_kernel<<<dim3(128, count), 256, 0, st>>>(gram, n, block, Wb);
-  xkv_status s = jacobi_launch(Wb, nullptr, lam, block, count, jws, st);
+  xkv_status s = spectrum_launch(Wb, lam, block, count, jws, st);
   if (s != XKV_OK) return s;
   ner_kernel<<<count, 256, 0, st>>>(lam, block, tol, ner, erank, rank);
   return cudaPeekAtLastError() == cudaSuccess ? XKV_OK : XKV_ERR_CUDA;
@@ -657,7 +657,7 @@ xkv_status energy_rank_launch(const float* gram, int n, int block, double energy
   double* lam = reinterpret_cast<double*>(w + align_up(static_cast<size_t>(count) * block * block * 8));
   void* jws = w + align_up(static_cast<size_t>(count) * block * block * 8) + align_up(static_cast<size_t>(count) * block * 8);
   extract_blocks_kernel<<<dim3(128, count), 256, 0, st>>>(gram, n, block, Wb);
-  xkv_status s = jacobi_launch(Wb, nullptr, lam, block, count, jws, st);
+  xkv_status s = spectrum_launch(Wb, lam, block, count, jws, st);
   if (s != XKV_OK) return s;
   const size_t smem = static_cast<size_t>(block) * 8;
   cudaFuncSetAttribute(energy_rank_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));

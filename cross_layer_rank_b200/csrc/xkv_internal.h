@@ -118,4 +118,10 @@ xkv_status ner_launch(const float* gram, int n, int block, double tol, float* ne
 size_t jacobi_workspace(int n, int count);
 xkv_status jacobi_launch(double* W, double* V, double* lam, int n, int count, void* ws, cudaStream_t st);
 
+// Eigenvalues only of `count` symmetric n x n problems (row-major fp64 at W,
+// overwritten): Householder tridiagonalisation and bisection; lam receives
+// each problem's eigenvalues in ascending order.
+size_t spectrum_workspace(int n, int count);
+xkv_status spectrum_launch(double* W, double* lam, int n, int count, void* ws, cudaStream_t st);
+
 }  // namespace xkv

@@ -40,21 +40,19 @@ import cross_layer_rank_b200 as xkv
 import synth
 w = synth.WORKLOADS["tiny_f32"]
 X = [torch.from_numpy(l).cuda() for l in synth.kv_group(w, 0, 0, "K")]
-n = 4 * w.d
-C = torch.zeros((n, n), dtype=torch.float32, device="cuda")
-xkv.xkv_gram_accumulate(X, C)
-ner = torch.empty(4, dtype=torch.float32, device="cuda")
-xkv.xkv_ner(C, w.d, ner)
+A = torch.empty((w.T, 64), dtype=torch.float32, device="cuda")
+Bt = torch.empty((4 * w.d, 64), dtype=torch.float32, device="cuda")
+xkv.xkv_compress_group(X, 64, A, Bt, oversample=64, shard_rows=512)
 print(xkv.get_device_status(), xkv.get_device_status())
 """
 
 
 @pytest.mark.parametrize("cap, expect", [("1", 5), ("", 0)])
 def test_unconverged_eigensolver_is_reported(xkv, cap, expect):
-    # the eigen-solver's sweep limit cut to one sweep (a diagnostic override
-    # read once per process, hence the child process) leaves the NER spectra
-    # unconverged: the device status reports XKV_ERR_NUMERICAL once, then 0;
-    # with the default limit nothing is reported
+    # the Rayleigh-Ritz eigen-solver's sweep limit cut to one sweep (a
+    # diagnostic override read once per process, hence the child process)
+    # leaves the Ritz problem unconverged: the device status reports
+    # XKV_ERR_NUMERICAL once, then 0; with the default limit nothing is reported
     import os
     import subprocess
     import sys
