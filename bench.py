@@ -284,8 +284,9 @@ def build_model(xkv, w, device, groups=None, log=print):
     return model, prefill
 
 
-def measure_gram(xkv, w, device):
-    """Device time of the Gram of one (batch 0, group 0) K shard set (T rows)."""
+def measure_gram(xkv, w, device, spectra=True):
+    """Device time of the Gram of one (batch 0, group 0) K shard set (T rows),
+    of KV-CoRE's NER and energy rank on it (spectra=True) and of A = X V_r."""
     import torch
     X = synth.kv_group_torch(w, 0, 0, "K", device)
     n = w.group * w.d
@@ -309,9 +310,10 @@ def measure_gram(xkv, w, device):
     # Gram (the diagonal d x d blocks; scale-invariant, so the repeated sums do)
     ner = torch.empty(w.group, dtype=torch.float32, device=device)
     wsn = xkv.workspace(xkv.xkv_ner_workspace_size(n, w.d), device)
+    todo = (("ner", lambda: xkv.xkv_ner(C, w.d, ner, ws=wsn)),
+            ("energy_rank_95", lambda: xkv.xkv_energy_rank(C, w.d, 0.95, ws=wsn))) if spectra else ()
     spectra = {}
-    for name, fn in (("ner", lambda: xkv.xkv_ner(C, w.d, ner, ws=wsn)),
-                     ("energy_rank_95", lambda: xkv.xkv_energy_rank(C, w.d, 0.95, ws=wsn))):
+    for name, fn in todo:
         fn()
         torch.cuda.synchronize()
         e0.record()
@@ -529,6 +531,17 @@ def run_cuda(args, rank, world, log):
             xk = measure_xk_sr(xkv, w, model, device, stream, L, args.steps, args.warmup, _peaks()[0])
         except Exception as e:  # noqa: BLE001
             log(f"xK-SR mode not measured: {e!r}")
+        try:
+            if xk is not None:
+                xk["host_values"] = measure_xk_sr_host(xkv, w, model, device, stream)
+        except Exception as e:  # noqa: BLE001
+            log(f"xK-SR with host values not measured: {e!r}")
+    appended = None
+    if world == 1 and args.xk:
+        try:
+            appended = measure_append(xkv, w, device, stream)
+        except Exception as e:  # noqa: BLE001
+            log(f"append not measured: {e!r}")
 
     ms_total, e2e_ms = max_over_ranks([ms_total, e2e_ms], world, device)
     ms_step = ms_total / args.steps
@@ -577,6 +590,8 @@ def run_cuda(args, rank, world, log):
         res["comparison"] = comparison
     if xk is not None:
         res["xk_sr"] = xk
+    if appended is not None:
+        res["multistep_append"] = appended
     if args.prefill:
         cm = prefill["compress_ms"]
         res["prefill"] = {"compress_group_ms_median": round(statistics.median(cm), 3), "groups_compressed": len(cm),
@@ -656,6 +671,85 @@ def measure_xk_sr(xkv, w, model, device, stream, L, steps, warmup, peak_gbs):
                                 "frac": round(gbs / peak_gbs, 4), "bytes_per_launch": bytes_attend},
             "value_cache_gb": round(L * w.batch * w.T * w.d * 2 / 1e9, 2),
             "cache_ratio": dict(zip(("a_b", "with_landmarks"), cache_ratio(w, values_compressed=False)))}
+
+
+def measure_xk_sr_host(xkv, w, model, device, stream, layers=4):
+    """The xK-SR step with the uncompressed values in pinned host memory (the
+    explainer's placement): per layer call only the kept chunks' value rows
+    (B Hkv k chunk hd elements) cross the host link.  Device time per layer call
+    (eager, median over calls) and the host-link bytes per call."""
+    import torch
+    bf = torch.bfloat16
+    Vh = torch.empty((w.batch, w.T, w.d), dtype=bf).pin_memory()
+    Vh.copy_(synth.normal_torch(synth.stream_key(w.name, "Vraw", 0, w.T), w.batch * w.T * w.d, device, bf)
+             .view(w.batch, w.T, w.d).cpu())
+    p = xkv.xk_sr_params(w.batch, w.n_q_heads, w.n_kv_heads, w.head_dim, w.T, w.rank_k, w.chunk, w.topk, w.sink,
+                         w.recent, w.rope_theta, bf)
+    ws = xkv.workspace(xkv.xkv_xk_sr_host_workspace_size(p), device)
+    out = torch.empty((w.batch, w.n_q_heads, w.head_dim), dtype=torch.float32, device=device)
+    times = []
+    with torch.cuda.stream(stream):
+        for i in range(3 * layers):
+            l = i % layers
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            xkv.xkv_xk_sr_attention_decode_host_values(p, model["q"][l], model["A_K"][l], model["Bt_K"][l], Vh,
+                                                       model["lm"][l], model["srK"][l], model["srV"][l], out, None,
+                                                       ws, stream)
+            e1.record(stream)
+            e1.synchronize()
+            if i >= layers:
+                times.append(e0.elapsed_time(e1))
+    assert xkv.get_device_status(stream) == 0
+    ms = statistics.median(times)
+    link = w.batch * w.n_kv_heads * w.topk * w.chunk * w.head_dim * 2
+    return {"path": "xkv_xk_sr_attention_decode_host_values (values in pinned host memory)",
+            "ms_per_layer_call": round(ms, 4), "host_link_bytes_per_call": link,
+            "host_link_gbs": round(link / (ms / 1e3) / 1e9, 2),
+            "note": "eager calls; the value rows cross the host link, the rest is the HBM-resident xK-SR step"}
+
+
+def measure_append(xkv, w, device, stream):
+    """xkv_sr_append for one group of the workload (batch, G layers): the device
+    time of an append that only writes the window, and of one that rolls a
+    chunk into the compressed cache (landmarks, projection of x onto the
+    stored bases, window move)."""
+    import torch
+    bf = torch.bfloat16
+    B, G, d, C = w.batch, w.group, w.d, w.chunk
+    n = G * d
+    T0 = w.sink + w.recent + C * 64
+    cap = 80
+    Tcap = w.sink + cap * C + w.recent + C
+    A_K = torch.zeros((B, Tcap, w.rank_k), dtype=bf, device=device)
+    A_V = torch.zeros((B, Tcap, w.rank_v), dtype=bf, device=device)
+    Bt_K = torch.randn((B, n, w.rank_k), device=device).to(bf)
+    Bt_V = torch.randn((B, n, w.rank_v), device=device).to(bf)
+    lms = [torch.zeros((B, w.n_kv_heads, cap, w.head_dim), dtype=bf, device=device) for _ in range(G)]
+    wk = [torch.randn((B, w.sink + w.recent + C, d), device=device).to(bf) for _ in range(G)]
+    wv = [torch.randn((B, w.sink + w.recent + C, d), device=device).to(bf) for _ in range(G)]
+    kn = [torch.randn((B, d), device=device).to(bf) for _ in range(G)]
+    vn = [torch.randn((B, d), device=device).to(bf) for _ in range(G)]
+    wbs = (w.sink + w.recent + C) * d
+    times = {False: [], True: []}
+    T = T0
+    with torch.cuda.stream(stream):
+        for _ in range(4 * C):
+            ap = xkv.append_params(B, G, w.n_kv_heads, w.head_dim, C, w.sink, w.recent, w.rope_theta, bf, T,
+                                   w.rank_k, w.rank_v, Tcap * w.rank_k, Tcap * w.rank_v, n * w.rank_k, n * w.rank_v,
+                                   wbs, cap)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            rolled = xkv.xkv_sr_append(ap, kn, vn, wk, wv, Bt_K, Bt_V, A_K, A_V, lms, stream=stream)
+            e1.record(stream)
+            e1.synchronize()
+            times[rolled].append(e0.elapsed_time(e1))
+            T += 1
+    assert xkv.get_device_status(stream) == 0
+    return {"path": "xkv_sr_append (one token per layer of a group; a chunk rolled every chunk steps)",
+            "append_ms": round(statistics.median(times[False]), 4),
+            "append_with_roll_ms": round(statistics.median(times[True]), 4),
+            "group": f"batch {B}, G = {G}, d = {d}, ranks {w.rank_k} / {w.rank_v}"}
 
 
 def measure_full_reconstruction(xkv, w, model, device, stream, sr_call_ms):
@@ -763,6 +857,9 @@ def main():
                     help="comma-separated further workloads measured on one GPU (empty string: none)")
     ap.add_argument("--no-comparison", dest="comparison", action="store_false",
                     help="skip timing the full-reconstruction comparison path")
+    ap.add_argument("--prefill-only", action="store_true",
+                    help="time only the compression kernels (Gram, projection, the compression sweep) and print "
+                         "them; no decode step (a profiling aid)")
     args = ap.parse_args()
     rank = int(os.environ.get("RANK", 0))
     world = int(os.environ.get("WORLD_SIZE", 1))
@@ -771,6 +868,20 @@ def main():
     if args.impl == "reference":
         if rank == 0:
             print(json.dumps(run_reference(args, log)), flush=True)
+        return
+    if args.prefill_only:
+        import torch
+        import cross_layer_rank_b200 as xkv
+        device = torch.device("cuda", 0)
+        w = synth.WORKLOADS[args.workload]
+        _, bf16_peak, _, _ = _peaks()
+        gram_ms, gram_flops, _, proj_ms, proj_flops = measure_gram(xkv, w, device, spectra=False)
+        res = {"workload": w.name, "gram_ms": round(gram_ms, 4),
+               "gram_frac_of_bf16_peak": round(gram_flops / (gram_ms / 1e3) / 1e12 / bf16_peak, 4),
+               "projection_ms": round(proj_ms, 4),
+               "projection_frac_of_bf16_peak": round(proj_flops / (proj_ms / 1e3) / 1e12 / bf16_peak, 4),
+               "sweep": measure_compress_sweep(xkv, device, bf16_peak, log)}
+        print(json.dumps(res), flush=True)
         return
     if world > 1:
         import datetime
