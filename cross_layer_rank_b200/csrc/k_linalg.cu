@@ -18,33 +18,63 @@
 namespace xkv {
 
 // --------------------------------------------------------------- SIMT GEMM
+// 64 x 64 output tile per CTA, 16-deep K slabs through shared memory; the next
+// slab's global loads are issued before the current slab's products, so their
+// latency overlaps the arithmetic.  Split K (gridDim.z > 1): slice z covers
+// K rows [z kchunk, (z + 1) kchunk) and writes alpha * its sum to
+// part[z][M][N]; gemm_reduce_kernel then sums the slices in a fixed order
+// (deterministic).  lower: tiles wholly above the diagonal are skipped.
 template <typename TA, typename TB, typename TC, typename ACC>
 __global__ void __launch_bounds__(256) gemm_simt_kernel(const TA* __restrict__ A, int64_t sam, int64_t sak,
                                                         const TB* __restrict__ B, int64_t sbk, int64_t sbn,
                                                         TC* __restrict__ C, int64_t ldc, int M, int N, int K,
-                                                        double alpha, double beta) {
+                                                        double alpha, double beta, ACC* __restrict__ part,
+                                                        int kchunk, int lower) {
   __shared__ ACC As[16][65];
   __shared__ ACC Bs[16][65];
   const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
   const int m0 = blockIdx.y * 64, n0 = blockIdx.x * 64;
+  if (lower && n0 >= m0 + 64) return;
+  const int kb = blockIdx.z * kchunk, ke = min(K, kb + kchunk);
+  // element q of this thread's share of a slab: A at (kk, mm), B at (kb2, nn);
+  // the order makes consecutive threads touch consecutive memory
+  auto a_idx = [&](int q, int& kk, int& mm) {
+    const int i = threadIdx.x + q * 256;
+    if (sam == 1) { mm = i & 63; kk = i >> 6; } else { kk = i & 15; mm = i >> 4; }
+  };
+  auto b_idx = [&](int q, int& kk, int& nn) {
+    const int i = threadIdx.x + q * 256;
+    if (sbn == 1) { nn = i & 63; kk = i >> 6; } else { kk = i & 15; nn = i >> 4; }
+  };
+  ACC ra[4], rb[4];
+  auto load = [&](int k0) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      int kk, mm, k2, nn;
+      a_idx(q, kk, mm);
+      b_idx(q, k2, nn);
+      const int m = m0 + mm, k = k0 + kk, n = n0 + nn, kB = k0 + k2;
+      ra[q] = (m < M && k < ke) ? static_cast<ACC>(to_f_any(A[m * sam + k * sak])) : ACC(0);
+      rb[q] = (n < N && kB < ke) ? static_cast<ACC>(to_f_any(B[kB * sbk + n * sbn])) : ACC(0);
+    }
+  };
   ACC acc[4][4];
 #pragma unroll
   for (int i = 0; i < 4; ++i)
 #pragma unroll
     for (int j = 0; j < 4; ++j) acc[i][j] = ACC(0);
-  for (int k0 = 0; k0 < K; k0 += 16) {
-    for (int i = threadIdx.x; i < 16 * 64; i += 256) {
-      // A tile: choose the order that makes consecutive threads touch consecutive memory
-      int kk, mm;
-      if (sam == 1) { mm = i & 63; kk = i >> 6; } else { kk = i & 15; mm = i >> 4; }
-      const int m = m0 + mm, k = k0 + kk;
-      As[kk][mm] = (m < M && k < K) ? static_cast<ACC>(to_f_any(A[m * sam + k * sak])) : ACC(0);
-      int kb, nn;
-      if (sbn == 1) { nn = i & 63; kb = i >> 6; } else { kb = i & 15; nn = i >> 4; }
-      const int n = n0 + nn, k2 = k0 + kb;
-      Bs[kb][nn] = (n < N && k2 < K) ? static_cast<ACC>(to_f_any(B[k2 * sbk + n * sbn])) : ACC(0);
+  if (kb < ke) load(kb);
+  for (int k0 = kb; k0 < ke; k0 += 16) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      int kk, mm, k2, nn;
+      a_idx(q, kk, mm);
+      b_idx(q, k2, nn);
+      As[kk][mm] = ra[q];
+      Bs[k2][nn] = rb[q];
     }
     __syncthreads();
+    if (k0 + 16 < ke) load(k0 + 16);
 #pragma unroll
     for (int kk = 0; kk < 16; ++kk) {
       ACC a[4], b[4];
@@ -67,10 +97,30 @@ __global__ void __launch_bounds__(256) gemm_simt_kernel(const TA* __restrict__ A
     for (int j = 0; j < 4; ++j) {
       const int n = n0 + tx + 16 * j;
       if (n >= N) continue;
-      TC* c = C + static_cast<int64_t>(m) * ldc + n;
-      const double prev = beta != 0.0 ? static_cast<double>(to_f_any(*c)) : 0.0;
-      store_any(c, alpha * static_cast<double>(acc[i][j]) + beta * prev);
+      if (part) {
+        part[(static_cast<int64_t>(blockIdx.z) * M + m) * N + n] = static_cast<ACC>(alpha * static_cast<double>(acc[i][j]));
+      } else {
+        TC* c = C + static_cast<int64_t>(m) * ldc + n;
+        const double prev = beta != 0.0 ? static_cast<double>(to_f_any(*c)) : 0.0;
+        store_any(c, alpha * static_cast<double>(acc[i][j]) + beta * prev);
+      }
     }
+  }
+}
+
+template <typename TC, typename ACC>
+__global__ void gemm_reduce_kernel(const ACC* __restrict__ part, int splits, TC* __restrict__ C, int64_t ldc, int M,
+                                   int N, double beta, int lower) {
+  const int64_t total = static_cast<int64_t>(M) * N;
+  for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < total;
+       e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int m = static_cast<int>(e / N), n = static_cast<int>(e % N);
+    if (lower && (n >> 6) > (m >> 6)) continue;
+    double v = 0.0;
+    for (int z = 0; z < splits; ++z) v += static_cast<double>(part[z * total + e]);
+    TC* c = C + static_cast<int64_t>(m) * ldc + n;
+    if (beta != 0.0) v += beta * static_cast<double>(to_f_any(*c));
+    store_any(c, v);
   }
 }
 
@@ -78,7 +128,34 @@ template <typename TA, typename TB, typename TC, typename ACC>
 void gemm_simt(const TA* A, int64_t sam, int64_t sak, const TB* B, int64_t sbk, int64_t sbn, TC* C, int64_t ldc,
                int M, int N, int K, double alpha, double beta, cudaStream_t st) {
   dim3 grid((N + 63) / 64, (M + 63) / 64);
-  gemm_simt_kernel<TA, TB, TC, ACC><<<grid, 256, 0, st>>>(A, sam, sak, B, sbk, sbn, C, ldc, M, N, K, alpha, beta);
+  gemm_simt_kernel<TA, TB, TC, ACC><<<grid, 256, 0, st>>>(A, sam, sak, B, sbk, sbn, C, ldc, M, N, K, alpha, beta,
+                                                          nullptr, K, 0);
+}
+
+int gemm_splits(int M, int N, int K) {
+  const int tiles = ((M + 63) / 64) * ((N + 63) / 64);
+  int s = (2 * 148 + tiles - 1) / tiles;
+  s = std::min(s, kGemmMaxSplits);
+  s = std::min(s, std::max(1, K / 256));
+  return std::max(s, 1);
+}
+
+template <typename TA, typename TB, typename TC, typename ACC>
+void gemm_simt_split(const TA* A, int64_t sam, int64_t sak, const TB* B, int64_t sbk, int64_t sbn, TC* C,
+                     int64_t ldc, int M, int N, int K, double alpha, double beta, ACC* part, bool lower,
+                     cudaStream_t st) {
+  const int splits = gemm_splits(M, N, K);
+  if (splits <= 1 || part == nullptr) {
+    dim3 grid((N + 63) / 64, (M + 63) / 64);
+    gemm_simt_kernel<TA, TB, TC, ACC><<<grid, 256, 0, st>>>(A, sam, sak, B, sbk, sbn, C, ldc, M, N, K, alpha, beta,
+                                                            nullptr, K, lower ? 1 : 0);
+    return;
+  }
+  const int kchunk = ((K + splits - 1) / splits + 15) / 16 * 16;
+  dim3 grid((N + 63) / 64, (M + 63) / 64, splits);
+  gemm_simt_kernel<TA, TB, TC, ACC><<<grid, 256, 0, st>>>(A, sam, sak, B, sbk, sbn, C, ldc, M, N, K, alpha, 0.0,
+                                                          part, kchunk, lower ? 1 : 0);
+  gemm_reduce_kernel<TC, ACC><<<256, 256, 0, st>>>(part, splits, C, ldc, M, N, beta, lower ? 1 : 0);
 }
 
 #define XKV_GEMM_INST(TA, TB, TC, ACC)                                                                        \
@@ -93,28 +170,37 @@ XKV_GEMM_INST(float, float, double, double)
 XKV_GEMM_INST(float, double, double, double)
 XKV_GEMM_INST(double, double, double, double)
 #undef XKV_GEMM_INST
+template void gemm_simt_split<float, float, double, double>(const float*, int64_t, int64_t, const float*, int64_t,
+                                                            int64_t, double*, int64_t, int, int, int, double,
+                                                            double, double*, bool, cudaStream_t);
 
 // ---------------------------------------------------- Cholesky QR pieces
 // Lower Cholesky factor of (W + shift I), b x b fp64 row-major, in place (only
 // the lower triangle is meaningful afterwards), right-looking and blocked by
 // kCholNB: per block column k
 //   1. chol_diag_kernel  factors the diagonal block in shared memory (one CTA)
-//      and writes its inverse to a scratch block;
+//      and writes its inverse to dblk[k];
 //   2. chol_panel_kernel  L_ik = W_ik L_kk^{-T} for the rows below (64 rows a CTA);
 //   3. the trailing update W_ij -= L_ik L_jk^T as an fp64 GEMM over the whole
 //      trailing square (the upper part of W is scratch).
 // shift = shift_rel * trace(W) when a device trace is given; it is added to
 // each diagonal element when its block is factored.  A non-positive pivot is
-// recorded as a numerical fault and replaced by a tiny positive one so that
-// results stay finite.
+// recorded as a numerical fault and replaced by a unit pivot over a zero
+// column, so that results stay finite.
 constexpr int kCholNB = 64;
 
+// The diagonal block is eliminated in the unscaled (L D L^T) form, one barrier
+// per column: a_il -= a_ij a_lj / d_j for j < l <= i; afterwards
+// L_ij = a_ij / sqrt(d_j) and L_jj = sqrt(d_j).  Its inverse X = L^{-1} is then
+// formed row by row, X_ic = (delta_ic - sum_{c <= k < i} L_ik X_kc) / L_ii, with
+// four threads sharing each column's sum.
 __global__ void __launch_bounds__(256) chol_diag_kernel(double* __restrict__ W, int b, int k0, double shift_rel,
                                                         const double* __restrict__ trace, int* status,
                                                         double* __restrict__ dinv) {
   extern __shared__ double chol_sm[];
   double(*a)[kCholNB + 1] = reinterpret_cast<double(*)[kCholNB + 1]>(chol_sm);
   double(*x)[kCholNB + 1] = reinterpret_cast<double(*)[kCholNB + 1]>(chol_sm + kCholNB * (kCholNB + 1));
+  __shared__ double dg[kCholNB];
   const int tid = threadIdx.x;
   const int nb = min(kCholNB, b - k0);
   const double shift = trace ? shift_rel * (*trace) : 0.0;
@@ -125,36 +211,51 @@ __global__ void __launch_bounds__(256) chol_diag_kernel(double* __restrict__ W, 
     a[i][j] = v;
   }
   __syncthreads();
+  // thread (ty, tx) of a 16 x 16 grid owns rows ty + 16 u and columns tx + 16 v
+  const int ty = tid >> 4, tx = tid & 15;
   for (int j = 0; j < nb; ++j) {
+    const double d = a[j][j];
+    const bool bad = !(d > 0.0) || !isfinite(d);
     if (tid == 0) {
-      double d = a[j][j];
-      if (!(d > 0.0) || !isfinite(d)) {
-        record_status(status, kDevNumerical);
-        d = 1e-300;
-      }
-      a[j][j] = sqrt(d);
+      dg[j] = bad ? 0.0 : d;
+      if (bad) record_status(status, kDevNumerical);
     }
-    __syncthreads();
-    const double piv = a[j][j];
-    for (int i = j + 1 + tid; i < nb; i += blockDim.x) a[i][j] /= piv;
-    __syncthreads();
-    // trailing update of the block: pairs (i, l), j < l <= i < nb
-    const int m = nb - j - 1;
-    for (int e = tid; e < m * m; e += blockDim.x) {
-      const int i = j + 1 + e / m, l = j + 1 + e % m;
-      if (l <= i) a[i][l] -= a[i][j] * a[l][j];
+    if (!bad) {
+      const double inv = 1.0 / d;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int i = ty + 16 * u;
+        if (i <= j || i >= nb) continue;
+        const double aij = a[i][j] * inv;
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          const int l = tx + 16 * v;
+          if (l > j && l <= i) a[i][l] -= aij * a[l][j];
+        }
+      }
     }
     __syncthreads();
   }
-  // inverse of the factor: column c of X = L^{-1} by forward substitution
-  for (int c = tid; c < nb; c += blockDim.x) {
-    for (int i = 0; i < nb; ++i) {
-      double s = i == c ? 1.0 : 0.0;
-      for (int k = c; k < i; ++k) s -= a[i][k] * x[k][c];
-      x[i][c] = i < c ? 0.0 : s / a[i][i];
-    }
+  for (int e = tid; e < nb * nb; e += blockDim.x) {
+    const int i = e / nb, j = e % nb;
+    if (j > i) continue;
+    const double d = dg[j];
+    if (j == i) a[i][i] = d > 0.0 ? sqrt(d) : 1.0;
+    else a[i][j] = d > 0.0 ? a[i][j] / sqrt(d) : 0.0;
   }
   __syncthreads();
+  {
+    const int c = tid >> 2, q = tid & 3;  // column c, quarter q of its sums
+    for (int i = 0; i < nb; ++i) {
+      double sm = 0.0;
+      if (c < i)
+        for (int k = c + q; k < i; k += 4) sm += a[i][k] * x[k][c];
+      sm += __shfl_xor_sync(0xffffffffu, sm, 1);
+      sm += __shfl_xor_sync(0xffffffffu, sm, 2);
+      if (q == 0 && c < nb) x[i][c] = c > i ? 0.0 : ((c == i ? 1.0 : 0.0) - sm) / a[i][i];
+      __syncthreads();
+    }
+  }
   for (int e = tid; e < nb * nb; e += blockDim.x) {
     const int i = e / nb, j = e % nb;
     if (j <= i) W[static_cast<int64_t>(k0 + i) * b + k0 + j] = a[i][j];
@@ -178,20 +279,44 @@ __global__ void __launch_bounds__(256) chol_panel_kernel(double* __restrict__ W,
   }
   for (int e = tid; e < nb * nb; e += blockDim.x) x[e / nb][e % nb] = dinv[(e / nb) * kCholNB + e % nb];
   __syncthreads();
-  for (int e = tid; e < rows * nb; e += blockDim.x) {
-    const int i = e / nb, j = e % nb;
-    double s = 0.0;
-    for (int k = 0; k <= j; ++k) s += w[i][k] * x[j][k];
-    W[static_cast<int64_t>(r0 + i) * b + k0 + j] = s;
+  // thread (ty, tx): rows ty + 16 u, columns tx + 16 v of the panel block
+  const int ty = tid >> 4, tx = tid & 15;
+  double acc[4][4];
+#pragma unroll
+  for (int u = 0; u < 4; ++u)
+#pragma unroll
+    for (int v = 0; v < 4; ++v) acc[u][v] = 0.0;
+  for (int k = 0; k < nb; ++k) {
+    double wv[4], xv[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) wv[u] = w[ty + 16 * u][k];
+#pragma unroll
+    for (int v = 0; v < 4; ++v) xv[v] = x[tx + 16 * v][k];  // zero above the diagonal (k > column)
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+#pragma unroll
+      for (int v = 0; v < 4; ++v) acc[u][v] += wv[u] * xv[v];
+  }
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const int i = ty + 16 * u;
+    if (i >= rows) continue;
+#pragma unroll
+    for (int v = 0; v < 4; ++v) {
+      const int j = tx + 16 * v;
+      if (j < nb) W[static_cast<int64_t>(r0 + i) * b + k0 + j] = acc[u][v];
+    }
   }
 }
 
-void cholesky_blocked(double* W, int b, double shift_rel, const double* trace, int* status, double* dinv,
+// dblk: one 64 x 64 block per block column (the inverse of its diagonal block)
+void cholesky_blocked(double* W, int b, double shift_rel, const double* trace, int* status, double* dblk,
                       cudaStream_t st) {
   const int smem = 2 * 64 * (kCholNB + 1) * 8;
   cudaFuncSetAttribute(chol_diag_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   cudaFuncSetAttribute(chol_panel_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   for (int k0 = 0; k0 < b; k0 += kCholNB) {
+    double* dinv = dblk + static_cast<int64_t>(k0 / kCholNB) * kCholNB * kCholNB;
     chol_diag_kernel<<<1, 256, smem, st>>>(W, b, k0, shift_rel, trace, status, dinv);
     const int nb = std::min(kCholNB, b - k0);
     const int rem = b - k0 - nb;
@@ -203,26 +328,92 @@ void cholesky_blocked(double* W, int b, double shift_rel, const double* trace, i
   }
 }
 
-// X = L^{-1} for a lower-triangular L (row-major b x b), one warp per column.
-__global__ void __launch_bounds__(256) tri_inverse_kernel(const double* __restrict__ L, double* __restrict__ X,
-                                                          int b) {
-  extern __shared__ double xs[];  // [8 warps][b]
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int j = blockIdx.x * 8 + warp;
-  if (j >= b) return;
-  double* x = xs + static_cast<int64_t>(warp) * b;
-  for (int i = lane; i < b; i += 32) x[i] = 0.0;
-  __syncwarp();
-  for (int i = j; i < b; ++i) {
-    const double* li = L + static_cast<int64_t>(i) * b;
-    double s = 0.0;
-    for (int k = j + lane; k < i; k += 32) s += li[k] * x[k];
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-    if (lane == 0) x[i] = ((i == j ? 1.0 : 0.0) - s) / li[i];
-    __syncwarp();
+// X = L^{-1} for the lower factor L (row-major b x b, the Cholesky above),
+// blocked by 64: X_JJ = dblk[J], and for I > J
+//   X_IJ = -dblk[I] (sum_{J <= K < I} L_IK X_KJ).
+// One CTA per block column J walks I downwards (each X_IJ needs the X_KJ above
+// it, written by the same CTA); the strict upper part of X is set to zero.
+__global__ void __launch_bounds__(256) tri_inverse_kernel(const double* __restrict__ L,
+                                                          const double* __restrict__ dblk, double* X, int b) {
+  extern __shared__ double tsm[];
+  double(*P)[kCholNB + 1] = reinterpret_cast<double(*)[kCholNB + 1]>(tsm);
+  double(*Q)[kCholNB + 1] = reinterpret_cast<double(*)[kCholNB + 1]>(tsm + kCholNB * (kCholNB + 1));
+  const int J = blockIdx.x, nblk = (b + kCholNB - 1) / kCholNB;
+  const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
+  const int j0 = J * kCholNB, nj = min(kCholNB, b - j0);
+  for (int e = tid; e < j0 * nj; e += 256) X[static_cast<int64_t>(e / nj) * b + j0 + e % nj] = 0.0;
+  for (int e = tid; e < nj * nj; e += 256) {
+    const int i = e / nj, c = e % nj;
+    X[static_cast<int64_t>(j0 + i) * b + j0 + c] = dblk[static_cast<int64_t>(J) * kCholNB * kCholNB + i * kCholNB + c];
   }
-  for (int i = lane; i < b; i += 32) X[static_cast<int64_t>(i) * b + j] = i >= j ? x[i] : 0.0;
+  __syncthreads();
+  for (int I = J + 1; I < nblk; ++I) {
+    const int i0 = I * kCholNB, ni = min(kCholNB, b - i0);
+    double acc[4][4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) acc[i][j] = 0.0;
+    for (int K = J; K < I; ++K) {  // K < I <= nblk - 1: a full block
+      const int kb0 = K * kCholNB;
+      for (int e = tid; e < kCholNB * kCholNB; e += 256) {
+        const int r = e >> 6, c = e & 63;
+        P[r][c] = r < ni ? L[static_cast<int64_t>(i0 + r) * b + kb0 + c] : 0.0;
+        Q[r][c] = c < nj ? __ldcg(X + static_cast<int64_t>(kb0 + r) * b + j0 + c) : 0.0;
+      }
+      __syncthreads();
+#pragma unroll 8
+      for (int kk = 0; kk < kCholNB; ++kk) {
+        double av[4], bv[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) av[i] = P[ty + 16 * i][kk];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) bv[j] = Q[kk][tx + 16 * j];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) acc[i][j] += av[i] * bv[j];
+      }
+      __syncthreads();
+    }
+    // X_IJ = -dblk[I] S
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) Q[ty + 16 * i][tx + 16 * j] = acc[i][j];
+    for (int e = tid; e < kCholNB * kCholNB; e += 256) {
+      const int r = e >> 6, c = e & 63;  // a partial last block holds ni x ni entries
+      P[r][c] = r < ni && c < ni ? dblk[static_cast<int64_t>(I) * kCholNB * kCholNB + e] : 0.0;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) acc[i][j] = 0.0;
+#pragma unroll 8
+    for (int kk = 0; kk < kCholNB; ++kk) {
+      double av[4], bv[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) av[i] = P[ty + 16 * i][kk];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) bv[j] = Q[kk][tx + 16 * j];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] += av[i] * bv[j];
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int r = ty + 16 * i;
+      if (r >= ni) continue;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int c = tx + 16 * j;
+        if (c < nj) X[static_cast<int64_t>(i0 + r) * b + j0 + c] = -acc[i][j];
+      }
+    }
+    __syncthreads();
+  }
 }
 
 __global__ void trace_kernel(const double* __restrict__ W, int b, double* __restrict__ out) {
@@ -240,20 +431,28 @@ __global__ void trace_kernel(const double* __restrict__ W, int b, double* __rest
   }
 }
 
-// One pass of (shifted) Cholesky QR: W = Y^T Y (fp64), L = chol(W + shift I),
-// Q = Y L^{-T}.  Y, Q: n x b fp32 row-major (distinct buffers).  W, Linv: b x b
-// fp64 scratch; scal: one fp64 scratch scalar.
-void cholqr_pass(const float* Y, float* Q, int n, int b, double shift_rel, double* W, double* Linv, double* scal,
-                 int* status, cudaStream_t st) {
-  gemm_simt<float, float, double, double>(Y, 1, b, Y, b, 1, W, b, b, b, n, 1.0, 0.0, st);
-  if (shift_rel > 0.0) trace_kernel<<<1, 256, 0, st>>>(W, b, scal);
-  // Linv is free until the inverse below: its first block holds the diagonal inverses
-  cholesky_blocked(W, b, shift_rel, shift_rel > 0.0 ? scal : nullptr, status, Linv, st);
-  const size_t smem2 = static_cast<size_t>(8) * b * 8;
-  cudaFuncSetAttribute(tri_inverse_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem2));
-  tri_inverse_kernel<<<(b + 7) / 8, 256, smem2, st>>>(W, Linv, b);
+size_t cholqr_dblk_bytes(int b) {
+  return align_up(static_cast<size_t>((b + kCholNB - 1) / kCholNB) * kCholNB * kCholNB * 8);
+}
+
+size_t cholqr_part_bytes(int n, int b) {
+  const int s = gemm_splits(b, b, n);
+  return s > 1 ? align_up(static_cast<size_t>(s) * b * b * 8) : 0;
+}
+
+// One pass of (shifted) Cholesky QR: W = Y^T Y (fp64, lower tiles, split K),
+// L = chol(W + shift I), Q = Y L^{-T}.  Y, Q: n x b fp32 row-major (distinct
+// buffers).
+void cholqr_pass(const float* Y, float* Q, int n, int b, double shift_rel, const CholQRScratch& s, int* status,
+                 cudaStream_t st) {
+  gemm_simt_split<float, float, double, double>(Y, 1, b, Y, b, 1, s.W, b, b, b, n, 1.0, 0.0, s.part, true, st);
+  if (shift_rel > 0.0) trace_kernel<<<1, 256, 0, st>>>(s.W, b, s.scal);
+  cholesky_blocked(s.W, b, shift_rel, shift_rel > 0.0 ? s.scal : nullptr, status, s.dblk, st);
+  const int smem2 = 2 * kCholNB * (kCholNB + 1) * 8;
+  cudaFuncSetAttribute(tri_inverse_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem2);
+  tri_inverse_kernel<<<(b + kCholNB - 1) / kCholNB, 256, smem2, st>>>(s.W, s.dblk, s.Linv, b);
   // Q(m, j) = sum_k Y(m, k) Linv(j, k)
-  gemm_simt<float, double, float, double>(Y, b, 1, Linv, 1, b, Q, b, n, b, b, 1.0, 0.0, st);
+  gemm_simt<float, double, float, double>(Y, b, 1, s.Linv, 1, b, Q, b, n, b, b, 1.0, 0.0, st);
 }
 
 // ------------------------------------------------------ one-sided Jacobi
@@ -262,15 +461,20 @@ void cholqr_pass(const float* Y, float* Q, int n, int b, double shift_rel, doubl
 // 16; every round pairs the blocks by the round-robin schedule and each CTA
 // orthogonalises the 32 columns of its pair: Gram G = Wc^T Wc, eigenvectors R
 // of G by cyclic Jacobi, Wc <- Wc R, Vc <- Vc R.  A sweep is nblk - 1 rounds;
-// a sweep that rotates nothing ends the iteration (later launches return at
-// once).  On convergence column i of W is lambda_i v_i, so |lambda_i| is its
-// norm and v_i is column i of V.
+// a sweep that rotates nothing ends the iteration.  On convergence column i of
+// W is lambda_i v_i, so |lambda_i| is its norm and v_i is column i of V.
 constexpr int kJB = 16;
 constexpr int kJacobiInnerSweeps = 2;
 
+// Sweep limit: 40, or XKV_JACOBI_MAX_SWEEPS (a diagnostic override, e.g. 1 to
+// see the non-convergence report), at most kJacobiSweepCap.
+constexpr int kJacobiSweepCap = 64;
+
 struct JacobiState {
-  int active;      // rotations performed in the current sweep
   int converged;
+  int pad;
+  int active[kJacobiSweepCap];  // pairs rotated in each sweep
+  GroupBarrier bar;             // the problem's CTAs (cooperative launch)
 };
 
 __device__ __forceinline__ int rr_player(int pos, int round, int nplayers) {
@@ -278,17 +482,18 @@ __device__ __forceinline__ int rr_player(int pos, int round, int nplayers) {
   return ((pos - 1 + round) % (nplayers - 1)) + 1;
 }
 
-__global__ void __launch_bounds__(256) jacobi_round_kernel(double* __restrict__ W, double* __restrict__ V, int n,
-                                                           int nblk, int round, JacobiState* __restrict__ state,
-                                                           double tol) {
+// One round for the pair of CTA blockIdx.x of problem blockIdx.y; rotations
+// are counted in state->active[sweep].  W and V are read through L2 (__ldcg):
+// in the persistent kernel other CTAs rewrote them since this SM last read.
+__device__ void jacobi_pair(double* __restrict__ W, double* __restrict__ V, int n, int nblk, int round, int sweep,
+                            JacobiState* __restrict__ state, double tol) {
   __shared__ double G[32][33];
   __shared__ double R[32][33];
-  __shared__ double tile[32][33];
+  __shared__ double tile[64][33];
   __shared__ double cs[16], sn[16];
   __shared__ int pp[16], qq[16];
   const int prob = blockIdx.y;
   JacobiState* stp = state + prob;
-  if (stp->converged) return;
   double* Wp = W + static_cast<int64_t>(prob) * n * n;
   double* Vp = V ? V + static_cast<int64_t>(prob) * n * n : nullptr;
   const int pair = blockIdx.x;
@@ -306,15 +511,17 @@ __global__ void __launch_bounds__(256) jacobi_round_kernel(double* __restrict__ 
   {
     const int a = tid >> 3, bb = (tid & 7) * 4;  // thread owns G[a][bb..bb+3]
     double acc[4] = {0, 0, 0, 0};
-    for (int r0 = 0; r0 < n; r0 += 32) {
-      for (int i = tid; i < 32 * 32; i += 256) {
-        const int c = i / 32, r = i % 32;
+    for (int r0 = 0; r0 < n; r0 += 64) {  // 64 rows a pass: 8 loads in flight per thread
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        const int i = tid + 256 * q;
+        const int c = i >> 6, r = i & 63;
         const int cc = cols[c];
-        tile[r][c] = (cc >= 0 && r0 + r < n) ? Wp[static_cast<int64_t>(cc) * n + r0 + r] : 0.0;
+        tile[r][c] = (cc >= 0 && r0 + r < n) ? __ldcg(Wp + static_cast<int64_t>(cc) * n + r0 + r) : 0.0;
       }
       __syncthreads();
 #pragma unroll 4
-      for (int r = 0; r < 32; ++r) {
+      for (int r = 0; r < 64; ++r) {
         const double x = tile[r][a];
 #pragma unroll
         for (int e = 0; e < 4; ++e) acc[e] += x * tile[r][bb + e];
@@ -352,11 +559,17 @@ __global__ void __launch_bounds__(256) jacobi_round_kernel(double* __restrict__ 
         pp[tid] = p;
         qq[tid] = q;
         const double gpq = G[p][q], gpp = G[p][p], gqq = G[q][q];
-        if (fabs(gpq) > 1e-14 * sqrt(fabs(gpp * gqq)) && gpq != 0.0) {
-          const double tau = (gqq - gpp) / (2.0 * gpq);
-          const double t = (tau >= 0.0 ? 1.0 : -1.0) / (fabs(tau) + sqrt(1.0 + tau * tau));
-          cs[tid] = 1.0 / sqrt(1.0 + t * t);
-          sn[tid] = t * cs[tid];
+        if (gpq * gpq > 1e-28 * fabs(gpp * gqq) && gpq != 0.0) {
+          // t = tan(theta) of the rotation that zeroes gpq, from the difference
+          // d = gqq - gpp without forming tau = d / (2 gpq):
+          //   t = sign(d) 2 gpq / (|d| + sqrt(d^2 + 4 gpq^2)),
+          // then c = (1 + t^2)^(-1/2), s = t c (one division, one square
+          // root, one reciprocal square root, all fp64)
+          const double d = gqq - gpp;
+          const double t = (d >= 0.0 ? 2.0 : -2.0) * gpq / (fabs(d) + sqrt(fma(d, d, 4.0 * gpq * gpq)));
+          const double c = rsqrt(fma(t, t, 1.0));
+          cs[tid] = c;
+          sn[tid] = t * c;
           s_any = 1;
         } else {
           cs[tid] = 1.0;
@@ -393,7 +606,7 @@ __global__ void __launch_bounds__(256) jacobi_round_kernel(double* __restrict__ 
     __syncthreads();
     if (!any) break;
   }
-  if (tid == 0) atomicAdd(&stp->active, 1);
+  if (tid == 0) atomicAdd(&stp->active[sweep], 1);
   // Wc <- Wc R, Vc <- Vc R (row by row)
   for (int mat = 0; mat < (Vp ? 2 : 1); ++mat) {
     double* M = mat == 0 ? Wp : Vp;
@@ -401,7 +614,7 @@ __global__ void __launch_bounds__(256) jacobi_round_kernel(double* __restrict__ 
       const int r = r0 + tid;
       double x[32];
 #pragma unroll
-      for (int c = 0; c < 32; ++c) x[c] = (cols[c] >= 0 && r < n) ? M[static_cast<int64_t>(cols[c]) * n + r] : 0.0;
+      for (int c = 0; c < 32; ++c) x[c] = (cols[c] >= 0 && r < n) ? __ldcg(M + static_cast<int64_t>(cols[c]) * n + r) : 0.0;
       if (r < n) {
         for (int c = 0; c < 32; ++c) {
           if (cols[c] < 0) continue;
@@ -415,11 +628,41 @@ __global__ void __launch_bounds__(256) jacobi_round_kernel(double* __restrict__ 
   }
 }
 
-__global__ void jacobi_sweep_end_kernel(JacobiState* state, int count) {
+// Per-round launches (used when the pairs of all problems cannot be resident
+// at once): a problem marked converged returns at once.
+__global__ void __launch_bounds__(256) jacobi_round_kernel(double* __restrict__ W, double* __restrict__ V, int n,
+                                                           int nblk, int round, int sweep,
+                                                           JacobiState* __restrict__ state, double tol) {
+  if (state[blockIdx.y].converged) return;
+  jacobi_pair(W, V, n, nblk, round, sweep, state, tol);
+}
+
+__global__ void jacobi_sweep_end_kernel(JacobiState* state, int count, int sweep) {
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= count) return;
-  if (!state[i].converged && state[i].active == 0) state[i].converged = 1;
-  state[i].active = 0;
+  if (!state[i].converged && state[i].active[sweep] == 0) state[i].converged = 1;
+}
+
+// Every sweep in one cooperative launch: the CTAs of a problem (one per pair)
+// meet at the problem's bounded barrier after each round; after the last round
+// of a sweep all of them read the sweep's rotation count, and a problem that
+// rotated nothing is converged.  A barrier that gives up (recorded as a device
+// timeout) ends the problem unconverged.
+__global__ void __launch_bounds__(256) jacobi_sweeps_kernel(double* __restrict__ W, double* __restrict__ V, int n,
+                                                            int nblk, int max_sweeps, JacobiState* __restrict__ state,
+                                                            double tol, int* status) {
+  JacobiState* stp = state + blockIdx.y;
+  const unsigned npairs = gridDim.x;
+  for (int sweep = 0; sweep < max_sweeps; ++sweep) {
+    for (int round = 0; round < nblk - 1; ++round) {
+      jacobi_pair(W, V, n, nblk, round, sweep, state, tol);
+      if (!group_barrier(&stp->bar, npairs, status)) return;
+    }
+    if (*reinterpret_cast<volatile int*>(&stp->active[sweep]) == 0) {
+      if (blockIdx.x == 0 && threadIdx.x == 0) stp->converged = 1;
+      return;
+    }
+  }
 }
 
 __global__ void jacobi_init_kernel(double* V, int n, int count, JacobiState* state) {
@@ -430,7 +673,7 @@ __global__ void jacobi_init_kernel(double* V, int n, int count, JacobiState* sta
       const int64_t w = i % (static_cast<int64_t>(n) * n);
       V[i] = (w / n == w % n) ? 1.0 : 0.0;
     }
-    if (i < count) { state[i].active = 0; state[i].converged = 0; }
+    if (i < count) state[i] = JacobiState{};
   }
 }
 
@@ -457,14 +700,12 @@ __global__ void jacobi_check_kernel(const JacobiState* state, int count, int* st
 
 size_t jacobi_workspace(int, int count) { return align_up(static_cast<size_t>(count) * sizeof(JacobiState)); }
 
-// Sweep limit: 40, or XKV_JACOBI_MAX_SWEEPS (a diagnostic override, e.g. 1 to
-// see the non-convergence report).
 static int jacobi_max_sweeps() {
   static int v = 0;
   if (v == 0) {
     const char* e = getenv("XKV_JACOBI_MAX_SWEEPS");
     const int x = e ? atoi(e) : 0;
-    v = x > 0 ? x : 40;
+    v = std::min(x > 0 ? x : 40, kJacobiSweepCap);
   }
   return v;
 }
@@ -477,11 +718,23 @@ xkv_status jacobi_launch(double* W, double* V, double* lam, int n, int count, vo
   if (nblk & 1) ++nblk;
   if (nblk < 2) nblk = 2;
   jacobi_init_kernel<<<256, 256, 0, st>>>(V, n, count, state);
-  const int max_sweeps = jacobi_max_sweeps();
-  for (int s = 0; s < max_sweeps; ++s) {
-    for (int r = 0; r < nblk - 1; ++r)
-      jacobi_round_kernel<<<dim3(nblk / 2, count), 256, 0, st>>>(W, V, n, nblk, r, state, 1e-11);
-    jacobi_sweep_end_kernel<<<(count + 127) / 128, 128, 0, st>>>(state, count);
+  int max_sweeps = jacobi_max_sweeps();
+  double tol = 1e-11;
+  // one cooperative launch when every pair of every problem can be resident
+  int per_sm = 0;
+  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, jacobi_sweeps_kernel, 256, 0);
+  const int64_t ctas = static_cast<int64_t>(nblk / 2) * count;
+  if (per_sm > 0 && ctas <= static_cast<int64_t>(per_sm) * num_sms() && count <= 65535) {
+    void* args[] = {&W, &V, &n, &nblk, &max_sweeps, &state, &tol, &status};
+    if (cudaLaunchCooperativeKernel(reinterpret_cast<void*>(jacobi_sweeps_kernel), dim3(nblk / 2, count), dim3(256),
+                                    args, 0, st) != cudaSuccess)
+      return XKV_ERR_CUDA;
+  } else {
+    for (int s = 0; s < max_sweeps; ++s) {
+      for (int r = 0; r < nblk - 1; ++r)
+        jacobi_round_kernel<<<dim3(nblk / 2, count), 256, 0, st>>>(W, V, n, nblk, r, s, state, tol);
+      jacobi_sweep_end_kernel<<<(count + 127) / 128, 128, 0, st>>>(state, count, s);
+    }
   }
   jacobi_check_kernel<<<(count + 127) / 128, 128, 0, st>>>(state, count, status);
   column_norms_kernel<<<dim3((n + 7) / 8, count), 256, 0, st>>>(W, lam, n, count);

@@ -23,49 +23,6 @@ namespace {
 
 constexpr int kTriThreads = 256;
 
-struct GroupBarrier {
-  unsigned count;
-  unsigned gen;
-  int abort;
-  int pad;
-};
-
-// Barrier of the `nblocks` CTAs of one problem.  Each CTA's writes are
-// released before it arrives; a wait longer than kWaitLimitNs records
-// kDevTimeout, sets the problem's abort flag and lets the CTA wind down.
-__device__ bool group_barrier(GroupBarrier* g, unsigned nblocks, int* status) {
-  __shared__ int s_ok;
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    bool ok = true;
-    volatile unsigned* genp = &g->gen;
-    volatile int* abortp = &g->abort;
-    const unsigned gen = *genp;
-    __threadfence();
-    if (atomicAdd(&g->count, 1u) == nblocks - 1) {
-      atomicExch(&g->count, 0u);
-      __threadfence();
-      atomicAdd(&g->gen, 1u);
-    } else {
-      const uint64_t t0 = globaltimer_ns();
-      while (*genp == gen) {
-        if (*abortp) { ok = false; break; }
-        if (globaltimer_ns() - t0 > kWaitLimitNs) {
-          record_status(status, kDevTimeout);
-          atomicExch(&g->abort, 1);
-          ok = false;
-          break;
-        }
-        __nanosleep(64);
-      }
-    }
-    __threadfence();
-    s_ok = ok;
-  }
-  __syncthreads();
-  return s_ok != 0;
-}
-
 __device__ double block_sum(double v, double* red) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 #pragma unroll

@@ -78,7 +78,8 @@ xkv_status gram_launch(const void* const* X, int G, int64_t rows, int d, int64_t
                        void* ws, cudaStream_t st);
 struct FactorPlan {
   int n, b, rank;
-  size_t off_Q, off_Y, off_W, off_H, off_U, off_lam, off_ord, off_Ur, off_Vr, off_jac, bytes;
+  size_t off_Q, off_Y, off_W, off_H, off_U, off_lam, off_ord, off_Ur, off_Vr, off_jac, off_dblk, off_part, off_chl,
+      off_qhl, bytes;
 };
 xkv_status factor_plan(int n, int64_t rows, int rank, int oversample, FactorPlan* plan);
 xkv_status factor_launch(const FactorPlan& plan, const float* C, xkv_dtype dt, int iters, uint64_t seed, void* Bt,
