@@ -8,7 +8,8 @@
 //      128 x 128), 256-row chunks accumulated in TMEM and summed in fp32
 //      registers, and a mirrored fp32 epilogue.
 //   2. top-r subspace: block subspace iteration Y = C Q, Q = qr(Y) (shifted
-//      Cholesky QR, two passes, fp64 small factors with a blocked Cholesky),
+//      Cholesky QR, fp64 small factors with a blocked Cholesky; one pass per
+//      iteration, two for the basis that enters Rayleigh-Ritz),
 //      started from a Gaussian block (Philox4x32-10 + Box-Muller on the
 //      device); Rayleigh-Ritz: H = Q^T C Q, eigenpairs of H by one-sided block
 //      Jacobi, V_r = Q U[:, top r].
@@ -30,23 +31,41 @@ struct LayerPtrs {
   const void* p[8];
 };
 
+// One 64 (rows t) x 64 (columns c) tile per CTA, moved in 16-byte vectors
+// both ways: row t's 8-column vectors land in shared memory at granule
+// (c / 8) ^ (t / 8 mod 8), so that the column reads of the store phase (8
+// values of t for one c) fall in different banks; each warp then writes 128
+// contiguous bytes of 4 rows of Xt.  Requires 16-byte aligned layers, ldx and
+// ldt multiples of 8.
 __global__ void __launch_bounds__(256) transpose_layers_kernel(const LayerPtrs X, int d, int64_t ldx, int64_t rows,
                                                                __nv_bfloat16* __restrict__ Xt, int64_t ldt) {
-  __shared__ __nv_bfloat16 tile[64][66];
+  __shared__ uint4 tile[64][8];
   const int l = blockIdx.z;
   const int64_t t0 = static_cast<int64_t>(blockIdx.x) * 64;
   const int c0 = blockIdx.y * 64;
+  const int tid = threadIdx.x;
   const __nv_bfloat16* src = static_cast<const __nv_bfloat16*>(X.p[l]);
-  for (int i = threadIdx.x; i < 64 * 64; i += 256) {
-    const int r = i / 64, c = i % 64;
+  for (int v = tid; v < 512; v += 256) {
+    const int r = v >> 3, cv = v & 7;
     const int64_t t = t0 + r;
-    tile[r][c] = t < rows ? src[t * ldx + c0 + c] : __float2bfloat16_rn(0.f);
+    const uint4 val = t < rows ? *reinterpret_cast<const uint4*>(src + t * ldx + c0 + 8 * cv) : make_uint4(0, 0, 0, 0);
+    tile[r][cv ^ ((r >> 3) & 7)] = val;
   }
   __syncthreads();
-  for (int i = threadIdx.x; i < 64 * 64; i += 256) {
-    const int c = i / 64, r = i % 64;
-    const int64_t t = t0 + r;
-    if (t < ldt) Xt[static_cast<int64_t>(l * d + c0 + c) * ldt + t] = tile[r][c];
+  const uint16_t* th = reinterpret_cast<const uint16_t*>(&tile[0][0]);
+  for (int v = tid; v < 512; v += 256) {
+    const int c = v >> 3, tv = v & 7;  // column c, rows 8 tv .. 8 tv + 7
+    const int g = (c >> 3) ^ tv;       // (8 tv + e) / 8 = tv
+    uint32_t w[4];
+#pragma unroll
+    for (int e = 0; e < 8; e += 2) {
+      const uint32_t lo = th[(8 * tv + e) * 64 + g * 8 + (c & 7)];
+      const uint32_t hi = th[(8 * tv + e + 1) * 64 + g * 8 + (c & 7)];
+      w[e / 2] = lo | (hi << 16);
+    }
+    const int64_t t = t0 + 8 * tv;
+    if (t < ldt)
+      *reinterpret_cast<uint4*>(Xt + static_cast<int64_t>(l * d + c0 + c) * ldt + t) = make_uint4(w[0], w[1], w[2], w[3]);
   }
 }
 
@@ -448,7 +467,10 @@ xkv_status gram_launch(const void* const* X, int G, int64_t rows, int d, int64_t
                        void* ws, cudaStream_t st) {
   const int n = G * d;
   if (rows <= 0) return XKV_OK;
-  if (gram_tc_ok(G, d, dt)) {
+  // the vectorised transpose reads 16-byte aligned layers and rows
+  bool vec_ok = ldx % 8 == 0 && d % 64 == 0;
+  for (int l = 0; l < G; ++l) vec_ok = vec_ok && (reinterpret_cast<uintptr_t>(X[l]) & 15) == 0;
+  if (gram_tc_ok(G, d, dt) && vec_ok) {
     const int64_t ldt = (rows + 7) / 8 * 8;
     __nv_bfloat16* Xt = static_cast<__nv_bfloat16*>(ws);
     LayerPtrs lp;
@@ -493,6 +515,154 @@ xkv_status gram_launch(const void* const* X, int G, int64_t rows, int d, int64_t
   return cudaPeekAtLastError() == cudaSuccess ? XKV_OK : XKV_ERR_CUDA;
 }
 
+// ------------------------------------------- subspace iteration on tcgen05
+// Y = C Q for the symmetric Gram C (n x n f32) and the block Q (n x b f32),
+// both split into bf16 hi/lo pairs (x = hi + lo keeps ~16 significant bits):
+// Y = Chi Qhi + Chi Qlo + Clo Qhi, the three products accumulated in fp32 in
+// TMEM (the dropped lo lo term and the split are of the order of the fp32
+// rounding of a 4096-term dot product).  Used for the iterations, which need
+// only the span of C Q.  C's pair is K-major (rows of C are
+// its columns: C is symmetric), Q's pair is MN-major (Q row-major).  One
+// 128 x bn output tile per CTA; warp 0 loads, warp 1 issues, warps 2-5 store.
+constexpr int kCqStages = 3;
+constexpr int kCqThreads = 192;
+
+inline size_t cq_smem(int bn) { return 1024 + kCqStages * (32768 + 2 * bn * 128) + (2 * kCqStages + 2) * 8 + 16; }
+
+__global__ void __launch_bounds__(kCqThreads, 1)
+    cq_tc_kernel(const __grid_constant__ CUtensorMap chi, const __grid_constant__ CUtensorMap clo,
+                 const __grid_constant__ CUtensorMap qhi, const __grid_constant__ CUtensorMap qlo, int n, int b,
+                 int bn, float* __restrict__ Y, int* status) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int SB = 32768 + 2 * bn * 128;  // A hi, A lo (128 x 64), B hi, B lo (64 x bn)
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kCqStages * SB);
+  uint64_t* empty = full + kCqStages;
+  uint64_t* accbar = empty + kCqStages;
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(accbar + 2);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int m0 = blockIdx.x * 128, n0 = blockIdx.y * bn;
+  const int nk = n / 64;
+  if (tid == 0) {
+    for (int i = 0; i < kCqStages; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
+    mbar_init(&accbar[0], 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) tmem_alloc(tslot, 128);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tslot;
+  if (warp == 0) {
+    if (lane == 0) {
+      for (int a = 0; a < nk; ++a) {
+        const int slot = a % kCqStages;
+        if (!mbar_wait(&empty[slot], ((a / kCqStages) & 1) ^ 1, status)) break;
+        uint8_t* st = smem + slot * SB;
+        mbar_arrive_expect_tx(&full[slot], SB);
+        tma_load_2d(st, &chi, &full[slot], a * 64, m0);
+        tma_load_2d(st + 16384, &clo, &full[slot], a * 64, m0);
+        for (int j = 0; j < bn / 64; ++j) {
+          tma_load_2d(st + 32768 + j * 8192, &qhi, &full[slot], n0 + 64 * j, a * 64);
+          tma_load_2d(st + 32768 + bn * 128 + j * 8192, &qlo, &full[slot], n0 + 64 * j, a * 64);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idesc = umma_idesc_bf16(128, bn, false, true);
+      for (int a = 0; a < nk; ++a) {
+        const int slot = a % kCqStages;
+        if (!mbar_wait(&full[slot], (a / kCqStages) & 1, status)) break;
+        tc_fence_after();
+        uint8_t* st = smem + slot * SB;
+        const uint64_t ah = umma_desc_sw128(smem_u32(st));
+        const uint64_t al = umma_desc_sw128(smem_u32(st + 16384));
+        const uint64_t bh = umma_desc_sw128_mn(smem_u32(st + 32768), 8192, 1024);
+        const uint64_t bl = umma_desc_sw128_mn(smem_u32(st + 32768 + bn * 128), 8192, 1024);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          umma_bf16(tmem, ah + 2 * kk, bh + 128 * kk, idesc, (a | kk) ? 1u : 0u);
+          umma_bf16(tmem, ah + 2 * kk, bl + 128 * kk, idesc, 1u);
+          umma_bf16(tmem, al + 2 * kk, bh + 128 * kk, idesc, 1u);
+        }
+        umma_commit(&empty[slot]);
+      }
+      umma_commit(&accbar[0]);
+    }
+  } else {
+    const int lq = warp & 3;
+    const int m = m0 + lq * 32 + lane;
+    const bool ok = mbar_wait(&accbar[0], 0, status);
+    __syncwarp();  // converged for the warp-wide tcgen05.ld
+    tc_fence_after();
+    const uint32_t taddr = tmem + (static_cast<uint32_t>(lq * 32) << 16);
+    if (ok) {
+      for (int jb = 0; jb < bn / 16; ++jb) {
+        float v[16];
+        tmem_ld16(taddr + jb * 16, v);
+        tmem_ld_wait();
+        float4* yrow = reinterpret_cast<float4*>(Y + static_cast<int64_t>(m) * b + n0 + jb * 16);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) yrow[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+      }
+    }
+  }
+  // reconverge the role warps before the block-wide barrier (TMEM release)
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 128);
+  }
+}
+
+// x (f32) -> hi = bf16(x), lo = bf16(x - hi), same layout
+__global__ void split_hilo_kernel(const float* __restrict__ x, int64_t count, __nv_bfloat16* __restrict__ hi,
+                                  __nv_bfloat16* __restrict__ lo) {
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < count;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const float v = x[i];
+    const __nv_bfloat16 h = __float2bfloat16_rn(v);
+    hi[i] = h;
+    lo[i] = __float2bfloat16_rn(v - __bfloat162float(h));
+  }
+}
+
+bool cq_tc_ok(int n, int b) { return n % 128 == 0 && b % 64 == 0 && n >= 128 && !force_simt(); }
+
+// Y = C Q on tensor cores; chl / qhl: the bf16 hi/lo pairs of C (n x n, split
+// once per factorisation) and of Q (n x b, split here)
+xkv_status cq_launch(const __nv_bfloat16* chl, const float* Q, __nv_bfloat16* qhl, float* Y, int n, int b,
+                     cudaStream_t st) {
+  const int64_t nb = static_cast<int64_t>(n) * b;
+  split_hilo_kernel<<<512, 256, 0, st>>>(Q, nb, qhl, qhl + nb);
+  const int64_t nn = static_cast<int64_t>(n) * n;
+  CUtensorMap mh, ml, bh, bl;
+  {
+    const uint64_t dims[2] = {static_cast<uint64_t>(n), static_cast<uint64_t>(n)};
+    const uint64_t str[1] = {static_cast<uint64_t>(n) * 2};
+    const uint32_t box[2] = {64, 128};
+    if (!make_tmap(&mh, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, chl, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_tmap(&ml, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, chl + nn, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B))
+      return XKV_ERR_CUDA;
+  }
+  {
+    const uint64_t dims[2] = {static_cast<uint64_t>(b), static_cast<uint64_t>(n)};
+    const uint64_t str[1] = {static_cast<uint64_t>(b) * 2};
+    const uint32_t box[2] = {64, 64};
+    if (!make_tmap(&bh, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, qhl, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_tmap(&bl, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, qhl + nb, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B))
+      return XKV_ERR_CUDA;
+  }
+  const int bn = b % 128 == 0 ? 128 : 64;
+  const size_t smem = cq_smem(bn);
+  cudaFuncSetAttribute(cq_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  cq_tc_kernel<<<dim3(n / 128, b / bn), kCqThreads, smem, st>>>(mh, ml, bh, bl, n, b, bn, Y, device_status_ptr());
+  return XKV_OK;
+}
+
 // ---------------------------------------------------------- factorisation
 // Block width of the subspace iteration: b = min(rank + oversample, G d, rows).
 xkv_status factor_plan(int n, int64_t rows, int rank, int oversample, FactorPlan* p) {
@@ -516,6 +686,12 @@ xkv_status factor_plan(int n, int64_t rows, int rank, int oversample, FactorPlan
   p->off_Ur = take(static_cast<size_t>(b) * rank * 4);
   p->off_Vr = take(static_cast<size_t>(n) * rank * 4);
   p->off_jac = take(jacobi_workspace(static_cast<int>(b), 1));
+  p->off_dblk = take(cholqr_dblk_bytes(static_cast<int>(b)));
+  p->off_part = take(cholqr_part_bytes(n, static_cast<int>(b)));
+  // bf16 hi/lo pairs of C and of the block for the tensor-core C Q
+  const bool tc = cq_tc_ok(n, static_cast<int>(b));
+  p->off_chl = take(tc ? static_cast<size_t>(n) * n * 4 : 0);
+  p->off_qhl = take(tc ? static_cast<size_t>(n) * b * 4 : 0);
   p->bytes = off;
   return XKV_OK;
 }
@@ -539,21 +715,41 @@ xkv_status factor_launch(const FactorPlan& P, const float* C, xkv_dtype dt, int 
   float* Vr = reinterpret_cast<float*>(w + P.off_Vr);
   int* status = device_status_ptr();
   if (!status) return XKV_ERR_CUDA;
+  double* part = gemm_splits(b, b, n) > 1 ? reinterpret_cast<double*>(w + P.off_part) : nullptr;
+  const CholQRScratch cs{W, H, reinterpret_cast<double*>(w + P.off_dblk), part, scal};
+  const bool tc = cq_tc_ok(n, b);
+  __nv_bfloat16* chl = reinterpret_cast<__nv_bfloat16*>(w + P.off_chl);
+  __nv_bfloat16* qhl = reinterpret_cast<__nv_bfloat16*>(w + P.off_qhl);
+  if (tc) split_hilo_kernel<<<512, 256, 0, st>>>(C, static_cast<int64_t>(n) * n, chl, chl + static_cast<int64_t>(n) * n);
+  // Y = C Q: on tensor cores (bf16 hi/lo splits) while iterating, where only
+  // the span matters; in fp32 on CUDA cores for the Rayleigh-Ritz product, whose
+  // Ritz values (eigvals, and the energy they leave out) need the full fp32
+  // accuracy of C Q
+  auto apply_c = [&](bool exact) -> xkv_status {
+    if (tc && !exact) return cq_launch(chl, Q, qhl, Y, n, b, st);
+    gemm_simt<float, float, float, float>(C, n, 1, Q, b, 1, Y, b, n, b, n, 1.0, 0.0, st);
+    return XKV_OK;
+  };
   gaussian_kernel<<<256, 256, 0, st>>>(Y, static_cast<int64_t>(n) * b, seed);
-  auto orthonormalise = [&](float* src) {
-    // shifted pass (robust to a rank-deficient block), then a plain pass
-    cholqr_pass(src, Q, n, b, 1e-13, W, H, scal, status, st);
-    cholqr_pass(Q, src, n, b, 0.0, W, H, scal, status, st);
+  // Q <- an orthonormal basis of span(src).  The iterations only need a
+  // well-conditioned basis of the right span (the span is what converges), so
+  // they take one shifted CholQR pass (orthogonal to ~1e-7 in fp32); the basis
+  // that enters Rayleigh-Ritz takes a second, plain pass (CholQR2).
+  auto orthonormalise = [&](float* src, bool twice) {
+    cholqr_pass(src, Q, n, b, 1e-13, cs, status, st);
+    if (!twice) return;
+    cholqr_pass(Q, src, n, b, 0.0, cs, status, st);
     cudaMemcpyAsync(Q, src, static_cast<size_t>(n) * b * 4, cudaMemcpyDeviceToDevice, st);
   };
-  orthonormalise(Y);
+  orthonormalise(Y, iters == 0);
   for (int it = 0; it < iters; ++it) {
-    gemm_simt<float, float, float, float>(C, n, 1, Q, b, 1, Y, b, n, b, n, 1.0, 0.0, st);
-    orthonormalise(Y);
+    xkv_status s = apply_c(false);
+    if (s != XKV_OK) return s;
+    orthonormalise(Y, it == iters - 1);
   }
   // Rayleigh-Ritz
-  gemm_simt<float, float, float, float>(C, n, 1, Q, b, 1, Y, b, n, b, n, 1.0, 0.0, st);
-  gemm_simt<float, float, double, double>(Q, 1, b, Y, b, 1, H, b, b, b, n, 1.0, 0.0, st);
+  if (xkv_status s = apply_c(true); s != XKV_OK) return s;
+  gemm_simt_split<float, float, double, double>(Q, 1, b, Y, b, 1, H, b, b, b, n, 1.0, 0.0, part, false, st);
   xkv_status s = jacobi_launch(H, U, lam, b, 1, w + P.off_jac, st);
   if (s != XKV_OK) return s;
   order_desc(lam, b, order, st);
