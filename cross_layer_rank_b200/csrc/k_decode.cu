@@ -41,8 +41,8 @@ constexpr int kTileChunks = 16;   // chunks of 8 rows per 128-row tile (tcgen05 
 constexpr int kMaxGQ = 8;
 constexpr int kKStages = 3;   // key stages: 16 chunks x kKAtoms 64-column atoms
 constexpr int kKAtoms = 2;
-constexpr int kBStages = 2;   // Bt_K atoms (128 rows x 64 columns)
-constexpr int kVStages = 4;   // value stages: 2 chunks x full rank
+constexpr int kBStages = 3;   // Bt_K atoms (128 rows x 64 columns): one stage and the next one's first
+constexpr int kVStages = 3;   // value stages: 2 chunks x full rank
 constexpr int kAtomBytes = 16384;  // 128 rows x 64 bf16
 constexpr int kAttendThreads = 512;  // 16 warps: 8 key epilogue, 4 value epilogue, 2 TMA, 2 MMA
 

@@ -488,7 +488,7 @@ __device__ __forceinline__ int rr_player(int pos, int round, int nplayers) {
 __device__ void jacobi_pair(double* __restrict__ W, double* __restrict__ V, int n, int nblk, int round, int sweep,
                             JacobiState* __restrict__ state, double tol) {
   __shared__ double G[32][33];
-  __shared__ double R[32][33];
+  __shared__ __align__(16) double R[32][34];  // even row stride: 16-byte pairs R[e][c..c+1]
   __shared__ double tile[64][33];
   __shared__ double cs[16], sn[16];
   __shared__ int pp[16], qq[16];
@@ -505,12 +505,16 @@ __device__ void jacobi_pair(double* __restrict__ W, double* __restrict__ V, int 
     const int c = blk * kJB + (tid & 15);
     cols[tid] = c < n ? c : -1;
   }
-  // Gram of the 32 columns
-  for (int i = tid; i < 32 * 32; i += 256) G[i / 32][i % 32] = 0.0;
-  __syncthreads();
+  // Gram of the 32 columns: thread (kg, ti, tj) owns the 4 x 4 block
+  // G[4 ti .. 4 ti + 3][4 tj .. 4 tj + 3] over rows kg, kg + 4, ... of each
+  // 64-row pass; the four row groups' blocks are then added in a fixed order
   {
-    const int a = tid >> 3, bb = (tid & 7) * 4;  // thread owns G[a][bb..bb+3]
-    double acc[4] = {0, 0, 0, 0};
+    const int kg = tid >> 6, ti = (tid >> 3) & 7, tj = tid & 7;
+    double acc[4][4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) acc[i][j] = 0.0;
     for (int r0 = 0; r0 < n; r0 += 64) {  // 64 rows a pass: 8 loads in flight per thread
 #pragma unroll
       for (int q = 0; q < 8; ++q) {
@@ -521,15 +525,27 @@ __device__ void jacobi_pair(double* __restrict__ W, double* __restrict__ V, int 
       }
       __syncthreads();
 #pragma unroll 4
-      for (int r = 0; r < 64; ++r) {
-        const double x = tile[r][a];
+      for (int r = kg; r < 64; r += 4) {
+        double av[4], bv[4];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) acc[e] += x * tile[r][bb + e];
+        for (int i = 0; i < 4; ++i) av[i] = tile[r][4 * ti + i];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) bv[j] = tile[r][4 * tj + j];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) acc[i][j] += av[i] * bv[j];
       }
       __syncthreads();
     }
+    for (int g = 0; g < 4; ++g) {
+      if (kg == g)
 #pragma unroll
-    for (int e = 0; e < 4; ++e) G[a][bb + e] = acc[e];
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) G[4 * ti + i][4 * tj + j] = g == 0 ? acc[i][j] : G[4 * ti + i][4 * tj + j] + acc[i][j];
+      __syncthreads();
+    }
   }
   // the pair is converged when every fresh column product is tiny relative to
   // the column norms: |w_p . w_q| <= tol ||w_p|| ||w_q||
@@ -607,21 +623,39 @@ __device__ void jacobi_pair(double* __restrict__ W, double* __restrict__ V, int 
     if (!any) break;
   }
   if (tid == 0) atomicAdd(&stp->active[sweep], 1);
-  // Wc <- Wc R, Vc <- Vc R (row by row)
+  // Wc <- Wc R, Vc <- Vc R: each thread rotates two rows, r and r + 256, so
+  // every 16-byte pair R[e][c..c+1] read from shared memory serves four
+  // products (columns beyond n, cols[c] < 0, hold zeros and are not stored)
   for (int mat = 0; mat < (Vp ? 2 : 1); ++mat) {
     double* M = mat == 0 ? Wp : Vp;
-    for (int r0 = 0; r0 < n; r0 += 256) {
-      const int r = r0 + tid;
-      double x[32];
+    for (int r0 = 0; r0 < n; r0 += 512) {
+      const int ra = r0 + tid, rb = ra + 256;
+      double xa[32], xb[32];
 #pragma unroll
-      for (int c = 0; c < 32; ++c) x[c] = (cols[c] >= 0 && r < n) ? __ldcg(M + static_cast<int64_t>(cols[c]) * n + r) : 0.0;
-      if (r < n) {
-        for (int c = 0; c < 32; ++c) {
-          if (cols[c] < 0) continue;
-          double y = 0.0;
+      for (int c = 0; c < 32; ++c) {
+        const int64_t off = static_cast<int64_t>(cols[c]) * n;
+        xa[c] = (cols[c] >= 0 && ra < n) ? __ldcg(M + off + ra) : 0.0;
+        xb[c] = (cols[c] >= 0 && rb < n) ? __ldcg(M + off + rb) : 0.0;
+      }
+#pragma unroll 1
+      for (int c = 0; c < 32; c += 2) {
+        double ya0 = 0.0, ya1 = 0.0, yb0 = 0.0, yb1 = 0.0;
 #pragma unroll
-          for (int e = 0; e < 32; ++e) y += x[e] * R[e][c];
-          M[static_cast<int64_t>(cols[c]) * n + r] = y;
+        for (int e = 0; e < 32; ++e) {
+          const double2 rv = *reinterpret_cast<const double2*>(&R[e][c]);
+          ya0 = fma(xa[e], rv.x, ya0);
+          ya1 = fma(xa[e], rv.y, ya1);
+          yb0 = fma(xb[e], rv.x, yb0);
+          yb1 = fma(xb[e], rv.y, yb1);
+        }
+        const int c0 = cols[c], c1 = cols[c + 1];
+        if (ra < n) {
+          if (c0 >= 0) M[static_cast<int64_t>(c0) * n + ra] = ya0;
+          if (c1 >= 0) M[static_cast<int64_t>(c1) * n + ra] = ya1;
+        }
+        if (rb < n) {
+          if (c0 >= 0) M[static_cast<int64_t>(c0) * n + rb] = yb0;
+          if (c1 >= 0) M[static_cast<int64_t>(c1) * n + rb] = yb1;
         }
       }
     }
