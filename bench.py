@@ -284,6 +284,37 @@ def build_model(xkv, w, device, groups=None, log=print):
     return model, prefill
 
 
+def compress_profile(w):
+    """xkv_compress_group (r = rank_k, p = max(64, r/4), 8 iterations,
+    8192-row shards) and xkv_ner on its Gram for the (batch 0, group 0) keys;
+    the second call pair runs between cudaProfilerStart and cudaProfilerStop."""
+    import torch
+    import cross_layer_rank_b200 as xkv
+    device = torch.device("cuda", 0)
+    X = synth.kv_group_torch(w, 0, 0, "K", device)
+    r, G, d = w.rank_k, w.group, w.d
+    A = torch.empty((w.T, r), dtype=torch.bfloat16, device=device)
+    Bt = torch.empty((G * d, r), dtype=torch.bfloat16, device=device)
+    C = torch.empty((G * d, G * d), dtype=torch.float32, device=device)
+    ner = torch.empty(G, dtype=torch.float32, device=device)
+
+    def once():
+        xkv.xkv_compress_group(X, r, A, Bt, iters=8, oversample=synth.oversample(r), shard_rows=8192, gram_out=C)
+        xkv.xkv_ner(C, d, ner)
+
+    once()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.cudart().cudaProfilerStart()
+    e0.record()
+    once()
+    e1.record()
+    torch.cuda.synchronize()
+    torch.cuda.cudart().cudaProfilerStop()
+    assert xkv.get_device_status() == 0
+    return {"workload": w.name, "compress_and_ner_ms": round(e0.elapsed_time(e1), 3)}
+
+
 def measure_gram(xkv, w, device, spectra=True):
     """Device time of the Gram of one (batch 0, group 0) K shard set (T rows),
     of KV-CoRE's NER and energy rank on it (spectra=True) and of A = X V_r."""
@@ -860,6 +891,10 @@ def main():
     ap.add_argument("--prefill-only", action="store_true",
                     help="time only the compression kernels (Gram, projection, the compression sweep) and print "
                          "them; no decode step (a profiling aid)")
+    ap.add_argument("--compress-profile", action="store_true",
+                    help="one xkv_compress_group + xkv_ner on the workload's (batch 0, group 0) keys, run once "
+                         "untimed and once between cudaProfilerStart / Stop (for ncu --profile-from-start off); "
+                         "prints the second run's device time")
     args = ap.parse_args()
     rank = int(os.environ.get("RANK", 0))
     world = int(os.environ.get("WORLD_SIZE", 1))
@@ -868,6 +903,9 @@ def main():
     if args.impl == "reference":
         if rank == 0:
             print(json.dumps(run_reference(args, log)), flush=True)
+        return
+    if args.compress_profile:
+        print(json.dumps(compress_profile(synth.WORKLOADS[args.workload])), flush=True)
         return
     if args.prefill_only:
         import torch
