@@ -831,7 +831,8 @@ xkv_status project_launch(const void* const* X, int G, int64_t T, int d, int64_t
     g.status = status;
     const size_t smem = gemm_smem_bytes<kProj>();
     cudaFuncSetAttribute(gemm_tc_kernel<kProj>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-    dim3 grid(static_cast<unsigned>((T + 127) / 128), r / bn);
+    if ((T + 127) / 128 > 65535) return XKV_ERR_UNSUPPORTED;  // row tiles on grid.y
+    dim3 grid(r / bn, static_cast<unsigned>((T + 127) / 128));
     gemm_tc_kernel<kProj><<<grid, kGemmThreads, smem, st>>>(am, bh, bl, g);
   } else if (dt == XKV_F32 && v_dt == XKV_F32) {
     const float* Vf = static_cast<const float*>(V);

@@ -1,5 +1,5 @@
 // tcgen05 GEMM tile kernel: D[m][n] = sum_k A[m][k] B[n][k] for one 128 x BN
-// output tile per CTA, both operands K-major bf16 loaded by TMA with the
+// output tile per CTA (grid: column tiles x row tiles), both operands K-major bf16 loaded by TMA with the
 // 128-byte swizzle, fp32 accumulation in TMEM.  Warp 0 issues TMA, warp 1
 // issues tcgen05.mma, warps 2..5 drain TMEM through a mode-specific epilogue:
 //   kRecon : bf16 store of A Bt^T with optional RoPE per head (position = row)
@@ -64,7 +64,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint32_t* tslot = reinterpret_cast<uint32_t*>(accbar + 2);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int tm = blockIdx.x, tn = blockIdx.y;
+  // the column tiles of one row tile are neighbours in launch order, so the
+  // row tile's A operand is read from DRAM once and from L2 after
+  const int tn = blockIdx.x, tm = blockIdx.y;
   const int m0 = tm * 128, n0 = tn * g.bn;
   const int nk = g.K / 64;
 

@@ -464,7 +464,7 @@ void cholqr_pass(const float* Y, float* Q, int n, int b, double shift_rel, const
 // a sweep that rotates nothing ends the iteration.  On convergence column i of
 // W is lambda_i v_i, so |lambda_i| is its norm and v_i is column i of V.
 constexpr int kJB = 16;
-constexpr int kJacobiInnerSweeps = 2;
+constexpr int kJacobiInnerSweeps = 1;
 
 // Sweep limit: 40, or XKV_JACOBI_MAX_SWEEPS (a diagnostic override, e.g. 1 to
 // see the non-convergence report), at most kJacobiSweepCap.

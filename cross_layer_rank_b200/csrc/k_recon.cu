@@ -362,7 +362,8 @@ xkv_status recon_launch(const void* A, const void* Bt, int64_t T, int rank, int 
     g.status = device_status_ptr();
     const size_t smem = gemm_smem_bytes<kRecon>();
     cudaFuncSetAttribute(gemm_tc_kernel<kRecon>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-    dim3 grid(static_cast<unsigned>((T + 127) / 128), d / bn);
+    if ((T + 127) / 128 > 65535) return XKV_ERR_UNSUPPORTED;  // row tiles on grid.y
+    dim3 grid(d / bn, static_cast<unsigned>((T + 127) / 128));
     gemm_tc_kernel<kRecon><<<grid, kGemmThreads, smem, st>>>(am, bm, bm, g);
   } else {
     const int64_t pairs = T * (d / 2);
