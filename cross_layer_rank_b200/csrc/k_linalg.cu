@@ -505,6 +505,9 @@ __device__ void jacobi_pair(double* __restrict__ W, double* __restrict__ V, int 
     const int c = blk * kJB + (tid & 15);
     cols[tid] = c < n ? c : -1;
   }
+  // every thread reads the pair's column list (which the previous round of a
+  // persistent CTA left different) only after it is complete
+  __syncthreads();
   // Gram of the 32 columns: thread (kg, ti, tj) owns the 4 x 4 block
   // G[4 ti .. 4 ti + 3][4 tj .. 4 tj + 3] over rows kg, kg + 4, ... of each
   // 64-row pass; the four row groups' blocks are then added in a fixed order
