@@ -240,8 +240,9 @@ static xkv_status check_compress(int G, int64_t T, int d, int rank, int iters, i
   if (rank > G * d || rank > T) return XKV_ERR_INVALID_ARG;
   if (dt != XKV_F32 && dt != XKV_BF16) return XKV_ERR_INVALID_ARG;
   if (dt == XKV_BF16 && rank % 64 != 0) return XKV_ERR_UNSUPPORTED;
-  // block width of the subspace iteration: its Cholesky QR's triangular
-  // inverse holds 8 columns of b doubles in shared memory (<= 224 KiB)
+  // block width of the subspace iteration: the widest the factorisation is
+  // built for (the Rayleigh-Ritz Jacobi's b / 32 pair CTAs in one cooperative
+  // launch)
   const int64_t b = std::min<int64_t>(std::min<int64_t>(static_cast<int64_t>(rank) + oversample, int64_t(G) * d), T);
   if (b > 3584) return XKV_ERR_UNSUPPORTED;
   return XKV_OK;

@@ -113,8 +113,9 @@ XKV_API xkv_status xkv_gram_accumulate(const void* const* X_layers, int G, int64
  * Requires d % 64 == 0, rank % 16 == 0, 1 <= rank <= min(T, G d), iters >= 1
  * (XKV_ERR_INVALID_ARG otherwise); a bf16 group also needs rank % 64 == 0 (the
  * tensor-core projection), and the block width b may not exceed 3584 (the
- * triangular inverse of the Cholesky QR keeps 8 of its b-long columns in
- * shared memory), else XKV_ERR_UNSUPPORTED.  At most G = 8 layers. */
+ * widest block the factorisation is built for: the Rayleigh-Ritz Jacobi's
+ * b / 32 pair CTAs then still run as one cooperative launch), else
+ * XKV_ERR_UNSUPPORTED.  At most G = 8 layers. */
 XKV_API xkv_status xkv_compress_workspace_size(int G, int64_t T, int d, int rank, int oversample,
                                        int64_t shard_rows, xkv_dtype dt, size_t* bytes);
 XKV_API xkv_status xkv_compress_group(const void* const* X_layers, int G, int64_t T, int d, int64_t ldx,

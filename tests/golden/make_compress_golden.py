@@ -16,9 +16,12 @@ Cases (name: workload, tensor, rank):
                         the key case also stores KV-CoRE's NER and the 95 %
                         energy rank of each 1024-wide layer block.
 
-Usage: python tests/golden/make_compress_golden.py [case ...]
+Usage: python tests/golden/make_compress_golden.py [--spectrum] [case ...]
 Each finished case is merged into the JSON file at once, so an interrupted run
-keeps what it has.
+keeps what it has.  --spectrum adds, for a case whose rank exceeds the
+generator's latent dimension m (sweep_g8), the energy that the exact top-rank
+subspace keeps in the directions m .. rank - 1 (eigenvalues of the oracle's
+fp64 Gram), without recomputing the factorisation.
 """
 from __future__ import annotations
 
@@ -86,23 +89,50 @@ def run_case(name, w, kind, rank):
     return rec
 
 
+def spectrum_fields(w, kind, rank):
+    """For a rank past the generator's latent dimension m: the energy of the
+    eigen-directions m .. rank - 1 that the exact top-rank subspace keeps,
+    sum of those eigenvalues of the oracle's fp64 Gram (LAPACK eigvalsh as a
+    library step), and the eigenvalues around m."""
+    layers = synth.kv_group(w, 0, 0, kind)
+    Cm = oracle.gram(layers)
+    lam = np.linalg.eigvalsh(Cm)[::-1]
+    m = int(w.latent)
+    return dict(latent=m, energy_latent_to_rank=float(lam[m:rank].sum()),
+                lam_at_latent=[float(x) for x in lam[max(m - 4, 0):m + 4]])
+
+
+def save(name, fields, replace):
+    data = {}
+    if os.path.exists(OUT):
+        with open(OUT) as f:
+            data = json.load(f)
+    data[name] = fields if replace else {**data.get(name, {}), **fields}
+    tmp = OUT + ".tmp"
+    with open(tmp, "w") as f:
+        json.dump(data, f, indent=1, sort_keys=True)
+        f.write("\n")
+    os.replace(tmp, OUT)
+
+
 def main(argv):
-    todo = argv or ORDER
+    spectrum = "--spectrum" in argv
+    todo = [a for a in argv if not a.startswith("--")] or ORDER
     allc = cases()
     for name in todo:
         w, kind, rank = allc[name]
         print(f"[{time.strftime('%H:%M:%S')}] {name}: {w.name} {kind} r={rank}", flush=True)
+        if spectrum:
+            if rank <= w.latent:
+                print("  rank within the latent dimension: nothing to add", flush=True)
+                continue
+            fields = spectrum_fields(w, kind, rank)
+            save(name, fields, replace=False)
+            print(f"  done: energy of directions {fields['latent']} .. {rank - 1}: "
+                  f"{fields['energy_latent_to_rank']:.6g}", flush=True)
+            continue
         rec = run_case(name, w, kind, rank)
-        data = {}
-        if os.path.exists(OUT):
-            with open(OUT) as f:
-                data = json.load(f)
-        data[name] = rec
-        tmp = OUT + ".tmp"
-        with open(tmp, "w") as f:
-            json.dump(data, f, indent=1, sort_keys=True)
-            f.write("\n")
-        os.replace(tmp, OUT)
+        save(name, rec, replace=True)
         print(f"  done: sweeps {rec['sweeps']}, {rec['oracle_seconds']} s, err_sub {rec['err_subspace']:.6g}, "
               f"err_sto {rec['err_stored']:.6g}", flush=True)
 

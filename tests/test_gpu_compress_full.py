@@ -14,6 +14,11 @@ through their errors, never elementwise; Eckart-Young, KQ-SVD 3.3):
     fp64, within 1e-3 (relative) of the oracle's;
   * stored-factor error ||X - A Bt^T||_F of the GPU's bf16 factors within 1e-3
     of the oracle's own bf16-rounded stored-factor error;
+  * where r exceeds the generator's latent dimension m (the G = 8 sweep point,
+    r = 1024, m = 768), the directions past m are a noise floor below fp32
+    resolution: both squared errors may then exceed the oracle's by at most
+    the energy the exact subspace keeps in directions m .. r - 1 (stored by the
+    oracle script), and never fall below the oracle's subspace error;
   * xkv_compress_group gives the same bits as its pieces (Gram over shards,
     xkv_factor_gram, xkv_project);
   * for the Llama keys, KV-CoRE's NER of every 1024-wide layer block within
@@ -94,8 +99,25 @@ def test_compress_matches_oracle_at_full_size(xkv, name):
     sub = _fro64(Xd - (Xd @ V) @ V.T)
     sto = _fro64(Xd - A.double() @ Bt.double().T)
     del Xd
-    assert abs(sub - rec["err_subspace"]) <= 1e-3 * rec["err_subspace"], (sub, rec["err_subspace"])
-    assert abs(sto - rec["err_stored"]) <= 1e-3 * rec["err_stored"], (sto, rec["err_stored"])
+    if r <= w.latent:
+        assert abs(sub - rec["err_subspace"]) <= 1e-3 * rec["err_subspace"], (sub, rec["err_subspace"])
+        assert abs(sto - rec["err_stored"]) <= 1e-3 * rec["err_stored"], (sto, rec["err_stored"])
+    else:
+        # the rank reaches past the generator's latent dimension m into the flat
+        # noise floor, whose eigenvalues (about 6.7 here) lie below the fp32
+        # rounding of the largest (2.5e8 x 6e-8): there the fp32 Gram does not
+        # determine which noise directions are the top ones.  The basis must
+        # hold every direction above m (missing one costs thousands), and it
+        # may lose at most the energy the exact top-r subspace keeps past m
+        extra = rec["energy_latent_to_rank"] * (1 + 1e-3)
+        assert sub ** 2 <= rec["err_subspace"] ** 2 + extra, (sub, rec["err_subspace"], extra)
+        assert sto ** 2 <= rec["err_stored"] ** 2 + extra, (sto, rec["err_stored"], extra)
+        # every direction above m is held: the Ritz values at m - 4 .. m - 1 are
+        # the oracle's eigenvalues there (a missed one would leave a noise-level
+        # Ritz value, 55 times smaller, among them)
+        m = rec["latent"]
+        evm = ev.double().cpu().numpy()
+        assert np.allclose(evm[m - 4:m], rec["lam_at_latent"][:4], rtol=1e-3), (evm[m - 4:m + 4], rec["lam_at_latent"])
     # Eckart-Young: no rank-r basis beats the oracle's (up to its rounding)
     assert sub >= rec["err_subspace"] * (1 - 1e-6)
     # the leading Ritz values are the leading eigenvalues
