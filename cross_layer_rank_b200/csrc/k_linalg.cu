@@ -7,6 +7,7 @@
 //     semi-definite matrices: the Rayleigh-Ritz step (eigenvalues + vectors);
 //   - ordering of eigenvalues, and the NER and energy-rank reductions of
 //     KV-CoRE's spectra (2.B), whose eigenvalues come from k_spectrum.cu.
+#include <cooperative_groups.h>
 #include <stdlib.h>
 
 #include <algorithm>
@@ -485,9 +486,16 @@ __device__ __forceinline__ int rr_player(int pos, int round, int nplayers) {
 // One round for the pair of CTA blockIdx.x of problem blockIdx.y; rotations
 // are counted in state->active[sweep].  W and V are read through L2 (__ldcg):
 // in the persistent kernel other CTAs rewrote them since this SM last read.
+//
+// With nparts > 1 (a cluster of nparts CTAs per pair, cluster rank = part),
+// each CTA forms the Gram over its share of the rows and rotates only those
+// rows; the partial Grams are added through distributed shared memory in
+// rank order, so every CTA of the cluster holds the same Gram and computes
+// the same rotation.
 __device__ void jacobi_pair(double* __restrict__ W, double* __restrict__ V, int n, int nblk, int round, int sweep,
-                            JacobiState* __restrict__ state, double tol) {
-  __shared__ double G[32][33];
+                            JacobiState* __restrict__ state, double tol, int nparts) {
+  __shared__ double G[32][33];   // this CTA's Gram (its rows' share of it when nparts > 1)
+  __shared__ double Gt[32][33];  // the pair's Gram, summed over the cluster (nparts > 1)
   __shared__ __align__(16) double R[32][34];  // even row stride: 16-byte pairs R[e][c..c+1]
   __shared__ double tile[64][33];
   __shared__ double cs[16], sn[16];
@@ -496,7 +504,10 @@ __device__ void jacobi_pair(double* __restrict__ W, double* __restrict__ V, int 
   JacobiState* stp = state + prob;
   double* Wp = W + static_cast<int64_t>(prob) * n * n;
   double* Vp = V ? V + static_cast<int64_t>(prob) * n * n : nullptr;
-  const int pair = blockIdx.x;
+  const int pair = blockIdx.x / nparts, part = blockIdx.x % nparts;
+  // rows of this CTA: a multiple of 64 per part
+  const int rows_per = ((n + nparts - 1) / nparts + 63) / 64 * 64;
+  const int r_lo = min(n, part * rows_per), r_hi = min(n, r_lo + rows_per);
   const int I = rr_player(pair, round, nblk), J = rr_player(nblk - 1 - pair, round, nblk);
   const int tid = threadIdx.x;
   __shared__ int cols[32];
@@ -518,13 +529,13 @@ __device__ void jacobi_pair(double* __restrict__ W, double* __restrict__ V, int 
     for (int i = 0; i < 4; ++i)
 #pragma unroll
       for (int j = 0; j < 4; ++j) acc[i][j] = 0.0;
-    for (int r0 = 0; r0 < n; r0 += 64) {  // 64 rows a pass: 8 loads in flight per thread
+    for (int r0 = r_lo; r0 < r_hi; r0 += 64) {  // 64 rows a pass: 8 loads in flight per thread
 #pragma unroll
       for (int q = 0; q < 8; ++q) {
         const int i = tid + 256 * q;
         const int c = i >> 6, r = i & 63;
         const int cc = cols[c];
-        tile[r][c] = (cc >= 0 && r0 + r < n) ? __ldcg(Wp + static_cast<int64_t>(cc) * n + r0 + r) : 0.0;
+        tile[r][c] = (cc >= 0 && r0 + r < r_hi) ? __ldcg(Wp + static_cast<int64_t>(cc) * n + r0 + r) : 0.0;
       }
       __syncthreads();
 #pragma unroll 4
@@ -550,6 +561,21 @@ __device__ void jacobi_pair(double* __restrict__ W, double* __restrict__ V, int 
       __syncthreads();
     }
   }
+  double(*Gw)[33] = G;
+  if (nparts > 1) {
+    namespace cg = cooperative_groups;
+    cg::cluster_group cl = cg::this_cluster();
+    cl.sync();  // every part's Gram is complete
+    for (int i = tid; i < 32 * 32; i += 256) {
+      double v = 0.0;
+      for (int q = 0; q < nparts; ++q) v += cl.map_shared_rank(&G[0][0], q)[(i >> 5) * 33 + (i & 31)];
+      Gt[i >> 5][i & 31] = v;
+    }
+    // (the parts' G stay untouched until the next round, which starts after
+    // the grid barrier that every part reaches only after these reads)
+    Gw = Gt;
+    __syncthreads();
+  }
   // the pair is converged when every fresh column product is tiny relative to
   // the column norms: |w_p . w_q| <= tol ||w_p|| ||w_q||
   __shared__ int s_need;
@@ -557,7 +583,7 @@ __device__ void jacobi_pair(double* __restrict__ W, double* __restrict__ V, int 
   __syncthreads();
   for (int i = tid; i < 32 * 32; i += 256) {
     const int p = i / 32, q = i % 32;
-    if (p < q && fabs(G[p][q]) > tol * sqrt(fabs(G[p][p] * G[q][q])) && G[p][q] != 0.0) s_need = 1;
+    if (p < q && fabs(Gw[p][q]) > tol * sqrt(fabs(Gw[p][p] * Gw[q][q])) && Gw[p][q] != 0.0) s_need = 1;
   }
   for (int i = tid; i < 32 * 32; i += 256) R[i / 32][i % 32] = (i / 32 == i % 32) ? 1.0 : 0.0;
   __syncthreads();
@@ -577,7 +603,7 @@ __device__ void jacobi_pair(double* __restrict__ W, double* __restrict__ V, int 
         if (p > q) { const int t = p; p = q; q = t; }
         pp[tid] = p;
         qq[tid] = q;
-        const double gpq = G[p][q], gpp = G[p][p], gqq = G[q][q];
+        const double gpq = Gw[p][q], gpp = Gw[p][p], gqq = Gw[q][q];
         if (gpq * gpq > 1e-28 * fabs(gpp * gqq) && gpq != 0.0) {
           // t = tan(theta) of the rotation that zeroes gpq, from the difference
           // d = gqq - gpp without forming tau = d / (2 gpq):
@@ -602,9 +628,9 @@ __device__ void jacobi_pair(double* __restrict__ W, double* __restrict__ V, int 
         const int p = pp[k], q = qq[k];
         const double c = cs[k], s = sn[k];
         if (s == 0.0) continue;
-        const double gp = G[r][p], gq = G[r][q];
-        G[r][p] = c * gp - s * gq;
-        G[r][q] = s * gp + c * gq;
+        const double gp = Gw[r][p], gq = Gw[r][q];
+        Gw[r][p] = c * gp - s * gq;
+        Gw[r][q] = s * gp + c * gq;
         const double rp = R[r][p], rq = R[r][q];
         R[r][p] = c * rp - s * rq;
         R[r][q] = s * rp + c * rq;
@@ -615,9 +641,9 @@ __device__ void jacobi_pair(double* __restrict__ W, double* __restrict__ V, int 
         const int p = pp[k], q = qq[k];
         const double c = cs[k], s = sn[k];
         if (s == 0.0) continue;
-        const double gp = G[p][cidx], gq = G[q][cidx];
-        G[p][cidx] = c * gp - s * gq;
-        G[q][cidx] = s * gp + c * gq;
+        const double gp = Gw[p][cidx], gq = Gw[q][cidx];
+        Gw[p][cidx] = c * gp - s * gq;
+        Gw[q][cidx] = s * gp + c * gq;
       }
       __syncthreads();
     }
@@ -625,20 +651,20 @@ __device__ void jacobi_pair(double* __restrict__ W, double* __restrict__ V, int 
     __syncthreads();
     if (!any) break;
   }
-  if (tid == 0) atomicAdd(&stp->active[sweep], 1);
+  if (tid == 0 && part == 0) atomicAdd(&stp->active[sweep], 1);
   // Wc <- Wc R, Vc <- Vc R: each thread rotates two rows, r and r + 256, so
   // every 16-byte pair R[e][c..c+1] read from shared memory serves four
   // products (columns beyond n, cols[c] < 0, hold zeros and are not stored)
   for (int mat = 0; mat < (Vp ? 2 : 1); ++mat) {
     double* M = mat == 0 ? Wp : Vp;
-    for (int r0 = 0; r0 < n; r0 += 512) {
+    for (int r0 = r_lo; r0 < r_hi; r0 += 512) {
       const int ra = r0 + tid, rb = ra + 256;
       double xa[32], xb[32];
 #pragma unroll
       for (int c = 0; c < 32; ++c) {
         const int64_t off = static_cast<int64_t>(cols[c]) * n;
-        xa[c] = (cols[c] >= 0 && ra < n) ? __ldcg(M + off + ra) : 0.0;
-        xb[c] = (cols[c] >= 0 && rb < n) ? __ldcg(M + off + rb) : 0.0;
+        xa[c] = (cols[c] >= 0 && ra < r_hi) ? __ldcg(M + off + ra) : 0.0;
+        xb[c] = (cols[c] >= 0 && rb < r_hi) ? __ldcg(M + off + rb) : 0.0;
       }
 #pragma unroll 1
       for (int c = 0; c < 32; c += 2) {
@@ -652,11 +678,11 @@ __device__ void jacobi_pair(double* __restrict__ W, double* __restrict__ V, int 
           yb1 = fma(xb[e], rv.y, yb1);
         }
         const int c0 = cols[c], c1 = cols[c + 1];
-        if (ra < n) {
+        if (ra < r_hi) {
           if (c0 >= 0) M[static_cast<int64_t>(c0) * n + ra] = ya0;
           if (c1 >= 0) M[static_cast<int64_t>(c1) * n + ra] = ya1;
         }
-        if (rb < n) {
+        if (rb < r_hi) {
           if (c0 >= 0) M[static_cast<int64_t>(c0) * n + rb] = yb0;
           if (c1 >= 0) M[static_cast<int64_t>(c1) * n + rb] = yb1;
         }
@@ -671,7 +697,7 @@ __global__ void __launch_bounds__(256) jacobi_round_kernel(double* __restrict__ 
                                                            int nblk, int round, int sweep,
                                                            JacobiState* __restrict__ state, double tol) {
   if (state[blockIdx.y].converged) return;
-  jacobi_pair(W, V, n, nblk, round, sweep, state, tol);
+  jacobi_pair(W, V, n, nblk, round, sweep, state, tol, 1);
 }
 
 __global__ void jacobi_sweep_end_kernel(JacobiState* state, int count, int sweep) {
@@ -687,13 +713,13 @@ __global__ void jacobi_sweep_end_kernel(JacobiState* state, int count, int sweep
 // timeout) ends the problem unconverged.
 __global__ void __launch_bounds__(256) jacobi_sweeps_kernel(double* __restrict__ W, double* __restrict__ V, int n,
                                                             int nblk, int max_sweeps, JacobiState* __restrict__ state,
-                                                            double tol, int* status) {
+                                                            double tol, int* status, int nparts) {
   JacobiState* stp = state + blockIdx.y;
-  const unsigned npairs = gridDim.x;
+  const unsigned nctas = gridDim.x;  // nparts CTAs (one cluster) per pair
   for (int sweep = 0; sweep < max_sweeps; ++sweep) {
     for (int round = 0; round < nblk - 1; ++round) {
-      jacobi_pair(W, V, n, nblk, round, sweep, state, tol);
-      if (!group_barrier(&stp->bar, npairs, status)) return;
+      jacobi_pair(W, V, n, nblk, round, sweep, state, tol, nparts);
+      if (!group_barrier(&stp->bar, nctas, status)) return;
     }
     if (*reinterpret_cast<volatile int*>(&stp->active[sweep]) == 0) {
       if (blockIdx.x == 0 && threadIdx.x == 0) stp->converged = 1;
@@ -757,13 +783,48 @@ xkv_status jacobi_launch(double* W, double* V, double* lam, int n, int count, vo
   jacobi_init_kernel<<<256, 256, 0, st>>>(V, n, count, state);
   int max_sweeps = jacobi_max_sweeps();
   double tol = 1e-11;
-  // one cooperative launch when every pair of every problem can be resident
+  // One cooperative launch when every pair of every problem can be resident:
+  // with clusters of 4 (else 2) CTAs per pair when that many clusters fit,
+  // else one CTA per pair.
+  const int npairs = nblk / 2;
+  bool launched = false;
+  for (int nparts : {4, 2}) {
+    if (count > 65535 || n < 64 * nparts) continue;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(npairs * nparts, count);
+    cfg.blockDim = dim3(256);
+    cfg.stream = st;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = nparts;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeCooperative;
+    attr[1].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;  // the occupancy query takes the cluster shape only
+    int nclusters = 0;
+    if (cudaOccupancyMaxActiveClusters(&nclusters, jacobi_sweeps_kernel, &cfg) != cudaSuccess) {
+      (void)cudaGetLastError();
+      continue;
+    }
+    if (static_cast<int64_t>(nclusters) < static_cast<int64_t>(npairs) * count) continue;
+    cfg.numAttrs = 2;
+    if (cudaLaunchKernelEx(&cfg, jacobi_sweeps_kernel, W, V, n, nblk, max_sweeps, state, tol, status, nparts) ==
+        cudaSuccess) {
+      launched = true;
+      break;
+    }
+    (void)cudaGetLastError();
+  }
   int per_sm = 0;
   cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, jacobi_sweeps_kernel, 256, 0);
-  const int64_t ctas = static_cast<int64_t>(nblk / 2) * count;
-  if (per_sm > 0 && ctas <= static_cast<int64_t>(per_sm) * num_sms() && count <= 65535) {
-    void* args[] = {&W, &V, &n, &nblk, &max_sweeps, &state, &tol, &status};
-    if (cudaLaunchCooperativeKernel(reinterpret_cast<void*>(jacobi_sweeps_kernel), dim3(nblk / 2, count), dim3(256),
+  const int64_t ctas = static_cast<int64_t>(npairs) * count;
+  if (launched) {
+  } else if (per_sm > 0 && ctas <= static_cast<int64_t>(per_sm) * num_sms() && count <= 65535) {
+    int one = 1;
+    void* args[] = {&W, &V, &n, &nblk, &max_sweeps, &state, &tol, &status, &one};
+    if (cudaLaunchCooperativeKernel(reinterpret_cast<void*>(jacobi_sweeps_kernel), dim3(npairs, count), dim3(256),
                                     args, 0, st) != cudaSuccess)
       return XKV_ERR_CUDA;
   } else {
