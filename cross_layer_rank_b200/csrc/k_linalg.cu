@@ -1,10 +1,12 @@
 // Small dense linear algebra of the factorisation path, on CUDA cores:
-//   - a strided SIMT GEMM (fp32 or fp64 accumulation) for the subspace
-//     iteration products and the f32 fall-backs;
+//   - a strided SIMT GEMM (fp32 or fp64 accumulation, optionally split along
+//     K with the slices summed in a fixed order) for the Rayleigh-Ritz and
+//     Cholesky-QR products and the f32 fall-backs;
 //   - shifted Cholesky QR pieces (Gram of a tall block, Cholesky, triangular
 //     inverse) in fp64;
 //   - a one-sided block Jacobi eigen-solver (fp64) for symmetric positive
-//     semi-definite matrices: the Rayleigh-Ritz step (eigenvalues + vectors);
+//     semi-definite matrices: the Rayleigh-Ritz step (eigenvalues + vectors),
+//     all sweeps in one cooperative launch of CTA clusters;
 //   - ordering of eigenvalues, and the NER and energy-rank reductions of
 //     KV-CoRE's spectra (2.B), whose eigenvalues come from k_spectrum.cu.
 #include <cooperative_groups.h>
@@ -716,6 +718,14 @@ __global__ void __launch_bounds__(256) jacobi_sweeps_kernel(double* __restrict__
                                                             double tol, int* status, int nparts) {
   JacobiState* stp = state + blockIdx.y;
   const unsigned nctas = gridDim.x;  // nparts CTAs (one cluster) per pair
+  // the partial Grams are read from the cluster's other CTAs: a launch whose
+  // cluster shape is not the one asked for (e.g. under a tool that drops the
+  // attribute) touches no distributed shared memory; the problem stays
+  // unconverged and is reported as such
+  if (nparts > 1 && cooperative_groups::this_cluster().num_blocks() != static_cast<unsigned>(nparts)) {
+    if (threadIdx.x == 0) record_status(status, kDevNumerical);
+    return;
+  }
   for (int sweep = 0; sweep < max_sweeps; ++sweep) {
     for (int round = 0; round < nblk - 1; ++round) {
       jacobi_pair(W, V, n, nblk, round, sweep, state, tol, nparts);
