@@ -239,12 +239,17 @@ __global__ void __launch_bounds__(256) chol_diag_kernel(double* __restrict__ W, 
     }
     __syncthreads();
   }
+  // 1 / L_jj = 1 / sqrt(d_j), once per column (1 for a replaced pivot, whose
+  // column below the diagonal is zeroed)
+  __shared__ double rl[kCholNB];
+  if (tid < nb) rl[tid] = dg[tid] > 0.0 ? rsqrt(dg[tid]) : 1.0;
+  __syncthreads();
   for (int e = tid; e < nb * nb; e += blockDim.x) {
     const int i = e / nb, j = e % nb;
     if (j > i) continue;
     const double d = dg[j];
     if (j == i) a[i][i] = d > 0.0 ? sqrt(d) : 1.0;
-    else a[i][j] = d > 0.0 ? a[i][j] / sqrt(d) : 0.0;
+    else a[i][j] = d > 0.0 ? a[i][j] * rl[j] : 0.0;
   }
   __syncthreads();
   {
@@ -255,7 +260,7 @@ __global__ void __launch_bounds__(256) chol_diag_kernel(double* __restrict__ W, 
         for (int k = c + q; k < i; k += 4) sm += a[i][k] * x[k][c];
       sm += __shfl_xor_sync(0xffffffffu, sm, 1);
       sm += __shfl_xor_sync(0xffffffffu, sm, 2);
-      if (q == 0 && c < nb) x[i][c] = c > i ? 0.0 : ((c == i ? 1.0 : 0.0) - sm) / a[i][i];
+      if (q == 0 && c < nb) x[i][c] = c > i ? 0.0 : ((c == i ? 1.0 : 0.0) - sm) * rl[i];
       __syncthreads();
     }
   }
