@@ -1,6 +1,7 @@
 // Shared device helpers of the xKV sm_100a library: element conversion, RoPE
 // angles, bounded waits, and thin inline-PTX wrappers for mbarriers, TMA
-// (cp.async.bulk.tensor, no multicast) and the 5th-generation tensor cores
+// (cp.async.bulk.tensor, each copy into the issuing CTA only) and the
+// 5th-generation tensor cores
 // (tcgen05.mma with TMEM accumulators).
 #pragma once
 
