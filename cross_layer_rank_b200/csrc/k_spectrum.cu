@@ -5,7 +5,7 @@
 //      belongs to CTA i mod cpp for the whole reduction) and meet at two
 //      bounded grid-group barriers per column;
 //   2. bisection on Sturm counts of the tridiagonal matrix, one thread per
-//      eigenvalue.
+//      eigenvalue, down to 1e-15 of the spectrum's span.
 // Householder step for column k (x = A[k+1:, k], m = n - k - 1 entries):
 //   alpha = -sign(x_0) ||x||, v = x - alpha e_1, beta = 2 / v^T v,
 //   p = beta A22 v, K = beta p^T v / 2, w = p - K v, A22 -= v w^T + w v^T,
@@ -160,11 +160,15 @@ __global__ void __launch_bounds__(256) bisect_kernel(const double* __restrict__ 
     s_piv = DBL_MIN * fmax(1.0, emax);
   }
   __syncthreads();
+  // stop once the bracket is below 1e-15 of the Gershgorin span (plus a few
+  // ulps of the value): the eigenvalues are then as accurate as the fp64
+  // reduction that produced the tridiagonal
+  const double tol = 1e-15 * (s_hi - s_lo);
   for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) {
     double lo = s_lo, hi = s_hi;
     for (int it = 0; it < 80; ++it) {
       const double mid = 0.5 * (lo + hi);
-      if (mid <= lo || mid >= hi) break;
+      if (mid <= lo || mid >= hi || hi - lo <= tol + 4.0 * DBL_EPSILON * fabs(mid)) break;
       if (sturm_count(ds, e2, n, mid, s_piv) > i) hi = mid;
       else lo = mid;
     }
