@@ -632,7 +632,7 @@ constexpr int kVAccCol = 256;  // TMEM columns of the value accumulators (2 x 64
 //      sums are reduce-scattered so each lane stores one).  With uncompressed
 //      values (xK-SR) U_g is already o_g's value sum and E is a scaled copy.
 constexpr int kCombineSplit = 4;
-constexpr int kCombineThreads = 256;
+constexpr int kCombineThreads = 512;
 constexpr int kMaxSlots = 64;
 constexpr int kCombineColsPerWarp = 4;
 constexpr int kCombineStageBytes = 64 * 1024;  // Bt_V rows staged for E, when they fit
@@ -1314,7 +1314,7 @@ __global__ void __launch_bounds__(kAttendThreads, 1)
 size_t attend_tc_smem() { return 1024 + kSmemEnd; }
 
 // ----------------------------------------------------------- sr_combine
-// Grid (unit, column split of kCombineSplit), 256 threads.
+// Grid (unit, column split of kCombineSplit), 512 threads.
 template <typename T>
 __global__ void __launch_bounds__(kCombineThreads) sr_combine_kernel(const T* __restrict__ BtV,
                                                                      const float* __restrict__ win,
